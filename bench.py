@@ -1,0 +1,596 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 / MXFP8 hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass over every row of the hot path, each on its workload
+(seeded synthetic inputs, resident in HBM before timing):
+
+  quant1g   a1-a4   amax + NVFP4 quantize (SWIZZLED scales) of bf16 [32768,16384]
+  gemv      a1,a6-a7  amax(x) + qmv: x [1,4096] bf16, W [14336,4096] pre-quantized
+  dequant   a5      NVFP4 dequantize of W [14336,4096] to bf16
+  prefill   a1-a4,a8-a9  qqmm op: amax x2, quantize x2 (SWIZZLED), FP4 GEMM 4096^3 -> bf16
+  moe       a10     gather_qmm: 64 experts [1408,2048], 4096 tokens, top-8 -> bf16
+  mxfp8     a11-a12 mxfp8 quantize x2 + FP8 GEMM 8192^3 -> bf16
+
+The headline ``value`` is the prefill qqmm op in TFLOP/s (2*M*N*K over the
+whole op: amaxes, quantizes and GEMM); every row's own metric, time and
+roofline are under ``rows``.  L2 (126 MB) is flushed before every row by
+writing a 256 MiB buffer, outside the row's timed window.  Kernel times are
+CUDA events on the launching stream.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs the same step on
+its own GPU (independent problems, no data-path collective): weak scaling;
+the reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [v.strip() for v in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# rows of the hot path
+# ---------------------------------------------------------------------------
+class Row:
+    name = ""
+    launches = 0  # our kernels per run
+
+    def __init__(self, nv, wl, dev, seed_offset):
+        self.nv, self.wl, self.dev, self.off = nv, wl, dev, seed_offset
+        self.timers = []  # (label, start_event, end_event) recorded by run()
+
+    def timed(self, label, fn):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        out = fn()
+        e.record()
+        self.timers.append((label, s, e))
+        return out
+
+
+def _gen(wl, name, dev, off):
+    d = wl.make(name, device=dev)
+    return d
+
+
+class Quant1G(Row):
+    name, launches = "quant1g", 2
+
+    def setup(self):
+        self.x = self.wl.make("quant1g", device=self.dev)["x"]
+        R, K = self.x.shape
+        self.g = torch.empty(1, dtype=torch.float32, device=self.dev)
+        self.codes = torch.empty(R, K // 8, dtype=torch.int32, device=self.dev)
+        self.scales = torch.empty(self.nv.scale_shape(R, K // 16, "swizzled"), dtype=torch.uint8, device=self.dev)
+        self.units = R * K
+        # algorithmic bytes of the quantize kernel: read x, write codes + scales
+        self.bytes_q = R * K * 2 + R * K // 2 + self.scales.numel()
+
+    def run(self):
+        self.timed("amax", lambda: self.nv.amax(self.x, self.g))
+        self.timed("quantize", lambda: self.nv.nvfp4_quantize(self.x, self.g, "swizzled", self.codes, self.scales))
+
+    def report(self, ms, peaks):
+        q = ms["quantize"]
+        return {"metric": "nvfp4 quantize GB/s", "unit": "GB/s", "value": self.bytes_q / q / 1e6,
+                "ms": ms, "roofline": {"bound": "hbm", "kernel": "k_nvfp4_quantize", "achieved": self.bytes_q / q / 1e6,
+                                       "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                       "frac": self.bytes_q / q / 1e6 / peaks["hbm_gbs"],
+                                       "frac_of_8tbs": self.bytes_q / q / 1e6 / 8000.0,
+                                       "algorithmic_bytes": self.bytes_q}}
+
+
+class Gemv(Row):
+    name, launches = "gemv", 2
+
+    def setup(self):
+        d = self.wl.make("gemv", device=self.dev)
+        self.x, w = d["x"], d["w"]
+        self.g_x = torch.empty(1, dtype=torch.float32, device=self.dev)
+        self.g_w = self.nv.amax(w)
+        self.wc, self.ws = self.nv.nvfp4_quantize(w, self.g_w, "linear")
+        del w
+        self.N, self.K = self.wc.shape[0], self.x.shape[1]
+        self.y = torch.empty(1, self.N, dtype=torch.bfloat16, device=self.dev)
+        self.bytes = self.wc.numel() * 4 + self.ws.numel() + self.x.numel() * 2 + self.y.numel() * 2
+
+    def run(self):
+        self.timed("amax", lambda: self.nv.amax(self.x, self.g_x))
+        self.timed("qmv", lambda: self.nv.qmv(self.x, self.wc, self.ws, self.g_x, self.g_w, self.y))
+
+    def report(self, ms, peaks):
+        q = ms["qmv"]
+        gbs = self.bytes / q / 1e6
+        return {"metric": "qmv GB/s", "unit": "GB/s", "value": gbs, "ms": ms,
+                "roofline": {"bound": "hbm", "kernel": "k_qmv", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "frac_of_8tbs": gbs / 8000.0,
+                             "algorithmic_bytes": self.bytes}}
+
+
+class Dequant(Row):
+    name, launches = "dequant", 1
+
+    def setup(self):
+        w = self.wl.make("gemv", device=self.dev)["w"]
+        g = self.nv.amax(w)
+        self.g = g
+        self.wc, self.ws = self.nv.nvfp4_quantize(w, g, "linear")
+        self.out = torch.empty_like(w)
+        self.bytes = self.wc.numel() * 4 + self.ws.numel() + w.numel() * 2
+        del w
+
+    def run(self):
+        self.timed("dequantize", lambda: self.nv.nvfp4_dequantize(self.wc, self.ws, self.g, "linear",
+                                                                  torch.bfloat16, out=self.out))
+
+    def report(self, ms, peaks):
+        q = ms["dequantize"]
+        gbs = self.bytes / q / 1e6
+        return {"metric": "nvfp4 dequantize GB/s", "unit": "GB/s", "value": gbs, "ms": ms,
+                "roofline": {"bound": "hbm", "kernel": "k_nvfp4_dequantize", "achieved": gbs,
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                             "algorithmic_bytes": self.bytes}}
+
+
+class Prefill(Row):
+    name, launches = "prefill", 5
+
+    def setup(self):
+        d = self.wl.make("prefill", device=self.dev)
+        self.x, self.w = d["x"], d["w"]
+        self.M, self.K = self.x.shape
+        self.N = self.w.shape[0]
+        self.g_x = torch.empty(1, dtype=torch.float32, device=self.dev)
+        self.g_w = torch.empty(1, dtype=torch.float32, device=self.dev)
+        mk = lambda r: (torch.empty(r, self.K // 8, dtype=torch.int32, device=self.dev),
+                        torch.empty(self.nv.scale_shape(r, self.K // 16, "swizzled"), dtype=torch.uint8,
+                                    device=self.dev))
+        self.xc, self.xs = mk(self.M)
+        self.wc, self.ws = mk(self.N)
+        self.y = torch.empty(self.M, self.N, dtype=torch.bfloat16, device=self.dev)
+        self.flop = 2 * self.M * self.N * self.K
+        # probe: raises if the GEMM kernel is not available
+        self.nv.nvfp4_quantize(self.x[:128], None, "swizzled")
+        self.nv.qqmm(self.xc[:128], self.xs[:128], self.wc[:128], self.ws[:128], self.K, "nvfp4",
+                     out=self.y[:128, :128].contiguous())
+
+    def op(self):
+        self.timed("amax_x", lambda: self.nv.amax(self.x, self.g_x))
+        self.timed("amax_w", lambda: self.nv.amax(self.w, self.g_w))
+        self.timed("quantize_x", lambda: self.nv.nvfp4_quantize(self.x, self.g_x, "swizzled", self.xc, self.xs))
+        self.timed("quantize_w", lambda: self.nv.nvfp4_quantize(self.w, self.g_w, "swizzled", self.wc, self.ws))
+        self.timed("gemm", lambda: self.nv.qqmm(self.xc, self.xs, self.wc, self.ws, self.K, "nvfp4",
+                                                self.g_x, self.g_w, out=self.y))
+
+    def run(self):
+        self.op()
+
+    def report(self, ms, peaks):
+        total = sum(ms.values())
+        fp4_peak = peaks["bf16_tflops"] * 4.0  # nominal dense fp4 : bf16 = 9 : 2.25
+        tf = self.flop / ms["gemm"] / 1e9
+        return {"metric": "qqmm FP4 TFLOP/s", "unit": "TFLOP/s", "value": self.flop / total / 1e9, "ms": ms,
+                "roofline": {"bound": "tensor", "kernel": "qqmm_sm100 (nvfp4)", "achieved": tf, "peak": fp4_peak,
+                             "unit": "TFLOP/s", "frac": tf / fp4_peak, "algorithmic_flop": self.flop,
+                             "peak_note": "measured bf16 burst x 4 (nominal fp4:bf16 ratio)"}}
+
+
+class Moe(Row):
+    name, launches = "moe", 3
+
+    def setup(self):
+        d = self.wl.make("moe", device=self.dev)
+        self.x, w, self.idx = d["x"], d["w"], d["idx"]
+        E, N, K = w.shape
+        self.E, self.N, self.K = E, N, K
+        self.g = torch.stack([self.nv.amax(w[e]) for e in range(E)]).view(E)
+        wc, ws = [], []
+        for e in range(E):
+            c, s = self.nv.nvfp4_quantize(w[e], self.g[e:e + 1], "linear")
+            wc.append(c)
+            ws.append(s)
+        self.wc, self.ws = torch.stack(wc), torch.stack(ws)
+        del w, wc, ws
+        T, topk = self.idx.shape
+        self.T, self.topk = T, topk
+        self.ws_buf = torch.empty(self.nv.gather_qmm_workspace_size(T, topk, E), dtype=torch.uint8, device=self.dev)
+        self.y = torch.empty(T, topk, N, dtype=torch.bfloat16, device=self.dev)
+        self.flop = 2 * T * topk * N * K
+        self.bytes = self.wc.numel() * 4 + self.ws.numel() + self.x.numel() * 2 + self.y.numel() * 2 + self.idx.numel() * 4
+        self.nv.gather_qmm(self.x[:16], self.wc, self.ws, self.g, self.idx[:16].contiguous())
+
+    def run(self):
+        self.timed("gather_qmm", lambda: self.nv.gather_qmm(self.x, self.wc, self.ws, self.g, self.idx,
+                                                            self.ws_buf, self.y))
+
+    def report(self, ms, peaks):
+        t = ms["gather_qmm"]
+        tf = self.flop / t / 1e9
+        return {"metric": "gather_qmm TFLOP/s", "unit": "TFLOP/s", "value": tf, "ms": ms,
+                "gbs": self.bytes / t / 1e6,
+                "roofline": {"bound": "tensor", "kernel": "gather_qmm", "achieved": tf, "peak": peaks["bf16_tflops"],
+                             "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"], "algorithmic_flop": self.flop,
+                             "hbm_frac": self.bytes / t / 1e6 / peaks["hbm_gbs"], "algorithmic_bytes": self.bytes}}
+
+
+class Mxfp8(Row):
+    name, launches = "mxfp8", 3
+
+    def setup(self):
+        d = self.wl.make("mxfp8", device=self.dev)
+        self.x, self.w = d["x"], d["w"]
+        self.M, self.K = self.x.shape
+        self.N = self.w.shape[0]
+        mk = lambda r: (torch.empty(r, self.K // 4, dtype=torch.int32, device=self.dev),
+                        torch.empty(self.nv.scale_shape(r, self.K // 32, "swizzled"), dtype=torch.uint8,
+                                    device=self.dev))
+        self.xc, self.xs = mk(self.M)
+        self.wc, self.ws = mk(self.N)
+        self.y = torch.empty(self.M, self.N, dtype=torch.bfloat16, device=self.dev)
+        self.flop = 2 * self.M * self.N * self.K
+        self.nv.qqmm(self.xc[:128], self.xs[:128], self.wc[:128], self.ws[:128], self.K, "mxfp8",
+                     out=self.y[:128, :128].contiguous())
+
+    def run(self):
+        self.timed("quantize_x", lambda: self.nv.mxfp8_quantize(self.x, "swizzled", self.xc, self.xs))
+        self.timed("quantize_w", lambda: self.nv.mxfp8_quantize(self.w, "swizzled", self.wc, self.ws))
+        self.timed("gemm", lambda: self.nv.qqmm(self.xc, self.xs, self.wc, self.ws, self.K, "mxfp8", out=self.y))
+
+    def report(self, ms, peaks):
+        fp8_peak = peaks["bf16_tflops"] * 2.0
+        tf = self.flop / ms["gemm"] / 1e9
+        return {"metric": "mxfp8 qqmm TFLOP/s", "unit": "TFLOP/s", "value": self.flop / sum(ms.values()) / 1e9,
+                "ms": ms, "roofline": {"bound": "tensor", "kernel": "qqmm_sm100 (mxfp8)", "achieved": tf,
+                                       "peak": fp8_peak, "unit": "TFLOP/s", "frac": tf / fp8_peak,
+                                       "peak_note": "measured bf16 burst x 2 (nominal fp8:bf16 ratio)"}}
+
+
+ROWS = [Quant1G, Gemv, Dequant, Prefill, Moe, Mxfp8]
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(world, v):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def e2e_prefill(nv, row, steps):
+    """The headline metric end to end through the public API with HOST
+    buffers: pinned bf16 x and W copied in, the qqmm op, y copied out."""
+    xh = row.x.cpu().pin_memory()
+    wh = row.w.cpu().pin_memory()
+    yh = torch.empty(row.M, row.N, dtype=torch.bfloat16).pin_memory()
+    xd, wd = torch.empty_like(row.x), torch.empty_like(row.w)
+
+    def once():
+        xd.copy_(xh, non_blocking=True)
+        wd.copy_(wh, non_blocking=True)
+        g_x, g_w = nv.amax(xd), nv.amax(wd)
+        xc, xs = nv.nvfp4_quantize(xd, g_x, "swizzled", row.xc, row.xs)
+        wc, ws = nv.nvfp4_quantize(wd, g_w, "swizzled", row.wc, row.ws)
+        nv.qqmm(xc, xs, wc, ws, row.K, "nvfp4", g_x, g_w, out=row.y)
+        yh.copy_(row.y, non_blocking=True)
+
+    for _ in range(2):
+        once()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        once()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    return {"ms": ms, "work": row.flop / 1e9, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": xh.numel() * 2 + wh.numel() * 2, "d2h_bytes_per_step": yh.numel() * 2}
+
+
+def e2e_gemv(nv, row, steps):
+    xh = row.x.cpu().pin_memory()
+    yh = torch.empty(1, row.N, dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(row.x)
+
+    def once():
+        xd.copy_(xh, non_blocking=True)
+        g = nv.amax(xd, row.g_x)
+        nv.qmv(xd, row.wc, row.ws, g, row.g_w, row.y)
+        yh.copy_(row.y, non_blocking=True)
+
+    for _ in range(3):
+        once()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        once()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    return {"ms": ms, "work": row.bytes / 1e6, "unit": "GB/s", "h2d_bytes_per_step": xh.numel() * 2,
+            "d2h_bytes_per_step": yh.numel() * 2}
+
+
+def cpu_baseline_prefill(sample_rows=16):
+    """The oracle as it stands on a bounded sample of the prefill qqmm op:
+    amax of x and W, quantize of `sample_rows` rows of x and all of W, exact
+    decode, float64 matmul.  Reported in TFLOP/s of the sampled outputs."""
+    from mxfp8_block_scaled_nvfp4_b200 import workloads
+    from oracle import oracle as orc
+    orc.build()
+    d = workloads.make("prefill", device="cpu")
+    x = d["x"][:sample_rows].contiguous().view(torch.int16).numpy().view(np.uint16)
+    wfull = d["w"].contiguous().view(torch.int16).numpy().view(np.uint16)
+    xfull = d["x"].contiguous().view(torch.int16).numpy().view(np.uint16)
+    t0 = time.perf_counter()
+    gx, gw = orc.amax(xfull, "bf16"), orc.amax(wfull, "bf16")
+    xq, xs = orc.nvfp4_quantize(x, "bf16", gx)
+    wq, ws = orc.nvfp4_quantize(wfull, "bf16", gw)
+    orc.qqmm(xq, xs, wq, ws, "nvfp4", gx, gw, "bf16")
+    dt = time.perf_counter() - t0
+    flop = 2 * sample_rows * wfull.shape[0] * wfull.shape[1]
+    threads = 1
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([1] + [i.get("num_threads", 1) for i in threadpool_info()])
+    except Exception:
+        pass
+    return {"value": flop / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "seconds": dt,
+            "sample": f"prefill qqmm op on {sample_rows} of 4096 rows of x (full W quantized, full amaxes); "
+                      f"element steps single-threaded C, contraction numpy float64 ({threads} BLAS threads)"}
+
+
+def run_ours(args):
+    world, rank, local = dist_setup(args.gpus)
+    from mxfp8_block_scaled_nvfp4_b200 import build, nvfp4 as nv, workloads as wl
+    if rank == 0:
+        build.build()
+    barrier(world)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    rows, unavailable = [], {}
+    for cls in ROWS:
+        if args.rows and cls.name not in args.rows:
+            continue
+        r = cls(nv, wl, dev, rank)
+        try:
+            r.setup()
+            torch.cuda.synchronize()
+            rows.append(r)
+        except nv.Nvfp4Error as e:
+            unavailable[cls.name] = str(e)
+            torch.cuda.synchronize()
+    if not rows:
+        raise SystemExit("no row of the hot path is available")
+
+    def step(record):
+        for r in rows:
+            flush.fill_(1.0)
+            if not record:
+                r.timers = []
+            r.run()
+
+    for _ in range(args.warmup):
+        step(False)
+    for r in rows:
+        r.timers = []
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    s_all, e_all = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s_all.record()
+    for _ in range(args.steps):
+        step(True)
+    e_all.record()
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    barrier(world)
+    ms_step = max_over_ranks(world, s_all.elapsed_time(e_all) / args.steps)
+    reports = {}
+    for r in rows:
+        per = {}
+        for label, s, e in r.timers:
+            per[label] = per.get(label, 0.0) + s.elapsed_time(e)
+        per = {k: max_over_ranks(world, v / args.steps) for k, v in per.items()}
+        reports[r.name] = r.report(per, peaks)
+    head_row = "prefill" if "prefill" in reports else ("gemv" if "gemv" in reports else rows[0].name)
+    head = reports[head_row]
+    e2e = None
+    byname = {r.name: r for r in rows}
+    if head_row == "prefill":
+        e2e = e2e_prefill(nv, byname["prefill"], max(3, args.steps))
+    elif head_row == "gemv":
+        e2e = e2e_gemv(nv, byname["gemv"], max(10, args.steps))
+    if e2e is not None:
+        # every rank solves its own problem: whole-job work / slowest rank
+        ms_e2e = max_over_ranks(world, e2e.pop("ms"))
+        e2e = {"value": world * e2e.pop("work") / ms_e2e, **e2e, "ms_per_step": ms_e2e}
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline_prefill()
+            if head_row != "prefill":
+                cpu["note"] = "headline row is not prefill; baseline of the prefill op shown"
+        roof = dict(head["roofline"])
+        roof["traffic"] = None
+        line = {
+            "metric": "qqmm FP4 TFLOP/s (% dense FP4 peak); quantize & qmv GB/s (% HBM peak)",
+            "value": head["value"] * world, "unit": head["unit"], "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4 (e2m1 codes, e4m3 block scales, fp32 accumulate), bf16 io",
+            "data": "synthetic (seeded torch generators; shapes and distributions of the workload configs)",
+            "config": {"workload": f"{head_row}: " + {
+                "prefill": "nvfp4 qqmm op, x [4096,4096] bf16 N(0,1), W [4096,4096] bf16 N(0,0.02) with 1% x50 "
+                           "outliers, g = amax, SWIZZLED scales, y bf16",
+                "gemv": "nvfp4 qmv, x [1,4096] bf16, W [14336,4096] pre-quantized"}.get(head_row, head_row),
+                "rows_per_step": [r.name for r in rows], "l2": "flushed (256 MiB write) before every row",
+                "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": sum(r.launches for r in rows) * args.steps,
+            "clocks": clocks,
+            "rows": reports,
+        }
+        if unavailable:
+            line["unavailable_rows"] = unavailable
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle (plain CPU code) on the same workload
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        pass
+    samples = []
+    t0 = time.perf_counter()
+    for _ in range(max(1, args.steps)):
+        samples.append(cpu_baseline_prefill(sample_rows=4))
+    wall = time.perf_counter() - t0
+    v = statistics.median(s["value"] for s in samples)
+    line = {"impl": "reference", "metric": "qqmm FP4 TFLOP/s (% dense FP4 peak); quantize & qmv GB/s (% HBM peak)",
+            "value": v, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": wall / max(1, args.steps) * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64 contraction of exactly decoded nvfp4 operands",
+            "data": "synthetic (same seeded generators)",
+            "config": {"workload": "prefill: nvfp4 qqmm op (oracle on a bounded sample of rows)"},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "kind": "oracle", "cores": samples[0]["cores"],
+                             "sample": samples[0]["sample"].replace("16 of", "4 of")},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--rows", nargs="*", default=None, help="subset of rows (default: all)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

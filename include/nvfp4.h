@@ -1,0 +1,194 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4.so: NVFP4 / MXFP8 block-scaled quantize,
+ * dequantize and quantized matmuls on NVIDIA B200 (sm_100a).
+ *
+ * Sources, cited by page title and section:
+ *  [P1] "mlx 0.30.7.2 -> 0.30.7.6" diff, page 8: ops.cpp validate_global_scale,
+ *       validate_qqmm_inputs, qqmm, fp_quantize, fp_dequantize; qqmm_utils.h
+ *       get_padded_scale_dims, pad_and_swizzle_scales.
+ *  [P2] "mlx 0.30.7.2 -> 0.30.7.6" diff, page 7: fp_quantize.cu kernels
+ *       fp_quantize_dequantize, fp_quantize_rowwise, fp_dequantize; qqmm.cpp
+ *       QQMatmul::eval_gpu; qqmm_impl.h GemmScalars; qqmm_utils.cu
+ *       compute_qqmm_pointers.
+ *  [P3] "[Metal] global scale for qmm" (ml-explore/mlx pull 4458): gather_qmm
+ *       with per-expert global scales; worked example.
+ *  [P4] osaurus-ai/mlx pull 31: "The fix" (global scale per block scale).
+ *  [P5] "mlx 0.30.7" diff, page 71: qqmm_utils.cu swizzle_scales, 128x4 tiles.
+ *
+ * Conventions for every call
+ *  - Ownership: the caller allocates every buffer; all tensor pointers are
+ *    DEVICE pointers on the current CUDA device.  The library allocates no
+ *    device memory and never synchronizes; each call only enqueues kernels on
+ *    `stream` (NULL = legacy default stream) and returns.
+ *  - Layout: row-major, contiguous.  Every tensor pointer must be 16-byte
+ *    aligned.  Codes of NVFP4 are uint32 words holding 8 e2m1 codes, element
+ *    8w+i of a row in bits 4i..4i+3 of word w; codes of MXFP8 hold 4 e4m3
+ *    bytes, element 4w+i in byte i.
+ *  - Scale layouts: NVFP4_LAYOUT_LINEAR is [rows, K/group] uint8.
+ *    NVFP4_LAYOUT_SWIZZLED is the 128x4-tile layout the block-scaled MMA
+ *    reads ([P5]; [P1] pad_and_swizzle_scales): a [ceil128(rows),
+ *    ceil4(K/group)] buffer where linear scale (r, c) sits at byte
+ *      ((r/128)*(Cp/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + c%4,
+ *    Cp = ceil4(K/group), and every padding byte is 0.
+ *  - Global scales g, g_x, g_w are `const float*` device pointers to one
+ *    fp32 (as the device alpha of [P2] GemmScalars); NULL means none (encode
+ *    and decode factors 1).  They are meaningful for NVFP4 only ([P1]
+ *    validate_global_scale) and must be finite and > 0.
+ *  - Errors: every call returns an nvfp4_status and never throws.  Argument
+ *    checks happen on the host before anything is enqueued; on failure
+ *    nothing is enqueued and nvfp4_last_error_message() explains.
+ *    NVFP4_ERR_CUDA reports a launch error.  Device-side checks (an expert
+ *    index out of range in gather_qmm; a bounded wait that gave up in the
+ *    tensor-core GEMM) set a device error word instead of trapping; read it
+ *    with nvfp4_check_device_errors().
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* nvfp4_stream_t;
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1, /* bad shape, mode, pointer alignment, scale combination */
+  NVFP4_ERR_UNSUPPORTED = 2, /* device is not sm_100, dtype or size not supported */
+  NVFP4_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  NVFP4_ERR_TIMEOUT = 4,     /* a kernel gave up a bounded wait (device error word) */
+  NVFP4_ERR_DEVICE_INDEX = 5 /* a kernel saw an index out of range (device error word) */
+} nvfp4_status;
+
+typedef enum { NVFP4_DT_F32 = 0, NVFP4_DT_F16 = 1, NVFP4_DT_BF16 = 2 } nvfp4_dtype;
+typedef enum { NVFP4_LAYOUT_LINEAR = 0, NVFP4_LAYOUT_SWIZZLED = 1 } nvfp4_layout;
+typedef enum { NVFP4_MODE_NVFP4 = 0, NVFP4_MODE_MXFP8 = 1 } nvfp4_mode;
+
+/* Short text of a status code. */
+NVFP4_API const char* nvfp4_status_string(nvfp4_status s);
+
+/* Message of the last failed call on this host thread ("" if none).  The
+ * texts of the argument checks follow [P1] (e.g. "[qqmm] For nvfp4 mode,
+ * either both global_scale_x and global_scale_w must be provided, or
+ * neither."). */
+NVFP4_API const char* nvfp4_last_error_message(void);
+
+/* Synchronizes `stream`, then reads and clears the device error word.
+ * Returns NVFP4_OK, NVFP4_ERR_TIMEOUT, NVFP4_ERR_DEVICE_INDEX or
+ * NVFP4_ERR_CUDA.  This is the only call that synchronizes. */
+NVFP4_API nvfp4_status nvfp4_check_device_errors(nvfp4_stream_t stream);
+
+/* Bytes of a scale buffer for `rows` x `cols` scales in `layout`
+ * ([P1] get_padded_scale_dims for SWIZZLED). */
+NVFP4_API size_t nvfp4_scale_bytes(int64_t rows, int64_t cols, nvfp4_layout layout);
+
+/* a1 -- tensor amax: *g_out = max |x| over n elements, fp32.  This is the
+ * global scale g the method uses ([P1] QQMatmul::vjp: astype(max(abs(cotan)),
+ * float32); [P2] compute_qqmm_pointers names its inputs tensor_amax_x/_w).
+ * x: [n] of dt.  g_out: device fp32, overwritten (zeroed then reduced). */
+NVFP4_API nvfp4_status nvfp4_amax(const void* x, nvfp4_dtype dt, int64_t n, float* g_out,
+                        nvfp4_stream_t stream);
+
+/* a2-a4 -- NVFP4 two-level quantize ([P2] fp_quantize_rowwise with global
+ * scale).  Per row, per 16-element block along K:
+ *   E = 2688 / g (1 if g == NULL);  s = e4m3_rne_satfinite((amax/6) * E);
+ *   q_i = e2m1_rne_satfinite(x_i * (E / f8(s)));  a block with s == 0 stores
+ *   zero codes.
+ * x: [rows, K] of dt (fp32, fp16, bf16), K % 16 == 0.
+ * codes: [rows, K/8] uint32 (written).  scales: e4m3 bytes in `layout`
+ * (written, padding included): nvfp4_scale_bytes(rows, K/16, layout). */
+NVFP4_API nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K,
+                            const float* g, uint32_t* codes, uint8_t* scales,
+                            nvfp4_layout layout, nvfp4_stream_t stream);
+
+/* a5 -- NVFP4 dequantize ([P2] fp_dequantize with global scale):
+ *   out = T(e2m1(q) * (f8(s) * g / 2688)),  products in fp32.
+ * codes [rows, K/8], scales in `layout`, out [rows, K] of out_dt. */
+NVFP4_API nvfp4_status nvfp4_dequantize(const uint32_t* codes, const uint8_t* scales,
+                              nvfp4_layout layout, int64_t rows, int64_t K, const float* g,
+                              void* out, nvfp4_dtype out_dt, nvfp4_stream_t stream);
+
+/* a11 -- MXFP8 quantize ([P2] fp_quantize_rowwise with 8 bits and the e8m0
+ * scale; group size 32, [P1] fp_quantize; the E8M0 scale is rounded up, [P3]
+ * mlxcel note).  Per 32-block: s = ue8m0_round_up(amax / 448);
+ *   q_i = e4m3_rne_satfinite(x_i / 2^(s-127)).
+ * x [rows, K] of dt, K % 32 == 0; codes [rows, K/4] uint32; scales e8m0
+ * bytes in `layout`: nvfp4_scale_bytes(rows, K/32, layout). */
+NVFP4_API nvfp4_status mxfp8_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K,
+                            uint32_t* codes, uint8_t* scales, nvfp4_layout layout,
+                            nvfp4_stream_t stream);
+
+/* MXFP8 dequantize ([P1] fp_dequantize fallback, e8m0 branch):
+ *   out = T(e4m3(q) * 2^(s-127)). */
+NVFP4_API nvfp4_status mxfp8_dequantize(const uint32_t* codes, const uint8_t* scales,
+                              nvfp4_layout layout, int64_t rows, int64_t K, void* out,
+                              nvfp4_dtype out_dt, nvfp4_stream_t stream);
+
+/* a4 -- LINEAR -> SWIZZLED re-layout of a [rows, cols] uint8 scale matrix
+ * ([P5] swizzle_scales; [P1] pad_and_swizzle_scales), for scales produced
+ * elsewhere.  swz: nvfp4_scale_bytes(rows, cols, SWIZZLED) bytes, all
+ * written (padding zero). */
+NVFP4_API nvfp4_status nvfp4_swizzle_scales(const uint8_t* lin, int64_t rows, int64_t cols,
+                                  uint8_t* swz, nvfp4_stream_t stream);
+
+/* a8-a9, a12 -- dense block-scaled quantized matmul y = x_hat . w_hat^T
+ * ([P2] QQMatmul::eval_gpu dense route; [P1] validate_qqmm_inputs).
+ *  mode NVFP4: a_codes [M, K/8], b_codes [N, K/8], e4m3 scales SWIZZLED
+ *    (nvfp4_scale_bytes(M, K/16, SWIZZLED) and (N, K/16)); optional g_x, g_w
+ *    (both or neither); y = alpha * sum_b f8(sx) f8(sw) sum_k e2m1 e2m1 with
+ *    alpha = (g_x / 2688) * (g_w / 2688) ([P2] compute_qqmm_pointers).
+ *  mode MXFP8: a_codes [M, K/4], b_codes [N, K/4], e8m0 scales SWIZZLED
+ *    (K/32 per row); g_x, g_w must be NULL.
+ *  K % 32 == 0 (NVFP4: K % 64 recommended; a ragged last 64-block is zero
+ *  padded by the kernel).  y: [M, N] of y_dt (fp32, fp16 or bf16), written. */
+NVFP4_API nvfp4_status qqmm(nvfp4_mode mode, int64_t M, int64_t N, int64_t K, const uint32_t* a_codes,
+                  const uint8_t* a_scales, const uint32_t* b_codes, const uint8_t* b_scales,
+                  const float* g_x, const float* g_w, void* y, nvfp4_dtype y_dt,
+                  nvfp4_stream_t stream);
+
+/* a6-a7 -- qmv, the small-M route of qqmm with a pre-quantized NVFP4 weight
+ * ([P2] QQMatmul::eval_gpu, M = 1 branch: fp_quantize_dequantize then
+ * fp_qmv):  x_hat = quantize-dequantize(x, g_x) in x's type;
+ *   y[m,n] = T(sum_k x_hat[m,k] * e2m1(q[n,k]) * sd[n,k/16]), fp32
+ *   accumulation, sd = f8(s) * (g_w / 2688) in fp32: the global scale is
+ *   applied to each block scale ([P4] "The fix"), and the weight is not
+ *   rounded to T on this path.
+ * x [M, K] of x_dt, 1 <= M <= 8, K % 32 == 0, M*K*4 bytes <= 160 KiB;
+ * w_codes [N, K/8]; w_scales LINEAR [N, K/16]; y [M, N] of x_dt. */
+NVFP4_API nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32_t* w_codes,
+                 const uint8_t* w_scales, const float* g_w, int64_t M, int64_t N, int64_t K,
+                 void* y, nvfp4_stream_t stream);
+
+/* a10 -- gather_qmm: MoE matmul with per-expert NVFP4 weights and per-expert
+ * global scales ([P3]: the global scale multiplies each fp8 block scale
+ * inside the dequantization, before the cast to bf16; weights transposed).
+ *   y[t, j, :] = x[t, :] . w_hat_e^T,  e = idx[t, j],
+ *   w_hat_e = bf16(e2m1(q) * (f8(s) * g[e] / 2688)),  fp32 accumulation.
+ * x [T, K] bf16; w_codes [E, N, K/8]; w_scales LINEAR [E, N, K/16];
+ * g [E] fp32 or NULL; idx [T, topk] int32 in [0, E) (checked on the device:
+ * out-of-range entries set NVFP4_ERR_DEVICE_INDEX and produce zero rows);
+ * y [T, topk, N] bf16.  K % 64 == 0, N % 16 == 0.
+ * workspace: device scratch of gather_qmm_workspace_size(T, topk, E) bytes,
+ * 16-byte aligned, contents undefined on entry and exit. */
+NVFP4_API nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const uint8_t* w_scales,
+                        const float* g, const int32_t* idx, int64_t T, int64_t topk,
+                        int64_t E, int64_t N, int64_t K, void* y, void* workspace,
+                        size_t workspace_bytes, nvfp4_stream_t stream);
+
+NVFP4_API size_t gather_qmm_workspace_size(int64_t T, int64_t topk, int64_t E);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

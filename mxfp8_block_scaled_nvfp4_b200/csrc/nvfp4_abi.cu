@@ -1,0 +1,381 @@
+// libnvfp4.so: the C ABI of include/nvfp4.h.  Host-side argument checks
+// (texts after ops.cpp validate_global_scale / validate_qqmm_inputs,
+// "mlx 0.30.7.2 -> 0.30.7.6" diff, page 8), launch configuration and the
+// device error word.  One translation unit: the kernels live in the .cuh
+// files it includes.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "nvfp4.h"
+#include "common.cuh"
+#include "quantize.cuh"
+#include "qmv.cuh"
+#include "qqmm_sm100.cuh"
+#include "gather_qmm.cuh"
+
+using namespace nvfp4;
+
+namespace {
+
+thread_local char t_msg[512] = "";
+
+nvfp4_status fail(nvfp4_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_msg, sizeof(t_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+nvfp4_status ok() {
+  t_msg[0] = '\0';
+  return NVFP4_OK;
+}
+
+nvfp4_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(NVFP4_ERR_CUDA, "[%s] launch failed: %s", what, cudaGetErrorString(e));
+  return ok();
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+  int sm_count = 0;
+  int cc_major = 0;
+  int cc_minor = 0;
+  bool ok = false;
+};
+
+DeviceInfo g_dev[64];
+std::mutex g_dev_mu;
+
+// Current device's properties; the library runs on sm_100 (B200) only.
+nvfp4_status device_info(const char* tag, DeviceInfo* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(NVFP4_ERR_CUDA, "[%s] cudaGetDevice: %s", tag, cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] device ordinal %d", tag, dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ok) {
+    if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return fail(NVFP4_ERR_CUDA, "[%s] cudaDeviceGetAttribute failed", tag);
+    d.ok = true;
+  }
+  if (d.cc_major != 10 || d.cc_minor != 0)
+    return fail(NVFP4_ERR_UNSUPPORTED,
+                "[%s] this library is built for sm_100a (B200); device has compute capability %d.%d",
+                tag, d.cc_major, d.cc_minor);
+  *out = d;
+  return NVFP4_OK;
+}
+
+bool valid_dt(nvfp4_dtype dt) { return dt == NVFP4_DT_F32 || dt == NVFP4_DT_F16 || dt == NVFP4_DT_BF16; }
+
+// Persistent elementwise grid: enough CTAs to fill every SM, never more than
+// the work needs.
+unsigned ew_grid(const DeviceInfo& d, uint64_t work_threads) {
+  uint64_t want = (work_threads + kEwThreads - 1) / kEwThreads;
+  uint64_t cap = (uint64_t)d.sm_count * 8;  // 8 x 256 threads resident per SM
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  return (unsigned)want;
+}
+
+template <typename F>
+void dispatch_dt(nvfp4_dtype dt, F&& f) {
+  switch (dt) {
+    case NVFP4_DT_F32: f(float{}); break;
+    case NVFP4_DT_F16: f(__half{}); break;
+    default: f(__nv_bfloat16{}); break;
+  }
+}
+
+constexpr int64_t kMaxElems = (int64_t)1 << 34;  // 16 Gi elements: 32-bit half-block indices
+
+}  // namespace
+
+extern "C" {
+
+const char* nvfp4_status_string(nvfp4_status s) {
+  switch (s) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_UNSUPPORTED: return "unsupported";
+    case NVFP4_ERR_CUDA: return "CUDA error";
+    case NVFP4_ERR_TIMEOUT: return "device wait timed out";
+    case NVFP4_ERR_DEVICE_INDEX: return "device-side index out of range";
+  }
+  return "unknown status";
+}
+
+const char* nvfp4_last_error_message(void) { return t_msg; }
+
+nvfp4_status nvfp4_check_device_errors(nvfp4_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return fail(NVFP4_ERR_CUDA, "[check_device_errors] %s", cudaGetErrorString(e));
+  unsigned int word = 0;
+  e = cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word));
+  if (e != cudaSuccess) return fail(NVFP4_ERR_CUDA, "[check_device_errors] %s", cudaGetErrorString(e));
+  if (word != 0) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+    if (word & kDevErrTimeout)
+      return fail(NVFP4_ERR_TIMEOUT, "[device] a kernel gave up a bounded wait (word 0x%x)", word);
+    return fail(NVFP4_ERR_DEVICE_INDEX, "[device] an index was out of range (word 0x%x)", word);
+  }
+  return ok();
+}
+
+size_t nvfp4_scale_bytes(int64_t rows, int64_t cols, nvfp4_layout layout) {
+  if (rows < 0 || cols < 0) return 0;
+  if (layout == NVFP4_LAYOUT_LINEAR) return (size_t)(rows * cols);
+  return (size_t)(((rows + 127) / 128 * 128) * ((cols + 3) / 4 * 4));
+}
+
+nvfp4_status nvfp4_amax(const void* x, nvfp4_dtype dt, int64_t n, float* g_out, nvfp4_stream_t stream) {
+  if (!valid_dt(dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[amax] dtype must be float32, float16 or bfloat16");
+  if (n < 0 || n > kMaxElems) return fail(NVFP4_ERR_INVALID_ARG, "[amax] bad size %lld", (long long)n);
+  if (!g_out || (n > 0 && !x)) return fail(NVFP4_ERR_INVALID_ARG, "[amax] null pointer");
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(g_out) & 3u))
+    return fail(NVFP4_ERR_INVALID_ARG, "[amax] x must be 16-byte aligned, g_out 4-byte aligned");
+  DeviceInfo d;
+  nvfp4_status st = device_info("amax", &d);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = cudaMemsetAsync(g_out, 0, sizeof(float), stream);
+  if (e != cudaSuccess) return fail(NVFP4_ERR_CUDA, "[amax] memset: %s", cudaGetErrorString(e));
+  if (n == 0) return ok();
+  const unsigned grid = ew_grid(d, (uint64_t)(n / 8 + 1));
+  dispatch_dt(dt, [&](auto tag) {
+    using T = decltype(tag);
+    k_amax<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n, g_out);
+  });
+  return check_launch("amax");
+}
+
+static nvfp4_status quantize_common(const char* tag, bool mx, const void* x, nvfp4_dtype dt,
+                                    int64_t rows, int64_t K, const float* g, uint32_t* codes,
+                                    uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
+  const int group = mx ? 32 : 16;
+  if (!valid_dt(dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] dtype must be float32, float16 or bfloat16", tag);
+  if (layout != NVFP4_LAYOUT_LINEAR && layout != NVFP4_LAYOUT_SWIZZLED)
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] unknown scale layout", tag);
+  if (rows < 0 || K < 0 || rows * K > kMaxElems)
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] bad shape [%lld, %lld]", tag, (long long)rows, (long long)K);
+  if (K % group != 0)
+    return fail(NVFP4_ERR_INVALID_ARG,
+                "[%s] The last dimension of the matrix needs to be divisible by the quantization group size %d. "
+                "However the provided matrix has shape [%lld, %lld]",
+                tag, group, (long long)rows, (long long)K);
+  if (rows * K > 0 && (!x || !codes || !scales)) return fail(NVFP4_ERR_INVALID_ARG, "[%s] null pointer", tag);
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(g) & 3u))
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] tensor pointers must be 16-byte aligned", tag);
+  DeviceInfo d;
+  nvfp4_status st = device_info(tag, &d);
+  if (st != NVFP4_OK) return st;
+  if (rows * K == 0) return ok();
+  ScaleOut so;
+  so.p = scales;
+  so.blocks_per_row = (uint32_t)(K / group);
+  so.Cp = (uint32_t)((K / group + 3) / 4 * 4);
+  so.swizzled = layout == NVFP4_LAYOUT_SWIZZLED;
+  const uint32_t n_half = (uint32_t)(rows * K / 8);
+  const unsigned grid = ew_grid(d, ((uint64_t)n_half + kUnroll - 1) / kUnroll);
+  dispatch_dt(dt, [&](auto tag_t) {
+    using T = decltype(tag_t);
+    if (mx)
+      k_mxfp8_quantize<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, codes, so,
+                                                           (uint32_t)rows);
+    else
+      k_nvfp4_quantize<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, g, codes, so,
+                                                           (uint32_t)rows);
+  });
+  return check_launch(tag);
+}
+
+nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K, const float* g,
+                            uint32_t* codes, uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
+  return quantize_common("quantize", false, x, dt, rows, K, g, codes, scales, layout, stream);
+}
+
+nvfp4_status mxfp8_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K, uint32_t* codes,
+                            uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
+  return quantize_common("mxfp8_quantize", true, x, dt, rows, K, nullptr, codes, scales, layout, stream);
+}
+
+static nvfp4_status dequantize_common(const char* tag, bool mx, const uint32_t* codes, const uint8_t* scales,
+                                      nvfp4_layout layout, int64_t rows, int64_t K, const float* g, void* out,
+                                      nvfp4_dtype out_dt, nvfp4_stream_t stream) {
+  const int group = mx ? 32 : 16;
+  if (!valid_dt(out_dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] output dtype must be float32, float16 or bfloat16", tag);
+  if (layout != NVFP4_LAYOUT_LINEAR && layout != NVFP4_LAYOUT_SWIZZLED)
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] unknown scale layout", tag);
+  if (rows < 0 || K < 0 || rows * K > kMaxElems || K % group != 0)
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] bad shape [%lld, %lld] for group size %d", tag, (long long)rows,
+                (long long)K, group);
+  if (rows * K > 0 && (!codes || !scales || !out)) return fail(NVFP4_ERR_INVALID_ARG, "[%s] null pointer", tag);
+  if (!aligned16(codes) || !aligned16(scales) || !aligned16(out) || (reinterpret_cast<uintptr_t>(g) & 3u))
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] tensor pointers must be 16-byte aligned", tag);
+  DeviceInfo d;
+  nvfp4_status st = device_info(tag, &d);
+  if (st != NVFP4_OK) return st;
+  if (rows * K == 0) return ok();
+  ScaleIn si;
+  si.p = scales;
+  si.blocks_per_row = (uint32_t)(K / group);
+  si.Cp = (uint32_t)((K / group + 3) / 4 * 4);
+  si.swizzled = layout == NVFP4_LAYOUT_SWIZZLED;
+  const uint32_t n_half = (uint32_t)(rows * K / 8);
+  const unsigned grid = ew_grid(d, n_half);
+  dispatch_dt(out_dt, [&](auto tag_t) {
+    using T = decltype(tag_t);
+    if (mx)
+      k_mxfp8_dequantize<T><<<grid, kEwThreads, 0, stream>>>(codes, si, n_half, static_cast<T*>(out));
+    else
+      k_nvfp4_dequantize<T><<<grid, kEwThreads, 0, stream>>>(codes, si, g, n_half, static_cast<T*>(out));
+  });
+  return check_launch(tag);
+}
+
+nvfp4_status nvfp4_dequantize(const uint32_t* codes, const uint8_t* scales, nvfp4_layout layout, int64_t rows,
+                              int64_t K, const float* g, void* out, nvfp4_dtype out_dt, nvfp4_stream_t stream) {
+  return dequantize_common("dequantize", false, codes, scales, layout, rows, K, g, out, out_dt, stream);
+}
+
+nvfp4_status mxfp8_dequantize(const uint32_t* codes, const uint8_t* scales, nvfp4_layout layout, int64_t rows,
+                              int64_t K, void* out, nvfp4_dtype out_dt, nvfp4_stream_t stream) {
+  return dequantize_common("mxfp8_dequantize", true, codes, scales, layout, rows, K, nullptr, out, out_dt, stream);
+}
+
+nvfp4_status nvfp4_swizzle_scales(const uint8_t* lin, int64_t rows, int64_t cols, uint8_t* swz,
+                                  nvfp4_stream_t stream) {
+  if (rows < 0 || cols < 0 || rows * cols > ((int64_t)1 << 31))
+    return fail(NVFP4_ERR_INVALID_ARG, "[swizzle_scales] bad shape");
+  if (rows * cols > 0 && (!lin || !swz)) return fail(NVFP4_ERR_INVALID_ARG, "[swizzle_scales] null pointer");
+  if (!aligned16(lin) || !aligned16(swz))
+    return fail(NVFP4_ERR_INVALID_ARG, "[swizzle_scales] Starting addresses must be 16-byte aligned");
+  DeviceInfo d;
+  nvfp4_status st = device_info("swizzle_scales", &d);
+  if (st != NVFP4_OK) return st;
+  if (rows * cols == 0) return ok();
+  const uint32_t Rp = (uint32_t)((rows + 127) / 128 * 128), Cp = (uint32_t)((cols + 3) / 4 * 4);
+  const unsigned grid = ew_grid(d, (uint64_t)Rp * Cp);
+  k_swizzle_scales<<<grid, kEwThreads, 0, stream>>>(lin, (uint32_t)rows, (uint32_t)cols, Rp, Cp, swz);
+  return check_launch("swizzle_scales");
+}
+
+// Global-scale checks of qqmm ("mlx 0.30.7.2 -> 0.30.7.6" diff, page 8,
+// ops.cpp validate_global_scale and validate_qqmm_inputs).
+static nvfp4_status check_qqmm_global_scales(nvfp4_mode mode, const float* g_x, const float* g_w) {
+  if (mode != NVFP4_MODE_NVFP4 && (g_x || g_w))
+    return fail(NVFP4_ERR_INVALID_ARG, "[qqmm] Global scale is only supported for 'nvfp4' quantization mode.");
+  if (mode == NVFP4_MODE_NVFP4 && ((g_x == nullptr) != (g_w == nullptr)))
+    return fail(NVFP4_ERR_INVALID_ARG,
+                "[qqmm] For nvfp4 mode, either both global_scale_x and global_scale_w must be provided, or neither.");
+  return NVFP4_OK;
+}
+
+nvfp4_status qqmm(nvfp4_mode mode, int64_t M, int64_t N, int64_t K, const uint32_t* a_codes,
+                  const uint8_t* a_scales, const uint32_t* b_codes, const uint8_t* b_scales, const float* g_x,
+                  const float* g_w, void* y, nvfp4_dtype y_dt, nvfp4_stream_t stream) {
+  if (mode != NVFP4_MODE_NVFP4 && mode != NVFP4_MODE_MXFP8)
+    return fail(NVFP4_ERR_INVALID_ARG, "[qqmm] Only 'nvfp4' and 'mxfp8' modes are supported.");
+  nvfp4_status st = check_qqmm_global_scales(mode, g_x, g_w);
+  if (st != NVFP4_OK) return st;
+  if (!valid_dt(y_dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[qqmm] output dtype must be float32, float16 or bfloat16");
+  if (M < 0 || N < 0 || K < 0 || M > (1 << 30) || N > (1 << 30) || K > (1 << 30))
+    return fail(NVFP4_ERR_INVALID_ARG, "[qqmm] bad shape");
+  if (K % 32 != 0)
+    return fail(NVFP4_ERR_INVALID_ARG, "[qqmm] K must be a multiple of 32, got %lld", (long long)K);
+  if (M * N > 0 && (!a_codes || !a_scales || !b_codes || !b_scales || !y))
+    return fail(NVFP4_ERR_INVALID_ARG, "[qqmm] null pointer");
+  if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) || !aligned16(y) ||
+      (reinterpret_cast<uintptr_t>(g_x) & 3u) || (reinterpret_cast<uintptr_t>(g_w) & 3u))
+    return fail(NVFP4_ERR_INVALID_ARG, "[qqmm] tensor pointers must be 16-byte aligned");
+  DeviceInfo d;
+  st = device_info("qqmm", &d);
+  if (st != NVFP4_OK) return st;
+  if (M * N == 0) return ok();
+  return qqmm_launch(mode == NVFP4_MODE_MXFP8, M, N, K, a_codes, a_scales, b_codes, b_scales, g_x, g_w, y,
+                     (int)y_dt, d.sm_count, stream, t_msg, sizeof(t_msg));
+}
+
+nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32_t* w_codes, const uint8_t* w_scales,
+                 const float* g_w, int64_t M, int64_t N, int64_t K, void* y, nvfp4_stream_t stream) {
+  if (!valid_dt(x_dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[qmv] dtype must be float32, float16 or bfloat16");
+  if ((g_x == nullptr) != (g_w == nullptr))
+    return fail(NVFP4_ERR_INVALID_ARG,
+                "[qqmm] For nvfp4 mode, either both global_scale_x and global_scale_w must be provided, or neither.");
+  if (M < 1 || M > kQmvMaxM) return fail(NVFP4_ERR_INVALID_ARG, "[qmv] M must be in [1, %d], got %lld", kQmvMaxM, (long long)M);
+  if (N < 0 || K < 32 || K % 32 != 0 || N > (1 << 30))
+    return fail(NVFP4_ERR_INVALID_ARG, "[qmv] bad shape N=%lld K=%lld (K %% 32 == 0)", (long long)N, (long long)K);
+  if (M * K * 4 > 160 * 1024)
+    return fail(NVFP4_ERR_UNSUPPORTED, "[qmv] M*K*4 bytes of x_hat must fit 160 KiB of shared memory");
+  if (N > 0 && (!x || !w_codes || !w_scales || !y)) return fail(NVFP4_ERR_INVALID_ARG, "[qmv] null pointer");
+  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y) ||
+      (reinterpret_cast<uintptr_t>(g_x) & 3u) || (reinterpret_cast<uintptr_t>(g_w) & 3u))
+    return fail(NVFP4_ERR_INVALID_ARG, "[qmv] tensor pointers must be 16-byte aligned");
+  DeviceInfo d;
+  nvfp4_status st = device_info("qmv", &d);
+  if (st != NVFP4_OK) return st;
+  if (N == 0) return ok();
+  const size_t smem = (size_t)M * K * sizeof(float);
+  // one CTA of 16 warps per SM; each warp owns whole weight rows
+  uint64_t grid = ((uint64_t)N + (kQmvThreads / 32) - 1) / (kQmvThreads / 32);
+  if (grid > (uint64_t)d.sm_count) grid = d.sm_count;
+  cudaError_t e = cudaSuccess;
+  dispatch_dt(x_dt, [&](auto tag_t) {
+    using T = decltype(tag_t);
+    auto x_t = [](const void* p) { return static_cast<const T*>(p); };
+    auto y_t = [](void* p) { return static_cast<T*>(p); };
+    auto go = [&](auto kern) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess)
+        kern<<<(unsigned)grid, kQmvThreads, smem, stream>>>(x_t(x), g_x, w_codes, w_scales, g_w, (int)M, (int)N,
+                                                           (int)K, y_t(y));
+    };
+    if (M == 1) go(k_qmv<T, 1>);
+    else if (M == 2) go(k_qmv<T, 2>);
+    else if (M <= 4) go(k_qmv<T, 4>);
+    else go(k_qmv<T, 8>);
+  });
+  if (e != cudaSuccess) return fail(NVFP4_ERR_CUDA, "[qmv] %s", cudaGetErrorString(e));
+  return check_launch("qmv");
+}
+
+size_t gather_qmm_workspace_size(int64_t T, int64_t topk, int64_t E) {
+  return gather_workspace_bytes(T, topk, E);
+}
+
+nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const uint8_t* w_scales, const float* g,
+                        const int32_t* idx, int64_t T, int64_t topk, int64_t E, int64_t N, int64_t K, void* y,
+                        void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+  if (T < 0 || topk < 1 || E < 1 || N < 0 || K < 0 || T * topk > (1 << 30) || E > (1 << 20))
+    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm] bad shape");
+  if (K % 64 != 0 || N % 16 != 0)
+    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm] K must be a multiple of 64 and N of 16 (K=%lld N=%lld)",
+                (long long)K, (long long)N);
+  if (workspace_bytes < gather_workspace_bytes(T, topk, E))
+    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm] workspace too small: %zu < %zu", workspace_bytes,
+                gather_workspace_bytes(T, topk, E));
+  if (T * N > 0 && (!x || !w_codes || !w_scales || !idx || !y || !workspace))
+    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm] null pointer");
+  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y) || !aligned16(workspace) ||
+      !aligned16(idx) || !aligned16(g))
+    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm] tensor pointers must be 16-byte aligned");
+  DeviceInfo d;
+  nvfp4_status st = device_info("gather_qmm", &d);
+  if (st != NVFP4_OK) return st;
+  if (T * N == 0) return ok();
+  return gather_qmm_launch(x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, workspace, d.sm_count, stream, t_msg,
+                           sizeof(t_msg));
+}
+
+}  // extern "C"

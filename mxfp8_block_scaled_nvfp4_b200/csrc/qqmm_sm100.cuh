@@ -1,0 +1,462 @@
+// Dense block-scaled quantized matmul on the 5th-generation tensor cores
+// (tcgen05), sm_100a.
+//
+//   y[m, n] = alpha * sum_b sx[m, b] * sw[n, b] * sum_{k in b} qx[m, k] * qw[n, k]
+//
+// NVFP4: e2m1 codes, ue4m3 scales per 16 elements, alpha = (g_x / 2688) *
+// (g_w / 2688) (the device alpha of compute_qqmm_pointers, "mlx 0.30.7.2 ->
+// 0.30.7.6" diff, page 7, qqmm_utils.cu).  MXFP8: e4m3 codes, ue8m0 scales per
+// 32 elements, alpha = 1.  Folding the global scales into alpha is exact in
+// real arithmetic (sum (c sx dx)(c sw dw) = dx dw sum c sx c sw), and no
+// operand is rounded to a narrower type on this path, so it is equivalent to
+// decoding each block with its global scale.
+//
+// Kernel structure (one CTA per 128 x 256 output tile, 192 threads):
+//   warp 0   TMA producer: per K stage, A codes [128 rows x 128 B] and B codes
+//            [256 rows x 128 B] as 128-byte-swizzled tiles, plus the scale
+//            tiles as plain bulk copies (the 128x4 scale-tile layout of the
+//            operands is already the order the MMA's scale tensor memory
+//            expects, so the copies are contiguous 512-byte blocks).
+//   warp 1   TMEM allocator and MMA issuer: one thread moves the stage's
+//            scale tiles into tensor memory (tcgen05.cp 32x128b.warpx4) and
+//            issues the block-scaled MMAs (M=128, N=256, K=64 NVFP4 / 32
+//            MXFP8 per instruction) into a 128 x 256 fp32 accumulator in TMEM;
+//            tcgen05.commit frees the stage when its MMAs are done.
+//   warps 2-5 epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//            32*(w%4)...), alpha, conversion, stores.
+// Every mbarrier wait is bounded; on timeout the kernel sets the device
+// error word (NVFP4_ERR_TIMEOUT through nvfp4_check_device_errors), drains,
+// frees its TMEM and exits.  No cluster multicast is used.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cstdio>
+
+#include "common.cuh"
+#include "nvfp4.h"
+
+namespace nvfp4 {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BKB = 128;  // bytes of K per row per stage (256 FP4 / 128 FP8 elements)
+constexpr int STAGES = 4;
+constexpr int THREADS = 192;
+constexpr int A_STAGE = BM * BKB;    // 16 KiB
+constexpr int B_STAGE = BN * BKB;    // 32 KiB
+constexpr int SFA_STAGE = 4 * 512;   // up to 4 scale tiles (NVFP4)
+constexpr int SFB_STAGE = 2 * 4 * 512;
+constexpr int SMEM_A = 0;
+constexpr int SMEM_B = SMEM_A + STAGES * A_STAGE;
+constexpr int SMEM_SFA = SMEM_B + STAGES * B_STAGE;
+constexpr int SMEM_SFB = SMEM_SFA + STAGES * SFA_STAGE;
+constexpr int SMEM_BYTES = SMEM_SFB + STAGES * SFB_STAGE;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_SF = 256;       // scale-factor columns start here
+constexpr uint32_t TMEM_SF_STAGE = 48;  // 16 (A) + 32 (B) columns per stage
+constexpr uint32_t kWaitLimit = 1u << 26;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: false (and the device error word set) if the phase never
+// completes.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  atomicOr(&g_device_error, (unsigned)kDevErrTimeout);
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// Shared-memory matrix descriptor of tcgen05 (start >> 4 in bits 0-13,
+// leading byte offset >> 4 in 16-29, stride byte offset >> 4 in 32-45,
+// version 1 in bits 46-47, layout type in 61-63).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)(layout & 7u) << 61;
+  return d;
+}
+
+// K-major operand tile, 128-byte swizzle: 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t kmajor_sw128_desc(uint32_t addr) { return smem_desc(addr, 16, 1024, 2); }
+// A 512-byte scale tile: 32 rows of 16 bytes, no swizzle (8-row core
+// matrices 128 bytes apart).
+__device__ __forceinline__ uint64_t sf_tile_desc(uint32_t addr) { return smem_desc(addr, 0, 128, 0); }
+
+// Instruction descriptor of the block-scaled MMA: A/B formats (bits 7-9,
+// 10-12), K-major A and B, N >> 3 (bits 17-22), scale format (bit 23:
+// 0 = ue4m3, 1 = ue8m0), M >> 4 (bits 24-28), scale-factor byte ids of B
+// (bits 4-5) and A (bits 29-30).
+__host__ __device__ constexpr uint32_t block_scaled_idesc(uint32_t ab_format, uint32_t scale_ue8m0, uint32_t sf_id) {
+  return (sf_id << 4) | (ab_format << 7) | (ab_format << 10) | ((uint32_t)(BN >> 3) << 17) | (scale_ue8m0 << 23) |
+         ((uint32_t)(BM >> 4) << 24) | (sf_id << 29);
+}
+
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+template <bool MX>
+__device__ __forceinline__ void mma_block_scaled(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  if constexpr (MX) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+  }
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive fp32 accumulator columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+struct Params {
+  const uint8_t* sfa;  // SWIZZLED scale buffers
+  const uint8_t* sfb;
+  const float* g_x;
+  const float* g_w;
+  void* y;
+  int M, N, K;
+  int y_dt;             // nvfp4_dtype
+  uint32_t kb_count;    // K stages
+  uint32_t k_bytes;     // bytes of K per row (K/2 NVFP4, K MXFP8)
+  uint32_t sf_groups;   // Cp / 4: scale-tile columns per 128-row block
+  uint32_t rows_b_pad;  // ceil128(N)
+};
+
+template <typename T>
+__device__ __forceinline__ void store_out(T* dst, const float* v, int n);
+
+template <>
+__device__ __forceinline__ void store_out<float>(float* dst, const float* v, int n) {
+  if (n == 32 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+  } else {
+    for (int i = 0; i < n; ++i) dst[i] = v[i];
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void store_out_16(T* dst, const float* v, int n) {
+  if (n == 32 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+      float t[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) t[j] = v[i + j];
+      store8<T>(dst + i, t);
+    }
+  } else {
+    for (int i = 0; i < n; ++i) dst[i] = Elem<T>::from_f(v[i]);
+  }
+}
+
+template <>
+__device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* dst, const float* v, int n) {
+  store_out_16<__nv_bfloat16>(dst, v, n);
+}
+template <>
+__device__ __forceinline__ void store_out<__half>(__half* dst, const float* v, int n) {
+  store_out_16<__half>(dst, v, n);
+}
+
+template <bool MX>
+__global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUtensorMap tmap_a,
+                                                     const __grid_constant__ CUtensorMap tmap_b, Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t accum_bar;
+  __shared__ uint32_t tmem_base_holder;
+  __shared__ int abort_flag;
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile_n = blockIdx.x * BN, tile_m = blockIdx.y * BM;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    mbar_init(smem_u32(&accum_bar), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_holder;
+
+  // scale tiles present in this tile's column of row blocks
+  const bool b_second = (uint32_t)(tile_n + 128) < p.rows_b_pad;
+  const uint32_t tiles_per_stage = MX ? 1u : 4u;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t issued = 0;
+      for (uint32_t kb = 0; kb < p.kb_count; ++kb) {
+        const uint32_t s = kb % STAGES;
+        const uint32_t par = ((kb / STAGES) & 1u) ^ 1u;
+        if (!mbar_wait(smem_u32(&empty_bar[s]), par)) {
+          abort_flag = 1;
+          break;
+        }
+        // scale tiles of this stage that exist (ragged K)
+        const uint32_t g0 = kb * tiles_per_stage;
+        uint32_t nt = p.sf_groups > g0 ? p.sf_groups - g0 : 0;
+        if (nt > tiles_per_stage) nt = tiles_per_stage;
+        const uint32_t sf_bytes_a = nt * 512u, sf_bytes_b = nt * 512u * (b_second ? 2u : 1u);
+        const uint32_t bar = smem_u32(&full_bar[s]);
+        mbar_expect_tx(bar, A_STAGE + B_STAGE + sf_bytes_a + sf_bytes_b);
+        tma_load_2d(sbase + SMEM_A + s * A_STAGE, &tmap_a, (int)(kb * BKB), tile_m, bar);
+        tma_load_2d(sbase + SMEM_B + s * B_STAGE, &tmap_b, (int)(kb * BKB), tile_n, bar);
+        if (nt) {
+          const uint8_t* sa = p.sfa + ((size_t)(tile_m / 128) * p.sf_groups + g0) * 512u;
+          bulk_load(sbase + SMEM_SFA + s * SFA_STAGE, sa, sf_bytes_a, bar);
+          const uint8_t* sb = p.sfb + ((size_t)(tile_n / 128) * p.sf_groups + g0) * 512u;
+          bulk_load(sbase + SMEM_SFB + s * SFB_STAGE, sb, sf_bytes_a, bar);
+          if (b_second) {
+            const uint8_t* sb2 = p.sfb + ((size_t)(tile_n / 128 + 1) * p.sf_groups + g0) * 512u;
+            bulk_load(sbase + SMEM_SFB + s * SFB_STAGE + 4 * 512, sb2, sf_bytes_a, bar);
+          }
+        }
+        ++issued;
+      }
+      // drain: every stage issued must have landed before the CTA may exit
+      const uint32_t first = issued > (uint32_t)STAGES ? issued - STAGES : 0;
+      for (uint32_t kb = first; kb < issued; ++kb)
+        mbar_wait(smem_u32(&full_bar[kb % STAGES]), (kb / STAGES) & 1u);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (uint32_t kb = 0; kb < p.kb_count; ++kb) {
+        const uint32_t s = kb % STAGES;
+        if (!mbar_wait(smem_u32(&full_bar[s]), (kb / STAGES) & 1u) || *(volatile int*)&abort_flag) {
+          abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tsfa = tmem + TMEM_SF + s * TMEM_SF_STAGE;
+        const uint32_t tsfb = tsfa + 16;
+        const uint32_t g0 = kb * tiles_per_stage;
+        uint32_t nt = p.sf_groups > g0 ? p.sf_groups - g0 : 0;
+        if (nt > tiles_per_stage) nt = tiles_per_stage;
+        for (uint32_t t = 0; t < nt; ++t) {
+          tmem_cp_sf(tsfa + 4 * t, sf_tile_desc(sbase + SMEM_SFA + s * SFA_STAGE + 512 * t));
+          tmem_cp_sf(tsfb + 8 * t, sf_tile_desc(sbase + SMEM_SFB + s * SFB_STAGE + 512 * t));
+          if (b_second) tmem_cp_sf(tsfb + 8 * t + 4, sf_tile_desc(sbase + SMEM_SFB + s * SFB_STAGE + 4 * 512 + 512 * t));
+        }
+        const uint32_t a0 = sbase + SMEM_A + s * A_STAGE, b0 = sbase + SMEM_B + s * B_STAGE;
+#pragma unroll
+        for (uint32_t j = 0; j < 4; ++j) {
+          if (kb * BKB + j * 32u >= p.k_bytes) break;  // ragged K: no codes left
+          const uint64_t ad = kmajor_sw128_desc(a0 + j * 32u);
+          const uint64_t bd = kmajor_sw128_desc(b0 + j * 32u);
+          uint32_t idesc, sfa, sfb;
+          if (MX) {
+            idesc = block_scaled_idesc(0u, 1u, j);  // e4m3 x e4m3, ue8m0, byte j of the scale words
+            sfa = tsfa;
+            sfb = tsfb;
+          } else {
+            idesc = block_scaled_idesc(1u, 0u, 0u);  // e2m1 x e2m1, ue4m3
+            sfa = tsfa + 4 * j;
+            sfb = tsfb + 8 * j;
+          }
+          mma_block_scaled<MX>(tmem, ad, bd, idesc, sfa, sfb, (kb | j) != 0);
+        }
+        mma_commit(smem_u32(&empty_bar[s]));
+      }
+      mma_commit(smem_u32(&accum_bar));
+    }
+  } else {
+    // epilogue warps 2..5: TMEM lane quarter q = warp % 4
+    const int q = warp & 3;
+    const int row = tile_m + q * 32 + lane;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&accum_bar), 0) && !*(volatile int*)&abort_flag);
+    tc_fence_after();
+    float alpha = 1.0f;
+    if (!MX && p.g_x != nullptr) alpha = (__ldg(p.g_x) / kGlobalEncode) * (__ldg(p.g_w) / kGlobalEncode);
+    if (ok) {
+      for (int c = 0; c < BN; c += 32) {
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
+        const int col = tile_n + c;
+        if (row < p.M && col < p.N) {
+          const int n = min(32, p.N - col);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= alpha;
+          const size_t off = (size_t)row * p.N + col;
+          if (p.y_dt == NVFP4_DT_F32) store_out<float>(static_cast<float*>(p.y) + off, v, n);
+          else if (p.y_dt == NVFP4_DT_BF16) store_out<__nv_bfloat16>(static_cast<__nv_bfloat16*>(p.y) + off, v, n);
+          else store_out<__half>(static_cast<__half*>(p.y) + off, v, n);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D byte tensor [rows, row_bytes] (row stride row_bytes), box [box_rows, 128 B],
+// 128-byte swizzle, out-of-range elements read as zero.
+inline bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t row_bytes, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)BKB, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+inline nvfp4_status qqmm_launch(bool mx, int64_t M, int64_t N, int64_t K, const uint32_t* a_codes,
+                                const uint8_t* a_scales, const uint32_t* b_codes, const uint8_t* b_scales,
+                                const float* g_x, const float* g_w, void* y, int y_dt, int sm_count,
+                                cudaStream_t stream, char* msg, size_t msg_len) {
+  using namespace tc;
+  const uint64_t k_bytes = mx ? (uint64_t)K : (uint64_t)K / 2;
+  CUtensorMap ta, tb;
+  if (!make_tmap(&ta, a_codes, (uint64_t)M, k_bytes, BM) || !make_tmap(&tb, b_codes, (uint64_t)N, k_bytes, BN)) {
+    snprintf(msg, msg_len, "[qqmm] cuTensorMapEncodeTiled failed");
+    return NVFP4_ERR_CUDA;
+  }
+  Params p;
+  p.sfa = a_scales;
+  p.sfb = b_scales;
+  p.g_x = g_x;
+  p.g_w = g_w;
+  p.y = y;
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.y_dt = y_dt;
+  p.k_bytes = (uint32_t)k_bytes;
+  p.kb_count = (uint32_t)((k_bytes + BKB - 1) / BKB);
+  const int64_t sf_cols = mx ? K / 32 : K / 16;
+  p.sf_groups = (uint32_t)((sf_cols + 3) / 4);
+  p.rows_b_pad = (uint32_t)((N + 127) / 128 * 128);
+  dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+  cudaError_t e;
+  if (mx) {
+    e = cudaFuncSetAttribute(k_qqmm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+    if (e == cudaSuccess) k_qqmm<true><<<grid, THREADS, SMEM_ALLOC, stream>>>(ta, tb, p);
+  } else {
+    e = cudaFuncSetAttribute(k_qqmm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+    if (e == cudaSuccess) k_qqmm<false><<<grid, THREADS, SMEM_ALLOC, stream>>>(ta, tb, p);
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    snprintf(msg, msg_len, "[qqmm] launch failed: %s", cudaGetErrorString(e));
+    return NVFP4_ERR_CUDA;
+  }
+  msg[0] = '\0';
+  (void)sm_count;
+  return NVFP4_OK;
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,269 @@
+// HBM-bound elementwise kernels: tensor amax, NVFP4 / MXFP8 quantize,
+// dequantize and the standalone scale re-layout.
+//
+// Work mapping.  A tensor [rows, K] is viewed as a flat sequence of
+// "half-blocks" of 8 consecutive elements (K % 16 == 0, so a 16-element NVFP4
+// block is two adjacent half-blocks of the same row, and a 32-element MXFP8
+// block four).  Lane l of a warp takes half-block base + l, so one warp load
+// instruction reads 32 x 16 contiguous bytes (bf16 / fp16), the block amax
+// is two (NVFP4) or three (MXFP8) xor-shuffles, and each lane stores one
+// packed uint32 of eight e2m1 codes (NVFP4) or two of e4m3 codes (MXFP8):
+// 128 or 256 contiguous bytes per warp store.  Scales are written by the
+// first lane of each block, directly at their LINEAR or 128x4-tile offset.
+// Grids are persistent (a multiple of the SM count); each warp processes
+// kUnroll x 32 half-blocks per iteration to keep several loads in flight.
+#pragma once
+
+#include "common.cuh"
+
+namespace nvfp4 {
+
+constexpr int kEwThreads = 256;
+constexpr int kUnroll = 4;
+
+// ---------------------------------------------------------------------------
+// a1: g = max |x|, atomically combined into *out (which the host zeroes).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kEwThreads) k_amax(const T* __restrict__ x, int64_t n,
+                                                     float* __restrict__ out) {
+  const int64_t nvec = n / 8;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+  float m = 0.0f;
+  for (int64_t i = tid; i < nvec; i += nthr) {
+    float v[8];
+    load8<T>(x + i * 8, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+  }
+  for (int64_t i = nvec * 8 + tid; i < n; i += nthr) m = fmaxf(m, fabsf(Elem<T>::to_f(x[i])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  __shared__ float red[kEwThreads / 32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    // non-negative floats order like their bit patterns
+    if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned int*>(out), __float_as_uint(m));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Shared pieces of the quantizers
+// ---------------------------------------------------------------------------
+struct ScaleOut {
+  uint8_t* p;
+  uint32_t blocks_per_row;  // K / group
+  uint32_t Cp;              // padded columns (swizzled) = ceil4(blocks_per_row)
+  bool swizzled;
+  __device__ __forceinline__ void store(uint32_t block, uint32_t byte) const {
+    if (!swizzled) {
+      p[block] = (uint8_t)byte;
+    } else {
+      uint32_t r = block / blocks_per_row, c = block - r * blocks_per_row;
+      p[swizzled_offset(r, c, Cp)] = (uint8_t)byte;
+    }
+  }
+};
+
+// Zero the padding bytes of a 128x4-tile scale buffer: rows [rows, Rp) and
+// columns [bpr, Cp) ("mlx 0.30.7.2 -> 0.30.7.6" diff, page 8, qqmm_utils.h,
+// pad_and_swizzle_scales: out-of-bounds values must be zero).
+__device__ __forceinline__ void zero_scale_padding(const ScaleOut& so, uint32_t rows) {
+  if (!so.swizzled) return;
+  const uint32_t Rp = (rows + 127u) & ~127u;
+  const uint32_t tid = blockIdx.x * blockDim.x + threadIdx.x, nthr = gridDim.x * blockDim.x;
+  const uint32_t n1 = (Rp - rows) * so.Cp;
+  for (uint32_t i = tid; i < n1; i += nthr) {
+    uint32_t r = rows + i / so.Cp, c = i % so.Cp;
+    so.p[swizzled_offset(r, c, so.Cp)] = 0;
+  }
+  const uint32_t pc = so.Cp - so.blocks_per_row;
+  if (pc == 0) return;
+  const uint32_t n2 = rows * pc;
+  for (uint32_t i = tid; i < n2; i += nthr) {
+    uint32_t r = i / pc, c = so.blocks_per_row + i % pc;
+    so.p[swizzled_offset(r, c, so.Cp)] = 0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a2-a4: NVFP4 two-level quantize ("mlx 0.30.7.2 -> 0.30.7.6" diff, page 7,
+// fp_quantize.cu, fp_quantize_rowwise with global scale):
+//   E = 2688 / g (1 without g);  per 16-block: a = max|x|;
+//   s = e4m3_rne_satfinite((a / 6) * E);  k = E / f8(s);
+//   q_i = e2m1_rne_satfinite(x_i * k);  a block with f8(s) == 0 stores 0 codes.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kEwThreads) k_nvfp4_quantize(
+    const T* __restrict__ x, uint32_t n_half, const float* __restrict__ g,
+    uint32_t* __restrict__ codes, ScaleOut so, uint32_t rows) {
+  const float E = g ? kGlobalEncode / __ldg(g) : 1.0f;
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (uint32_t base = warp * 32u * kUnroll; base < n_half; base += nwarps * 32u * kUnroll) {
+    float v[kUnroll][8];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const uint32_t hb = base + u * 32u + lane;
+      if (hb < n_half) {
+        load8<T>(x + (size_t)hb * 8, v[u]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const uint32_t hb = base + u * 32u + lane;
+      float a = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[u][j]));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+      float t = a / kE2M1Max;
+      t = t * E;
+      const uint32_t s = f32_to_e4m3(t);
+      const float fs = e4m3_to_f32(s);
+      uint32_t w = 0;
+      if (fs != 0.0f) {
+        const float k = E / fs;
+        float q[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) q[j] = v[u][j] * k;
+        w = f32x8_to_e2m1x8(q);
+      }
+      if (hb < n_half) {
+        codes[hb] = w;
+        if ((lane & 1u) == 0) so.store(hb >> 1, s);
+      }
+    }
+  }
+  zero_scale_padding(so, rows);
+}
+
+// ---------------------------------------------------------------------------
+// a11: MXFP8 quantize (fp_quantize_rowwise with bits 8 and the e8m0 scale;
+// the scale is rounded up, as the mlxcel note on the "[Metal] global scale
+// for qmm" page records for CUDA):  per 32-block: v = max|x| / 448;
+//   s = ue8m0 rounded up (v);  k = 1 / 2^(s-127);  q_i = e4m3_rne_satfinite(x_i * k)
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kEwThreads) k_mxfp8_quantize(
+    const T* __restrict__ x, uint32_t n_half, uint32_t* __restrict__ codes, ScaleOut so,
+    uint32_t rows) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (uint32_t base = warp * 32u * kUnroll; base < n_half; base += nwarps * 32u * kUnroll) {
+    float v[kUnroll][8];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const uint32_t hb = base + u * 32u + lane;
+      if (hb < n_half) {
+        load8<T>(x + (size_t)hb * 8, v[u]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const uint32_t hb = base + u * 32u + lane;
+      float a = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[u][j]));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+      const float sv = a / kE4M3Max;
+      const uint32_t s = f32_to_ue8m0_rp(sv);
+      const float k = 1.0f / ue8m0_to_f32(s);
+      const uint32_t w0 = f32x4_to_e4m3x4(v[u][0] * k, v[u][1] * k, v[u][2] * k, v[u][3] * k);
+      const uint32_t w1 = f32x4_to_e4m3x4(v[u][4] * k, v[u][5] * k, v[u][6] * k, v[u][7] * k);
+      if (hb < n_half) {
+        reinterpret_cast<uint2*>(codes)[hb] = make_uint2(w0, w1);
+        if ((lane & 3u) == 0) so.store(hb >> 2, s);
+      }
+    }
+  }
+  zero_scale_padding(so, rows);
+}
+
+// Scale byte of block `block` from a LINEAR or 128x4-tile buffer.
+struct ScaleIn {
+  const uint8_t* p;
+  uint32_t blocks_per_row;
+  uint32_t Cp;
+  bool swizzled;
+  __device__ __forceinline__ uint32_t load(uint32_t block) const {
+    if (!swizzled) return __ldg(p + block);
+    uint32_t r = block / blocks_per_row, c = block - r * blocks_per_row;
+    return __ldg(p + swizzled_offset(r, c, Cp));
+  }
+};
+
+// ---------------------------------------------------------------------------
+// a5: NVFP4 dequantize ("mlx 0.30.7.2 -> 0.30.7.6" diff, page 7,
+// fp_dequantize with global scale): w_hat = T(e2m1(q) * (f8(s) * (g / 2688))).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kEwThreads) k_nvfp4_dequantize(
+    const uint32_t* __restrict__ codes, ScaleIn si, const float* __restrict__ g,
+    uint32_t n_half, T* __restrict__ out) {
+  const float d = g ? __ldg(g) / kGlobalEncode : 1.0f;
+  const uint32_t tid = blockIdx.x * blockDim.x + threadIdx.x, nthr = gridDim.x * blockDim.x;
+  for (uint32_t hb = tid; hb < n_half; hb += nthr) {
+    const uint32_t w = __ldg(codes + hb);
+    const float sd = e4m3_to_f32(si.load(hb >> 1)) * d;
+    float v[8];
+    e2m1x8_to_f32(w, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = v[j] * sd;
+    store8<T>(out + (size_t)hb * 8, v);
+  }
+}
+
+// MXFP8 dequantize ("mlx 0.30.7.2 -> 0.30.7.6" diff, page 8, ops.cpp
+// fp_dequantize fallback, e8m0 branch): w_hat = T(e4m3(q) * 2^(s-127)).
+template <typename T>
+__global__ void __launch_bounds__(kEwThreads) k_mxfp8_dequantize(
+    const uint32_t* __restrict__ codes, ScaleIn si, uint32_t n_half, T* __restrict__ out) {
+  const uint32_t tid = blockIdx.x * blockDim.x + threadIdx.x, nthr = gridDim.x * blockDim.x;
+  for (uint32_t hb = tid; hb < n_half; hb += nthr) {
+    const uint2 w = __ldg(reinterpret_cast<const uint2*>(codes) + hb);
+    const float sc = ue8m0_to_f32(si.load(hb >> 2));
+    float a[4], b[4], v[8];
+    e4m3x4_to_f32(w.x, a);
+    e4m3x4_to_f32(w.y, b);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[j] = a[j] * sc;
+      v[4 + j] = b[j] * sc;
+    }
+    store8<T>(out + (size_t)hb * 8, v);
+  }
+}
+
+// Standalone LINEAR -> 128x4-tile re-layout of a [rows, cols] scale matrix,
+// with zero padding ("mlx 0.30.7" diff, page 71, qqmm_utils.cu swizzle_scales).
+// One thread per output byte: every byte of the padded buffer is written.
+__global__ void __launch_bounds__(kEwThreads) k_swizzle_scales(
+    const uint8_t* __restrict__ lin, uint32_t rows, uint32_t cols, uint32_t Rp, uint32_t Cp,
+    uint8_t* __restrict__ swz) {
+  const uint32_t tid = blockIdx.x * blockDim.x + threadIdx.x, nthr = gridDim.x * blockDim.x;
+  const uint32_t total = Rp * Cp;
+  for (uint32_t o = tid; o < total; o += nthr) {
+    // invert the tile offset: o = (tile * 512) + (r%32)*16 + ((r%128)/32)*4 + c%4
+    const uint32_t tile = o >> 9, in = o & 511u;
+    const uint32_t rb = tile / (Cp >> 2), cb = tile - rb * (Cp >> 2);
+    const uint32_t r = rb * 128u + ((in >> 2) & 3u) * 32u + (in >> 4);
+    const uint32_t c = cb * 4u + (in & 3u);
+    swz[o] = (r < rows && c < cols) ? __ldg(lin + (size_t)r * cols + c) : (uint8_t)0;
+  }
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,213 @@
+"""Thin Python binding of libnvfp4.so (include/nvfp4.h).
+
+Argument marshalling only: every step of the method runs in the library's
+CUDA kernels.  PyTorch provides device memory and the current stream.  There
+is no CPU fallback: if the shared library is missing or the device is not a
+B200 (sm_100), calls raise.
+
+The raw C functions are available as ``lib().<name>`` (ctypes), with the same
+names and arguments as the header; the wrappers below allocate outputs with
+torch and pass device pointers plus ``torch.cuda.current_stream()``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE_INDEX = range(6)
+DT = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+LAYOUT = {"linear": 0, "swizzled": 1}
+MODE = {"nvfp4": 0, "mxfp8": 1}
+
+# (name, restype, argtypes) of every symbol declared in include/nvfp4.h
+_P, _I64, _I, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = [
+    ("nvfp4_status_string", ctypes.c_char_p, [_I]),
+    ("nvfp4_last_error_message", ctypes.c_char_p, []),
+    ("nvfp4_check_device_errors", _I, [_P]),
+    ("nvfp4_scale_bytes", _SZ, [_I64, _I64, _I]),
+    ("nvfp4_amax", _I, [_P, _I, _I64, _P, _P]),
+    ("nvfp4_quantize", _I, [_P, _I, _I64, _I64, _P, _P, _P, _I, _P]),
+    ("nvfp4_dequantize", _I, [_P, _P, _I, _I64, _I64, _P, _P, _I, _P]),
+    ("mxfp8_quantize", _I, [_P, _I, _I64, _I64, _P, _P, _I, _P]),
+    ("mxfp8_dequantize", _I, [_P, _P, _I, _I64, _I64, _P, _I, _P]),
+    ("nvfp4_swizzle_scales", _I, [_P, _I64, _I64, _P, _P]),
+    ("qqmm", _I, [_I, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
+    ("qmv", _I, [_P, _I, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    ("gather_qmm", _I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    ("gather_qmm_workspace_size", _SZ, [_I64, _I64, _I64]),
+]
+
+_lib = None
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{message} (status {status})")
+        self.status = status
+
+
+def lib():
+    """The loaded libnvfp4.so (ctypes.CDLL) with argument types set."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is not built; run `python -m mxfp8_block_scaled_nvfp4_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, res, args in SIGNATURES:
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != OK:
+        L = lib()
+        msg = L.nvfp4_last_error_message().decode() or L.nvfp4_status_string(status).decode()
+        raise Nvfp4Error(status, msg)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("tensors must be CUDA tensors (no CPU fallback)")
+            if not t.is_contiguous():
+                raise ValueError("tensors must be contiguous")
+
+
+def check_device_errors():
+    _check(lib().nvfp4_check_device_errors(_stream()))
+
+
+def scale_bytes(rows: int, cols: int, layout: str) -> int:
+    return int(lib().nvfp4_scale_bytes(rows, cols, LAYOUT[layout]))
+
+
+def scale_shape(rows: int, cols: int, layout: str):
+    if layout == "linear":
+        return (rows, cols)
+    return ((rows + 127) // 128 * 128, (cols + 3) // 4 * 4)
+
+
+# ---------------------------------------------------------------------------
+def amax(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """fp32 [1] tensor holding max |x| (the global scale g)."""
+    _need_cuda(x)
+    out = torch.empty(1, dtype=torch.float32, device=x.device) if out is None else out
+    _check(lib().nvfp4_amax(_ptr(x), DT[x.dtype], x.numel(), _ptr(out), _stream()))
+    return out
+
+
+def nvfp4_quantize(x: torch.Tensor, g: torch.Tensor | None = None, layout: str = "linear",
+                   codes: torch.Tensor | None = None, scales: torch.Tensor | None = None):
+    """(codes uint32 [rows, K/8] viewed as int32, scales uint8) of a 2-D x."""
+    _need_cuda(x, g)
+    rows, K = x.shape
+    if codes is None:
+        codes = torch.empty(rows, K // 8, dtype=torch.int32, device=x.device)
+    if scales is None:
+        scales = torch.empty(scale_shape(rows, K // 16, layout), dtype=torch.uint8, device=x.device)
+    _check(lib().nvfp4_quantize(_ptr(x), DT[x.dtype], rows, K, _ptr(g), _ptr(codes), _ptr(scales),
+                                LAYOUT[layout], _stream()))
+    return codes, scales
+
+
+def nvfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, g: torch.Tensor | None = None,
+                     layout: str = "linear", dtype=torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
+    _need_cuda(codes, scales, g)
+    rows, K = codes.shape[0], codes.shape[1] * 8
+    if out is None:
+        out = torch.empty(rows, K, dtype=dtype, device=codes.device)
+    dtype = out.dtype
+    _check(lib().nvfp4_dequantize(_ptr(codes), _ptr(scales), LAYOUT[layout], rows, K, _ptr(g), _ptr(out),
+                                  DT[dtype], _stream()))
+    return out
+
+
+def mxfp8_quantize(x: torch.Tensor, layout: str = "linear", codes=None, scales=None):
+    _need_cuda(x)
+    rows, K = x.shape
+    if codes is None:
+        codes = torch.empty(rows, K // 4, dtype=torch.int32, device=x.device)
+    if scales is None:
+        scales = torch.empty(scale_shape(rows, K // 32, layout), dtype=torch.uint8, device=x.device)
+    _check(lib().mxfp8_quantize(_ptr(x), DT[x.dtype], rows, K, _ptr(codes), _ptr(scales), LAYOUT[layout],
+                                _stream()))
+    return codes, scales
+
+
+def mxfp8_dequantize(codes, scales, layout: str = "linear", dtype=torch.bfloat16) -> torch.Tensor:
+    _need_cuda(codes, scales)
+    rows, K = codes.shape[0], codes.shape[1] * 4
+    out = torch.empty(rows, K, dtype=dtype, device=codes.device)
+    _check(lib().mxfp8_dequantize(_ptr(codes), _ptr(scales), LAYOUT[layout], rows, K, _ptr(out), DT[dtype],
+                                  _stream()))
+    return out
+
+
+def swizzle_scales(lin: torch.Tensor) -> torch.Tensor:
+    _need_cuda(lin)
+    rows, cols = lin.shape
+    out = torch.empty(scale_shape(rows, cols, "swizzled"), dtype=torch.uint8, device=lin.device)
+    _check(lib().nvfp4_swizzle_scales(_ptr(lin), rows, cols, _ptr(out), _stream()))
+    return out
+
+
+def qqmm(a_codes, a_scales, b_codes, b_scales, K: int, mode: str = "nvfp4", g_x=None, g_w=None,
+         out_dtype=torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
+    """y [M, N] = x_hat . w_hat^T from quantized operands with SWIZZLED scales."""
+    _need_cuda(a_codes, a_scales, b_codes, b_scales, g_x, g_w)
+    M, N = a_codes.shape[0], b_codes.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=a_codes.device)
+    _check(lib().qqmm(MODE[mode], M, N, K, _ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales),
+                      _ptr(g_x), _ptr(g_w), _ptr(out), DT[out.dtype], _stream()))
+    return out
+
+
+def qmv(x: torch.Tensor, w_codes, w_scales, g_x=None, g_w=None, out=None) -> torch.Tensor:
+    """y [M, N] (x's dtype) = x_hat . w_hat^T, M <= 8, w pre-quantized (LINEAR scales)."""
+    _need_cuda(x, w_codes, w_scales, g_x, g_w)
+    M, K = x.shape
+    N = w_codes.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=x.dtype, device=x.device)
+    _check(lib().qmv(_ptr(x), DT[x.dtype], _ptr(g_x), _ptr(w_codes), _ptr(w_scales), _ptr(g_w), M, N, K,
+                     _ptr(out), _stream()))
+    return out
+
+
+def gather_qmm_workspace_size(T: int, topk: int, E: int) -> int:
+    return int(lib().gather_qmm_workspace_size(T, topk, E))
+
+
+def gather_qmm(x, w_codes, w_scales, g, idx, workspace=None, out=None) -> torch.Tensor:
+    """y [T, topk, N] bf16; w_codes [E, N, K/8], w_scales LINEAR [E, N, K/16]."""
+    _need_cuda(x, w_codes, w_scales, g, idx, workspace)
+    T, K = x.shape
+    topk = idx.shape[1]
+    E, N = w_codes.shape[0], w_codes.shape[1]
+    if workspace is None:
+        workspace = torch.empty(gather_qmm_workspace_size(T, topk, E), dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty(T, topk, N, dtype=torch.bfloat16, device=x.device)
+    _check(lib().gather_qmm(_ptr(x), _ptr(w_codes), _ptr(w_scales), _ptr(g), _ptr(idx), T, topk, E, N, K,
+                            _ptr(out), _ptr(workspace), workspace.numel(), _stream()))
+    return out

@@ -321,6 +321,24 @@ void orc_nvfp4_decode_exact(const uint32_t* codes, const uint8_t* scales,
   }
 }
 
+/* Weight values of the qmv route: e2m1(q) times the per-block decoded scale
+ * as the dequantize kernel forms it in fp32 (f8(s) * d(g), one rounding),
+ * the product exact in float64.  The weight is not rounded to an output
+ * type on that route ([P4] "The fix": the global scale goes on each block
+ * scale; the sum is not rescaled). */
+void orc_nvfp4_decode_blockscale(const uint32_t* codes, const uint8_t* scales,
+                                 int64_t rows, int64_t K, const float* g,
+                                 double* out) {
+  const int64_t nb = K / 16;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t k = 0; k < K; ++k) {
+      int64_t idx = r * K + k;
+      int q = (codes[idx / 8] >> (4 * (idx % 8))) & 15;
+      out[idx] = orc_e2m1_value(q) * (double)orc_nvfp4_block_scale(scales[r * nb + k / 16], g);
+    }
+  }
+}
+
 /* ------------------------------------------------------------------------ */
 /* 7. Quantize-dequantize x_hat ([P2] fp_quantize_dequantize; used by the    */
 /*    M=1 qqmm route before fp_qmv): quantize as in 5, decode as in 6.       */

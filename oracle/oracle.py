@@ -81,6 +81,7 @@ def _L():
                 "orc_nvfp4_block_scale": (ctypes.c_float, [ctypes.c_uint8, P]),
                 "orc_nvfp4_dequantize": (None, [P, P, I64, I64, P, P, I]),
                 "orc_nvfp4_decode_exact": (None, [P, P, I64, I64, P, P]),
+                "orc_nvfp4_decode_blockscale": (None, [P, P, I64, I64, P, P]),
                 "orc_nvfp4_quantize_dequantize": (None, [P, I, I64, I64, P, P]),
                 "orc_mxfp8_quantize": (None, [P, I, I64, I64, P, P]),
                 "orc_mxfp8_dequantize": (None, [P, P, I64, I64, P, I]),
@@ -314,14 +315,27 @@ def qqmm(a_codes, a_scales, b_codes, b_scales, mode="nvfp4", g_x=None, g_w=None,
 # --------------------------------------------------------------------------
 # a6-a7: qmv (small-M route of qqmm with pre-quantized w)
 # --------------------------------------------------------------------------
+def nvfp4_decode_blockscale(codes, scales, g=None) -> np.ndarray:
+    """float64 e2m1(q) * fp32(f8(s) * d(g)) per element (exact product)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, K = codes.shape[0], codes.shape[1] * 8
+    out = np.empty((rows, K), dtype=np.float64)
+    gb, gp = _g(g)
+    _L().orc_nvfp4_decode_blockscale(_p(codes), _p(scales), rows, K, gp, _p(out))
+    return out
+
+
 def qmv(x, x_dt, g_x, w_codes, w_scales, g_w):
     """y = x_hat . w_hat^T for a small number of rows of x ([P2] qqmm.cpp M=1
     route: fp_quantize_dequantize then fp_qmv).  x_hat is x quantize-
-    dequantized with g_x, in x's type; w_hat is w dequantized with g_w into
-    x's type, the global scale applied to each block scale before the cast
-    ([P3] worked example; [P4] "The fix").  float64 sum, one rounding to T."""
+    dequantized with g_x, in x's type (materialized, as the kernel writes
+    it); w_hat = e2m1(q) * (f8(s) * g_w / 2688) with the block scale formed
+    in fp32 and the global scale on each block scale ([P4] "The fix"); the
+    weight is not rounded to T on this route.  float64 sum, one rounding
+    to T."""
     xh = to_f64(nvfp4_quantize_dequantize(x, x_dt, g_x), x_dt)
-    wh = to_f64(nvfp4_dequantize(w_codes, w_scales, g_w, x_dt), x_dt)
+    wh = nvfp4_decode_blockscale(w_codes, w_scales, g_w)
     y_ref = xh @ wh.T
     abs_ref = np.abs(xh) @ np.abs(wh).T
     return {"y_ref": y_ref, "abs_ref": abs_ref, "y": round_to(y_ref, x_dt)}

@@ -1,0 +1,110 @@
+"""The C-ABI library loads, exports every symbol include/nvfp4.h declares, and
+rejects bad arguments on the host (no GPU needed: argument checks run before
+any device call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from mxfp8_block_scaled_nvfp4_b200 import build, nvfp4
+    build.build()
+    return nvfp4.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"NVFP4_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for s in ["nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize", "mxfp8_quantize", "qqmm", "qmv",
+              "gather_qmm", "gather_qmm_workspace_size", "nvfp4_check_device_errors"]:
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    for s in declared_symbols():
+        assert hasattr(L, s), s
+
+
+def test_binding_signatures_cover_the_header():
+    from mxfp8_block_scaled_nvfp4_b200 import nvfp4
+    assert sorted(n for n, _, _ in nvfp4.SIGNATURES) == declared_symbols()
+
+
+def test_status_strings(L):
+    assert L.nvfp4_status_string(0) == b"ok"
+    assert b"invalid" in L.nvfp4_status_string(1)
+
+
+A = 0x10000  # a fake, 16-byte aligned device address: never dereferenced
+
+
+def msg(L):
+    return L.nvfp4_last_error_message().decode()
+
+
+def test_qqmm_requires_both_global_scales_or_neither(L):
+    st = L.qqmm(0, 128, 128, 256, A, A, A, A, A, None, A, 2, None)
+    assert st == 1
+    assert msg(L) == ("[qqmm] For nvfp4 mode, either both global_scale_x and global_scale_w "
+                      "must be provided, or neither.")
+    st = L.qqmm(0, 128, 128, 256, A, A, A, A, None, A, A, 2, None)
+    assert st == 1
+
+
+def test_global_scale_only_for_nvfp4(L):
+    st = L.qqmm(1, 128, 128, 256, A, A, A, A, A, A, A, 2, None)
+    assert st == 1 and "only supported for 'nvfp4'" in msg(L)
+
+
+def test_qqmm_K_multiple_of_32(L):
+    assert L.qqmm(0, 128, 128, 48, A, A, A, A, None, None, A, 2, None) == 1
+
+
+def test_quantize_group_divisibility_and_alignment(L):
+    assert L.nvfp4_quantize(A, 2, 4, 24, None, A, A, 0, None) == 1
+    assert "divisible by the quantization group size 16" in msg(L)
+    assert L.mxfp8_quantize(A, 2, 4, 48, A, A, 0, None) == 1
+    assert L.nvfp4_quantize(A + 8, 2, 4, 32, None, A, A, 0, None) == 1
+    assert "aligned" in msg(L)
+
+
+def test_bad_dtype_and_layout(L):
+    assert L.nvfp4_quantize(A, 7, 4, 32, None, A, A, 0, None) == 2
+    assert L.nvfp4_quantize(A, 2, 4, 32, None, A, A, 5, None) == 1
+    assert L.nvfp4_dequantize(A, A, 0, 4, 32, None, A, 9, None) == 2
+
+
+def test_qmv_bounds(L):
+    assert L.qmv(A, 2, None, A, A, None, 9, 64, 256, A, None) == 1  # M > 8
+    assert L.qmv(A, 2, A, A, A, None, 1, 64, 256, A, None) == 1  # one global scale only
+    assert L.qmv(A, 2, None, A, A, None, 1, 64, 65536, A, None) == 2  # x_hat too large
+
+
+def test_gather_workspace_and_shape_checks(L):
+    ws = L.gather_qmm_workspace_size(4096, 8, 64)
+    assert ws > 0
+    assert L.gather_qmm(A, A, A, A, A, 16, 2, 4, 64, 96, A, A, ws, None) == 1  # K % 64
+    assert L.gather_qmm(A, A, A, A, A, 16, 2, 4, 64, 128, A, A, 0, None) == 1  # workspace
+
+
+def test_scale_bytes(L):
+    assert L.nvfp4_scale_bytes(67, 16, 0) == 67 * 16
+    assert L.nvfp4_scale_bytes(67, 16, 1) == 128 * 16
+    assert L.nvfp4_scale_bytes(200, 5, 1) == 256 * 8
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    from mxfp8_block_scaled_nvfp4_b200 import nvfp4
+    with pytest.raises(ValueError):
+        nvfp4.amax(torch.ones(16))

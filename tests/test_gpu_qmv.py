@@ -1,0 +1,71 @@
+"""GPU parity of qmv (small-M route of qqmm with a pre-quantized NVFP4
+weight) against the oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from helpers import TORCH_DT, check_gemm_output, raw
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    from mxfp8_block_scaled_nvfp4_b200 import build, nvfp4
+    build.build()
+    return nvfp4
+
+
+def run_case(nv, orc, M, N, K, dt, use_g, seed):
+    from mxfp8_block_scaled_nvfp4_b200 import workloads
+    x = workloads.normal((M, K), 1.0, seed, TORCH_DT[dt])
+    w = workloads.normal((N, K), 0.02, seed + 1, TORCH_DT[dt])
+    xg, wg = x.cuda(), w.cuda()
+    g_x = nv.amax(xg) if use_g else None
+    g_w = nv.amax(wg) if use_g else None
+    wc, ws = nv.nvfp4_quantize(wg, g_w, "linear")
+    y = nv.qmv(xg, wc, ws, g_x, g_w)
+    # the oracle quantizes w itself (bit-exactness of that step is tested
+    # separately); its qmv uses its own codes
+    gx = None if g_x is None else g_x.item()
+    gw = None if g_w is None else g_w.item()
+    owc, ows = orc.nvfp4_quantize(raw(w), dt, gw)
+    assert np.array_equal(raw(wc), owc) and np.array_equal(raw(ws), ows)
+    r = orc.qmv(raw(x), dt, gx, owc, ows, gw)
+    return check_gemm_output(raw(y), r, dt, orc)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f16", "f32"])
+@pytest.mark.parametrize("M,N,K", [(1, 64, 256), (1, 200, 1056), (2, 130, 512), (3, 130, 512), (8, 257, 2048),
+                                   (1, 33, 32), (5, 1000, 4096)])
+@pytest.mark.parametrize("use_g", [True, False])
+def test_qmv_parity(nv, orc, dt, M, N, K, use_g):
+    run_case(nv, orc, M, N, K, dt, use_g, seed=M * 100 + N + K)
+
+
+def test_qmv_decode_gemv_full_size(nv, orc):
+    """The decode GEMV config: x [1,4096] bf16 N(0,1), W [14336,4096] bf16
+    N(0,0.02), g = amax; every output element compared."""
+    floor_count = run_case(nv, orc, 1, 14336, 4096, "bf16", True, seed=1)
+    assert floor_count < 14336 * 0.01
+
+
+def test_qmv_worked_example(nv):
+    """K = 4096, x = ones, codes 6, block scale 0.5, decode factor 0.1:
+    y = 1232.0 ("[Metal] global scale for qmm"); K = 96 gives bf16(28.8)."""
+    for K, want in [(4096, 1232.0), (96, 28.75)]:
+        x = torch.ones(1, K, dtype=torch.bfloat16).cuda()
+        wc = torch.full((2, K // 8), 0x77777777, dtype=torch.int32).cuda()
+        ws = torch.full((2, K // 16), 0x30, dtype=torch.uint8).cuda()
+        g_x = nv.amax(x)
+        g_w = torch.tensor([268.8], dtype=torch.float32).cuda()
+        y = nv.qmv(x, wc, ws, g_x, g_w)
+        assert torch.all(y.float() == want), (K, y)
+
+
+def test_qmv_rejects_K_not_multiple_of_32(nv):
+    x = torch.ones(1, 48, dtype=torch.bfloat16).cuda()
+    wc = torch.zeros(4, 6, dtype=torch.int32).cuda()
+    ws = torch.zeros(4, 3, dtype=torch.uint8).cuda()
+    with pytest.raises(nv.Nvfp4Error):
+        nv.qmv(x, wc, ws)

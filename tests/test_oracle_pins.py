@@ -72,8 +72,9 @@ def test_worked_example_dequantize(orc):
 
 
 def test_worked_example_qmv_and_scale_after(orc):
-    """qmv with x = ones: y = 1232.0 (scale inside the dequantization);
-    scaling the bf16 product of the unscaled weights gives 1228.8000488."""
+    """qmv with x = ones: the bf16 result is 1232.0; scaling the bf16 product
+    of the unscaled weights by the fp32 decode factor gives 1228.8000488
+    (the page's "scale after")."""
     G = golden("worked_example_global_scale.txt")
     K = int(G["K"])
     g = float(np.float32(float(G["decode_factor"]) * 2688.0))
@@ -112,15 +113,29 @@ def test_worked_example_in_gather_layout(orc):
 
 
 def test_scale_inside_differs_from_scale_after_at_K96(orc):
-    """Derived from the worked example: with K = 96, y = 96 * 0.30078125 =
-    28.875 exactly, while scaling after the matmul gives bf16(28.8) = 28.75.
-    This separates the two orders even in a bf16 result."""
+    """Derived from the worked example, in the gather_qmm layout where the
+    weight is rounded to bf16 before the matmul: with K = 96, y = 96 *
+    0.30078125 = 28.875 exactly, while scaling after the matmul gives
+    bf16(28.8) = 28.75.  This separates the two orders in a bf16 result."""
+    K = 96
+    g = np.array([np.float32(268.8)], dtype=np.float32)
+    codes, scales = _worked_example_weights(orc, K, None)
+    x = bf16(np.ones((1, K)))
+    r = orc.gather_qmm(x, codes[None], scales[None], g, np.zeros((1, 1), dtype=np.int32))
+    assert bf16_value(r["y"])[0, 0, 0] == 28.875
+
+
+def test_qmv_does_not_round_the_weight(orc):
+    """qmv keeps w_hat = e2m1 * fp32(f8(s) * d): K = 96, x = ones gives
+    96 * 6 * fp32(0.5 * fp32(268.8/2688)) = 28.799998..., bf16 28.75."""
     K = 96
     g = float(np.float32(268.8))
     codes, scales = _worked_example_weights(orc, K, g)
     x = bf16(np.ones((1, K)))
     r = orc.qmv(x, "bf16", 1.0, codes, scales, g)
-    assert bf16_value(r["y"])[0, 0] == 28.875
+    sd = np.float32(np.float32(0.5) * (np.float32(g) / np.float32(2688.0)))
+    assert r["y_ref"][0, 0] == 96 * 6 * float(sd)
+    assert bf16_value(r["y"])[0, 0] == 28.75
 
 
 # ---------------------------------------------------------------------------
@@ -340,13 +355,14 @@ def test_tiny_workload_oracle_runs(orc):
 # Mutation checks: plant a mistake in a copy of an oracle step, see a pin fail
 # ---------------------------------------------------------------------------
 def test_mutation_global_scale_on_the_sum_fails_K96_pin(orc):
-    """Mistake: decode w without g, apply g to the bf16 result of the sum."""
+    """Mistake (gather_qmm): decode w without g into bf16, apply g to the
+    bf16 result of the sum."""
     K = 96
-    g = float(np.float32(268.8))
-    codes, scales = _worked_example_weights(orc, K, g)
+    g = np.array([np.float32(268.8)], dtype=np.float32)
+    codes, scales = _worked_example_weights(orc, K, None)
     x = bf16(np.ones((1, K)))
-    r0 = orc.qmv(x, "bf16", 1.0, codes, scales, None)
-    mutated = orc.round_to(np.array([r0["y_ref"][0, 0] * float(np.float32(g) / np.float32(2688.0))]), "bf16")
+    r0 = orc.gather_qmm(x, codes[None], scales[None], None, np.zeros((1, 1), dtype=np.int32))
+    mutated = orc.round_to(np.array([r0["y_ref"][0, 0, 0] * float(g[0] / np.float32(2688.0))]), "bf16")
     assert bf16_value(mutated)[0] != 28.875  # the pin catches it
 
 
