@@ -78,10 +78,9 @@ __device__ __forceinline__ void load8<__half>(const __half* p, float (&v)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
-    float2 f = __half22float2(h);
-    v[2 * i] = f.x;
-    v[2 * i + 1] = f.y;
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(v[2 * i]), "=f"(v[2 * i + 1])
+        : "r"(w[i]));
   }
 }
 
@@ -95,26 +94,29 @@ __device__ __forceinline__ void store8<float>(float* p, const float (&v)[8]) {
   reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
 }
 
+// Two fp32 values rounded (RNE) to a packed bf16x2 / f16x2 word, `lo` in
+// the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 template <>
 __device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16* p, const float (&v)[8]) {
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-    w[i] = *reinterpret_cast<uint32_t*>(&h);
-  }
-  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                            pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
 }
 
 template <>
 __device__ __forceinline__ void store8<__half>(__half* p, const float (&v)[8]) {
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
-    w[i] = *reinterpret_cast<uint32_t*>(&h);
-  }
-  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(p) = make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]),
+                                            pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
 }
 
 // ---------------------------------------------------------------------------
@@ -137,10 +139,15 @@ __device__ __forceinline__ uint32_t f32_to_ue8m0_rp(float v) {
 
 // Value of an e4m3 byte (exact: e4m3 is a subset of fp16).
 __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
-  uint32_t h2;
-  uint16_t in = (uint16_t)(b & 0xFFu);
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
-  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+  float f;
+  asm("{\n\t.reg .b16 in, l, h;\n\t.reg .b32 p;\n\t"
+      "cvt.u16.u32 in, %1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 p, in;\n\t"
+      "mov.b32 {l, h}, p;\n\t"
+      "cvt.f32.f16 %0, l;\n\t}"
+      : "=f"(f)
+      : "r"(b & 0xFFu));
+  return f;
 }
 
 // Value of a ue8m0 byte: 2^(b-127) (b = 0 gives the fp32 subnormal 2^-127).
@@ -173,36 +180,45 @@ __device__ __forceinline__ uint32_t f32x4_to_e4m3x4(float a, float b, float c, f
   return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
+// Two e2m1 codes in the low byte of `b` to fp32 values (exact).  The byte
+// reaches the .b8 operand of the conversion through cvt.u8.u32.
+__device__ __forceinline__ void e2m1x2_to_f32(uint32_t b, float& lo, float& hi) {
+  asm("{\n\t.reg .b8 q;\n\t.reg .b16 l, h;\n\t.reg .b32 p;\n\t"
+      "cvt.u8.u32 q, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 p, q;\n\t"
+      "mov.b32 {l, h}, p;\n\t"
+      "cvt.f32.f16 %0, l;\n\t"
+      "cvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(b));
+}
+
 // Eight e2m1 codes (element i in bits 4i..4i+3) to their values.
 __device__ __forceinline__ void e2m1x8_to_f32(uint32_t codes, float (&v)[8]) {
-  uint32_t h[4];
-  asm("{\n\t"
-      ".reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t"
-      "}"
-      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
-      : "r"(codes));
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
-    v[2 * i] = f.x;
-    v[2 * i + 1] = f.y;
-  }
+  for (int i = 0; i < 4; ++i) e2m1x2_to_f32((codes >> (8 * i)) & 0xFFu, v[2 * i], v[2 * i + 1]);
+}
+
+// Value of a 4-bit e2m1 code by arithmetic: the magnitude bits placed at
+// fp32 bits 22-24 read as 2^-126 times the e2m1 value (code 1 lands on the
+// subnormal 2^-127 = 0.5 * 2^-126), the sign at bit 31; one exact multiply.
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  return __uint_as_float(((c & 8u) << 28) | ((c & 7u) << 22)) * 0x1p126f;
 }
 
 // Four e4m3 bytes (element i in byte i) to their values.
 __device__ __forceinline__ void e4m3x4_to_f32(uint32_t codes, float (&v)[4]) {
-  uint32_t h0, h1;
-  uint16_t lo = (uint16_t)(codes & 0xFFFFu), hi = (uint16_t)(codes >> 16);
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h0) : "h"(lo));
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h1) : "h"(hi));
-  float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h0));
-  float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    asm("{\n\t.reg .b16 in, l, h;\n\t.reg .b32 p;\n\t"
+        "cvt.u16.u32 in, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 p, in;\n\t"
+        "mov.b32 {l, h}, p;\n\t"
+        "cvt.f32.f16 %0, l;\n\t"
+        "cvt.f32.f16 %1, h;\n\t}"
+        : "=f"(v[2 * i]), "=f"(v[2 * i + 1])
+        : "r"((codes >> (16 * i)) & 0xFFFFu));
+  }
 }
 
 // ---------------------------------------------------------------------------

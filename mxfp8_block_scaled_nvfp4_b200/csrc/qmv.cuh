@@ -32,25 +32,6 @@ constexpr int kQmvThreads = 512;
 constexpr int kQmvMaxM = 8;
 constexpr int kQmvCH = 4;  // 128-bit chunks per lane per unit
 
-// Two e2m1 codes in the low byte of `b` to fp32 values (exact).
-__device__ __forceinline__ void e2m1x2_to_f32(uint32_t b, float& lo, float& hi) {
-  asm("{\n\t.reg .b8 q;\n\t.reg .b16 l, h;\n\t.reg .b32 p;\n\t"
-      "cvt.u8.u32 q, %2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 p, q;\n\t"
-      "mov.b32 {l, h}, p;\n\t"
-      "cvt.f32.f16 %0, l;\n\t"
-      "cvt.f32.f16 %1, h;\n\t}"
-      : "=f"(lo), "=f"(hi)
-      : "r"(b));
-}
-
-// Value of a 4-bit e2m1 code by arithmetic: the magnitude bits placed at
-// fp32 bits 22-24 read as 2^-126 times the e2m1 value (code 1 lands on the
-// subnormal 2^-127 = 0.5 * 2^-126), the sign at bit 31; one exact multiply.
-__device__ __forceinline__ float e2m1_value(uint32_t c) {
-  return __uint_as_float(((c & 8u) << 28) | ((c & 7u) << 22)) * 0x1p126f;
-}
-
 // fp32 index of element k of row m in the swizzled x_hat layout.
 __device__ __forceinline__ uint32_t xs_index(uint32_t m, uint32_t K, uint32_t k) {
   const uint32_t c = k >> 5, seg = (k >> 2) & 7u;
