@@ -486,10 +486,12 @@ def run_ours(args):
     time.sleep(0.3)
     torch.cuda.synchronize()
     s_all, e_all = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("timed")
     s_all.record()
     for _ in range(args.steps):
         step(True)
     e_all.record()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     clocks = clk.stop()
     barrier(world)
