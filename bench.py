@@ -351,11 +351,20 @@ def barrier(world):
 
 
 def max_over_ranks(world, v):
+    """Largest value of `v` over all ranks (device timings: the slowest rank
+    sets the job's time).  Works on NCCL (CUDA tensor) and gloo (CPU)."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job(world, work_per_rank, ms_slowest):
+    """Weak scaling: every rank solves its own problem of `work_per_rank`
+    units; the job's throughput is all ranks' work over the slowest time."""
+    return world * work_per_rank / ms_slowest
 
 
 def e2e_prefill(nv, row, steps):
@@ -514,7 +523,7 @@ def run_ours(args):
     if e2e is not None:
         # every rank solves its own problem: whole-job work / slowest rank
         ms_e2e = max_over_ranks(world, e2e.pop("ms"))
-        e2e = {"value": world * e2e.pop("work") / ms_e2e, **e2e, "ms_per_step": ms_e2e}
+        e2e = {"value": whole_job(world, e2e.pop("work"), ms_e2e), **e2e, "ms_per_step": ms_e2e}
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
