@@ -187,6 +187,32 @@ NVFP4_API nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const 
 
 NVFP4_API size_t gather_qmm_workspace_size(int64_t T, int64_t topk, int64_t E);
 
+/* gather_qmm without a workspace argument; the pages have no counterpart of
+ * this entry point.  It is for callers that cannot allocate device memory
+ * themselves: code embedded in a host program that owns the device memory
+ * budget and forbids growth after start-up, plugin code that has no handle
+ * on its host framework's allocator, or a latency-critical loop where an
+ * allocation could block on the device.  It computes exactly what
+ * gather_qmm computes, with the same arguments minus the workspace.
+ *
+ * Scratch: a 1 MiB array inside the library (a static device variable,
+ * 256-byte aligned), present on every GPU that loads the library until the
+ * process exits.  Calls whose gather_qmm_workspace_size(T, topk, E) exceeds
+ * 1 MiB are rejected with NVFP4_ERR_UNSUPPORTED (e.g. T = 4096 tokens, top-8,
+ * 64 experts needs about 135 KB).  The call allocates nothing: no
+ * cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  All calls on a device share the
+ * one array, which keeps the previous call's contents (each call rewrites
+ * every entry it reads, so nothing has to be cleared); two calls whose
+ * kernels overlap on the GPU -- on different streams, or from different
+ * host threads -- race on it and must be serialized by the caller. */
+NVFP4_API nvfp4_status gather_qmm_noalloc(const void* x, const uint32_t* w_codes, const uint8_t* w_scales,
+                                          const float* g, const int32_t* idx, int64_t T, int64_t topk,
+                                          int64_t E, int64_t N, int64_t K, void* y, nvfp4_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

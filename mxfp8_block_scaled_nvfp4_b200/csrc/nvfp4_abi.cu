@@ -19,6 +19,14 @@
 
 using namespace nvfp4;
 
+// Scratch of gather_qmm_noalloc: a fixed device array that the library owns
+// for the life of the process (1 MiB on every GPU that loads the library).
+// Host code must not pass the symbol itself to a kernel -- on the host it
+// only names the array; the device address comes from
+// cudaGetSymbolAddress, looked up once per device (see noalloc_scratch).
+static constexpr size_t kNoAllocScratchBytes = (size_t)1 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
 namespace {
 
 thread_local char t_msg[512] = "";
@@ -376,6 +384,48 @@ nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const uint8_t* w
   if (T * N == 0) return ok();
   return gather_qmm_launch(x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, workspace, d.sm_count, stream, t_msg,
                            sizeof(t_msg));
+}
+
+// Device address of g_noalloc_scratch on the current device, resolved on
+// the first call per device (with that device current) and cached.
+static nvfp4_status noalloc_scratch(void** out) {
+  static void* addr[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(NVFP4_ERR_CUDA, "[gather_qmm_noalloc] cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(NVFP4_ERR_UNSUPPORTED, "[gather_qmm_noalloc] device ordinal %d", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(NVFP4_ERR_CUDA, "[gather_qmm_noalloc] cudaGetSymbolAddress of the static scratch failed: %s",
+                  cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return NVFP4_OK;
+}
+
+nvfp4_status gather_qmm_noalloc(const void* x, const uint32_t* w_codes, const uint8_t* w_scales, const float* g,
+                                const int32_t* idx, int64_t T, int64_t topk, int64_t E, int64_t N, int64_t K,
+                                void* y, nvfp4_stream_t stream) {
+  if (T < 0 || topk < 1 || E < 1 || T * topk > (1 << 30) || E > (1 << 20))
+    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm_noalloc] bad shape");
+  const size_t need = gather_workspace_bytes(T, topk, E);
+  if (need > kNoAllocScratchBytes)
+    return fail(NVFP4_ERR_UNSUPPORTED,
+                "[gather_qmm_noalloc] T=%lld, topk=%lld, E=%lld needs %zu bytes of scratch; the static scratch "
+                "holds %zu bytes (use gather_qmm with a caller-provided workspace)",
+                (long long)T, (long long)topk, (long long)E, need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  nvfp4_status st = noalloc_scratch(&scratch);
+  if (st != NVFP4_OK) return st;
+  // The routing kernel rewrites every scratch entry the grouped kernel reads
+  // (tile count, tile list, permutation), so nothing needs clearing between
+  // calls.
+  return gather_qmm(x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, scratch, kNoAllocScratchBytes, stream);
 }
 
 }  // extern "C"

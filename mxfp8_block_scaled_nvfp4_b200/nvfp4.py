@@ -41,6 +41,7 @@ SIGNATURES = [
     ("qmv", _I, [_P, _I, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     ("gather_qmm", _I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     ("gather_qmm_workspace_size", _SZ, [_I64, _I64, _I64]),
+    ("gather_qmm_noalloc", _I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P]),
 ]
 
 _lib = None
@@ -210,4 +211,20 @@ def gather_qmm(x, w_codes, w_scales, g, idx, workspace=None, out=None) -> torch.
         out = torch.empty(T, topk, N, dtype=torch.bfloat16, device=x.device)
     _check(lib().gather_qmm(_ptr(x), _ptr(w_codes), _ptr(w_scales), _ptr(g), _ptr(idx), T, topk, E, N, K,
                             _ptr(out), _ptr(workspace), workspace.numel(), _stream()))
+    return out
+
+
+def gather_qmm_noalloc(x, w_codes, w_scales, g, idx, out=None) -> torch.Tensor:
+    """gather_qmm using the library's own static scratch instead of a
+    workspace (for callers that cannot allocate device memory); see
+    include/nvfp4.h for its size limit and the rule that overlapping calls
+    must be serialized."""
+    _need_cuda(x, w_codes, w_scales, g, idx)
+    T, K = x.shape
+    topk = idx.shape[1]
+    E, N = w_codes.shape[0], w_codes.shape[1]
+    if out is None:
+        out = torch.empty(T, topk, N, dtype=torch.bfloat16, device=x.device)
+    _check(lib().gather_qmm_noalloc(_ptr(x), _ptr(w_codes), _ptr(w_scales), _ptr(g), _ptr(idx), T, topk, E, N, K,
+                                    _ptr(out), _stream()))
     return out
