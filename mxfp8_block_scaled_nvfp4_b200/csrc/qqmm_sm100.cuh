@@ -11,7 +11,8 @@
 // operand is rounded to a narrower type on this path, so it is equivalent to
 // decoding each block with its global scale.
 //
-// Kernel structure (one CTA per 128 x 256 output tile, 192 threads):
+// Kernel structure (persistent: one CTA per SM loops over 128 x 256 output
+// tiles; 320 threads):
 //   warp 0   TMA producer: per K stage, A codes [128 rows x 128 B] and B codes
 //            [256 rows x 128 B] as 128-byte-swizzled tiles, plus the scale
 //            tiles as plain bulk copies (the 128x4 scale-tile layout of the
@@ -22,8 +23,11 @@
 //            issues the block-scaled MMAs (M=128, N=256, K=64 NVFP4 / 32
 //            MXFP8 per instruction) into a 128 x 256 fp32 accumulator in TMEM;
 //            tcgen05.commit frees the stage when its MMAs are done.
-//   warps 2-5 epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
-//            32*(w%4)...), alpha, conversion, stores.
+//   warps 2-9 epilogue: two warps per TMEM lane quarter (warp w reads lanes
+//            32*(w%4)...), 128 accumulator columns each; they drain the
+//            accumulator into registers, release it to the MMA warp at once
+//            (so the next tile's MMAs start), then apply alpha, convert and
+//            store while the tensor core works on the next tile.
 // Every mbarrier wait is bounded; on timeout the kernel sets the device
 // error word (NVFP4_ERR_TIMEOUT through nvfp4_check_device_errors), drains,
 // frees its TMEM and exits.  No cluster multicast is used.
@@ -43,7 +47,8 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BKB = 128;  // bytes of K per row per stage (256 FP4 / 128 FP8 elements)
 constexpr int STAGES = 4;
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;  // producer, MMA, 8 epilogue warps
 constexpr int A_STAGE = BM * BKB;    // 16 KiB
 constexpr int B_STAGE = BN * BKB;    // 32 KiB
 constexpr int SFA_STAGE = 4 * 512;   // up to 4 scale tiles (NVFP4)
@@ -233,27 +238,41 @@ __device__ __forceinline__ void store_out<__half>(__half* dst, const float* v, i
   store_out_16<__half>(dst, v, n);
 }
 
+// Tile t of the persistent schedule -> (m tile, n tile): groups of 8 M tiles
+// sweep all N tiles, so the CTAs running at the same time share A and B
+// tiles in L2.
+__device__ __forceinline__ void tile_coords(uint32_t t, uint32_t mt, uint32_t nt, uint32_t& tm, uint32_t& tn) {
+  const uint32_t group = t / (8u * nt);
+  const uint32_t first_m = group * 8u;
+  const uint32_t gm = min(8u, mt - first_m);
+  const uint32_t r = t - group * 8u * nt;
+  tm = first_m + r % gm;
+  tn = r / gm;
+}
+
 template <bool MX>
 __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUtensorMap tmap_a,
                                                      const __grid_constant__ CUtensorMap tmap_b, Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
-  __shared__ __align__(8) uint64_t accum_bar;
+  __shared__ __align__(8) uint64_t accum_full;
+  __shared__ __align__(8) uint64_t accum_empty;
   __shared__ uint32_t tmem_base_holder;
   __shared__ int abort_flag;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile_n = blockIdx.x * BN, tile_m = blockIdx.y * BM;
+  const uint32_t mt = ((uint32_t)p.M + BM - 1) / BM, nt = ((uint32_t)p.N + BN - 1) / BN, tiles = mt * nt;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
-    mbar_init(smem_u32(&accum_bar), 1);
+    mbar_init(smem_u32(&accum_full), 1);
+    mbar_init(smem_u32(&accum_empty), EPI_WARPS);
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -267,109 +286,173 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_holder;
-
-  // scale tiles present in this tile's column of row blocks
-  const bool b_second = (uint32_t)(tile_n + 128) < p.rows_b_pad;
   const uint32_t tiles_per_stage = MX ? 1u : 4u;
 
   if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t issued = 0;
-      for (uint32_t kb = 0; kb < p.kb_count; ++kb) {
-        const uint32_t s = kb % STAGES;
-        const uint32_t par = ((kb / STAGES) & 1u) ^ 1u;
-        if (!mbar_wait(smem_u32(&empty_bar[s]), par)) {
-          abort_flag = 1;
-          break;
-        }
-        // scale tiles of this stage that exist (ragged K)
-        const uint32_t g0 = kb * tiles_per_stage;
-        uint32_t nt = p.sf_groups > g0 ? p.sf_groups - g0 : 0;
-        if (nt > tiles_per_stage) nt = tiles_per_stage;
-        const uint32_t sf_bytes_a = nt * 512u, sf_bytes_b = nt * 512u * (b_second ? 2u : 1u);
-        const uint32_t bar = smem_u32(&full_bar[s]);
-        mbar_expect_tx(bar, A_STAGE + B_STAGE + sf_bytes_a + sf_bytes_b);
-        tma_load_2d(sbase + SMEM_A + s * A_STAGE, &tmap_a, (int)(kb * BKB), tile_m, bar);
-        tma_load_2d(sbase + SMEM_B + s * B_STAGE, &tmap_b, (int)(kb * BKB), tile_n, bar);
-        if (nt) {
-          const uint8_t* sa = p.sfa + ((size_t)(tile_m / 128) * p.sf_groups + g0) * 512u;
-          bulk_load(sbase + SMEM_SFA + s * SFA_STAGE, sa, sf_bytes_a, bar);
-          const uint8_t* sb = p.sfb + ((size_t)(tile_n / 128) * p.sf_groups + g0) * 512u;
-          bulk_load(sbase + SMEM_SFB + s * SFB_STAGE, sb, sf_bytes_a, bar);
-          if (b_second) {
-            const uint8_t* sb2 = p.sfb + ((size_t)(tile_n / 128 + 1) * p.sf_groups + g0) * 512u;
-            bulk_load(sbase + SMEM_SFB + s * SFB_STAGE + 4 * 512, sb2, sf_bytes_a, bar);
+      uint32_t it = 0;  // global stage counter across tiles
+      for (uint32_t t = blockIdx.x; t < tiles && !*(volatile int*)&abort_flag; t += gridDim.x) {
+        uint32_t tm, tn;
+        tile_coords(t, mt, nt, tm, tn);
+        const int tile_m = (int)(tm * BM), tile_n = (int)(tn * BN);
+        const bool b_second = (uint32_t)(tile_n + 128) < p.rows_b_pad;
+        for (uint32_t kb = 0; kb < p.kb_count; ++kb, ++it) {
+          const uint32_t s = it % STAGES;
+          if (!mbar_wait(smem_u32(&empty_bar[s]), ((it / STAGES) & 1u) ^ 1u)) {
+            abort_flag = 1;
+            break;
+          }
+          const uint32_t g0 = kb * tiles_per_stage;
+          uint32_t ntl = p.sf_groups > g0 ? p.sf_groups - g0 : 0;
+          if (ntl > tiles_per_stage) ntl = tiles_per_stage;
+          const uint32_t sfa_bytes = ntl * 512u, sfb_bytes = ntl * 512u * (b_second ? 2u : 1u);
+          const uint32_t bar = smem_u32(&full_bar[s]);
+          mbar_expect_tx(bar, A_STAGE + B_STAGE + sfa_bytes + sfb_bytes);
+          tma_load_2d(sbase + SMEM_A + s * A_STAGE, &tmap_a, (int)(kb * BKB), tile_m, bar);
+          tma_load_2d(sbase + SMEM_B + s * B_STAGE, &tmap_b, (int)(kb * BKB), tile_n, bar);
+          if (ntl) {
+            bulk_load(sbase + SMEM_SFA + s * SFA_STAGE, p.sfa + ((size_t)tm * p.sf_groups + g0) * 512u, sfa_bytes, bar);
+            bulk_load(sbase + SMEM_SFB + s * SFB_STAGE, p.sfb + ((size_t)(tile_n / 128) * p.sf_groups + g0) * 512u,
+                      sfa_bytes, bar);
+            if (b_second)
+              bulk_load(sbase + SMEM_SFB + s * SFB_STAGE + 4 * 512,
+                        p.sfb + ((size_t)(tile_n / 128 + 1) * p.sf_groups + g0) * 512u, sfa_bytes, bar);
           }
         }
-        ++issued;
       }
-      // drain: every stage issued must have landed before the CTA may exit
-      const uint32_t first = issued > (uint32_t)STAGES ? issued - STAGES : 0;
-      for (uint32_t kb = first; kb < issued; ++kb)
-        mbar_wait(smem_u32(&full_bar[kb % STAGES]), (kb / STAGES) & 1u);
+      // drain: the last STAGES issued stages must have landed before exit
+      const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
+      for (uint32_t i = first; i < it; ++i) mbar_wait(smem_u32(&full_bar[i % STAGES]), (i / STAGES) & 1u);
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    // One thread issues everything, so the loop is kept lean: descriptors
+    // are built once and advanced by adding byte offsets >> 4 to their low
+    // 32-bit word (start address field); stage offsets advance
+    // incrementally.
     if (lane == 0) {
-      for (uint32_t kb = 0; kb < p.kb_count; ++kb) {
-        const uint32_t s = kb % STAGES;
-        if (!mbar_wait(smem_u32(&full_bar[s]), (kb / STAGES) & 1u) || *(volatile int*)&abort_flag) {
+      const uint64_t a_base = kmajor_sw128_desc(sbase + SMEM_A), b_base = kmajor_sw128_desc(sbase + SMEM_B);
+      const uint64_t sfa_base = sf_tile_desc(sbase + SMEM_SFA), sfb_base = sf_tile_desc(sbase + SMEM_SFB);
+      const uint32_t a_hi = (uint32_t)(a_base >> 32), b_hi = (uint32_t)(b_base >> 32);
+      const uint32_t sfa_hi = (uint32_t)(sfa_base >> 32), sfb_hi = (uint32_t)(sfb_base >> 32);
+      const uint32_t idesc_nv = block_scaled_idesc(1u, 0u, 0u);  // e2m1 x e2m1, ue4m3
+      auto mk = [](uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; };
+      uint32_t it = 0, tile_i = 0, s = 0, ph = 0;
+      bool ok = true;
+      for (uint32_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tile_i) {
+        uint32_t tm, tn;
+        tile_coords(t, mt, nt, tm, tn);
+        const bool b_second = (uint32_t)(tn * BN + 128) < p.rows_b_pad;
+        // the epilogue has drained the previous tile's accumulator
+        if (!mbar_wait(smem_u32(&accum_empty), (tile_i & 1u) ^ 1u) || *(volatile int*)&abort_flag) {
           abort_flag = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t tsfa = tmem + TMEM_SF + s * TMEM_SF_STAGE;
-        const uint32_t tsfb = tsfa + 16;
-        const uint32_t g0 = kb * tiles_per_stage;
-        uint32_t nt = p.sf_groups > g0 ? p.sf_groups - g0 : 0;
-        if (nt > tiles_per_stage) nt = tiles_per_stage;
-        for (uint32_t t = 0; t < nt; ++t) {
-          tmem_cp_sf(tsfa + 4 * t, sf_tile_desc(sbase + SMEM_SFA + s * SFA_STAGE + 512 * t));
-          tmem_cp_sf(tsfb + 8 * t, sf_tile_desc(sbase + SMEM_SFB + s * SFB_STAGE + 512 * t));
-          if (b_second) tmem_cp_sf(tsfb + 8 * t + 4, sf_tile_desc(sbase + SMEM_SFB + s * SFB_STAGE + 4 * 512 + 512 * t));
-        }
-        const uint32_t a0 = sbase + SMEM_A + s * A_STAGE, b0 = sbase + SMEM_B + s * B_STAGE;
-#pragma unroll
-        for (uint32_t j = 0; j < 4; ++j) {
-          if (kb * BKB + j * 32u >= p.k_bytes) break;  // ragged K: no codes left
-          const uint64_t ad = kmajor_sw128_desc(a0 + j * 32u);
-          const uint64_t bd = kmajor_sw128_desc(b0 + j * 32u);
-          uint32_t idesc, sfa, sfb;
-          if (MX) {
-            idesc = block_scaled_idesc(0u, 1u, j);  // e4m3 x e4m3, ue8m0, byte j of the scale words
-            sfa = tsfa;
-            sfb = tsfb;
-          } else {
-            idesc = block_scaled_idesc(1u, 0u, 0u);  // e2m1 x e2m1, ue4m3
-            sfa = tsfa + 4 * j;
-            sfb = tsfb + 8 * j;
+        for (uint32_t kb = 0; kb < p.kb_count; ++kb, ++it) {
+          if (!mbar_wait(smem_u32(&full_bar[s]), ph)) {
+            abort_flag = 1;
+            ok = false;
+            break;
           }
-          mma_block_scaled<MX>(tmem, ad, bd, idesc, sfa, sfb, (kb | j) != 0);
+          tc_fence_after();
+          const uint32_t tsfa = tmem + TMEM_SF + s * TMEM_SF_STAGE, tsfb = tsfa + 16;
+          const uint32_t sfa_lo = (uint32_t)sfa_base + s * (SFA_STAGE >> 4);
+          const uint32_t sfb_lo = (uint32_t)sfb_base + s * (SFB_STAGE >> 4);
+          const uint32_t a_lo = (uint32_t)a_base + s * (A_STAGE >> 4), b_lo = (uint32_t)b_base + s * (B_STAGE >> 4);
+          const uint32_t g0 = kb * tiles_per_stage;
+          if (g0 + tiles_per_stage <= p.sf_groups && p.k_bytes >= (kb + 1) * BKB) {
+            // full stage: all scale tiles and all four k-steps present
+            if (MX) {
+              tmem_cp_sf(tsfa, mk(sfa_lo, sfa_hi));
+              tmem_cp_sf(tsfb, mk(sfb_lo, sfb_hi));
+              if (b_second) tmem_cp_sf(tsfb + 4, mk(sfb_lo + (4 * 512 >> 4), sfb_hi));
+#pragma unroll
+              for (uint32_t j = 0; j < 4; ++j)
+                mma_block_scaled<true>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi),
+                                       block_scaled_idesc(0u, 1u, j), tsfa, tsfb, (kb | j) != 0);
+            } else {
+#pragma unroll
+              for (uint32_t u = 0; u < 4; ++u) {
+                tmem_cp_sf(tsfa + 4 * u, mk(sfa_lo + 32 * u, sfa_hi));
+                tmem_cp_sf(tsfb + 8 * u, mk(sfb_lo + 32 * u, sfb_hi));
+                if (b_second) tmem_cp_sf(tsfb + 8 * u + 4, mk(sfb_lo + (4 * 512 >> 4) + 32 * u, sfb_hi));
+              }
+#pragma unroll
+              for (uint32_t j = 0; j < 4; ++j)
+                mma_block_scaled<false>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi), idesc_nv, tsfa + 4 * j,
+                                        tsfb + 8 * j, (kb | j) != 0);
+            }
+          } else {
+            // ragged last stage: only the scale tiles and k-steps that exist
+            uint32_t ntl = p.sf_groups > g0 ? p.sf_groups - g0 : 0;
+            if (ntl > tiles_per_stage) ntl = tiles_per_stage;
+            for (uint32_t u = 0; u < ntl; ++u) {
+              tmem_cp_sf(tsfa + 4 * u, mk(sfa_lo + 32 * u, sfa_hi));
+              tmem_cp_sf(tsfb + 8 * u, mk(sfb_lo + 32 * u, sfb_hi));
+              if (b_second) tmem_cp_sf(tsfb + 8 * u + 4, mk(sfb_lo + (4 * 512 >> 4) + 32 * u, sfb_hi));
+            }
+            for (uint32_t j = 0; j < 4; ++j) {
+              if (kb * BKB + j * 32u >= p.k_bytes) break;
+              if (MX)
+                mma_block_scaled<true>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi),
+                                       block_scaled_idesc(0u, 1u, j), tsfa, tsfb, (kb | j) != 0);
+              else
+                mma_block_scaled<false>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi), idesc_nv, tsfa + 4 * j,
+                                        tsfb + 8 * j, (kb | j) != 0);
+            }
+          }
+          mma_commit(smem_u32(&empty_bar[s]));
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
-        mma_commit(smem_u32(&empty_bar[s]));
+        mma_commit(smem_u32(&accum_full));  // arrives when this tile's MMAs are done
       }
-      mma_commit(smem_u32(&accum_bar));
     }
   } else {
-    // epilogue warps 2..5: TMEM lane quarter q = warp % 4
-    const int q = warp & 3;
-    const int row = tile_m + q * 32 + lane;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&accum_bar), 0) && !*(volatile int*)&abort_flag);
-    tc_fence_after();
+    // ------------------------------------------------------------ epilogue warps 2..9
+    const int q = warp & 3;                // TMEM lane quarter this warp may read
+    const int half = (warp - 2) >> 2;      // which 128 accumulator columns
     float alpha = 1.0f;
     if (!MX && p.g_x != nullptr) alpha = (__ldg(p.g_x) / kGlobalEncode) * (__ldg(p.g_w) / kGlobalEncode);
-    if (ok) {
-      for (int c = 0; c < BN; c += 32) {
-        float v[32];
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
-        const int col = tile_n + c;
-        if (row < p.M && col < p.N) {
-          const int n = min(32, p.N - col);
+    uint32_t tile_i = 0;
+    for (uint32_t t = blockIdx.x; t < tiles; t += gridDim.x, ++tile_i) {
+      uint32_t tm, tn;
+      tile_coords(t, mt, nt, tm, tn);
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&accum_full), tile_i & 1u));
+      tc_fence_after();
+      if (!ok || *(volatile int*)&abort_flag) break;
+      float v[128];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= alpha;
-          const size_t off = (size_t)row * p.N + col;
-          if (p.y_dt == NVFP4_DT_F32) store_out<float>(static_cast<float*>(p.y) + off, v, n);
-          else if (p.y_dt == NVFP4_DT_BF16) store_out<__nv_bfloat16>(static_cast<__nv_bfloat16*>(p.y) + off, v, n);
-          else store_out<__half>(static_cast<__half*>(p.y) + off, v, n);
+      for (int c = 0; c < 4; ++c) {
+        float w32[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 128 + c * 32), w32);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[c * 32 + i] = w32[i];
+      }
+      // accumulator drained into registers: hand TMEM back to the MMA warp
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&accum_empty)) : "memory");
+      const int row = (int)(tm * BM) + q * 32 + lane;
+      const int col0 = (int)(tn * BN) + half * 128;
+      if (row < p.M) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int col = col0 + c * 32;
+          if (col < p.N) {
+            const int n = min(32, p.N - col);
+            float o[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = v[c * 32 + i] * alpha;
+            const size_t off = (size_t)row * p.N + col;
+            if (p.y_dt == NVFP4_DT_F32) store_out<float>(static_cast<float*>(p.y) + off, o, n);
+            else if (p.y_dt == NVFP4_DT_BF16) store_out<__nv_bfloat16>(static_cast<__nv_bfloat16*>(p.y) + off, o, n);
+            else store_out<__half>(static_cast<__half*>(p.y) + off, o, n);
+          }
         }
       }
     }
@@ -440,7 +523,8 @@ inline nvfp4_status qqmm_launch(bool mx, int64_t M, int64_t N, int64_t K, const 
   const int64_t sf_cols = mx ? K / 32 : K / 16;
   p.sf_groups = (uint32_t)((sf_cols + 3) / 4);
   p.rows_b_pad = (uint32_t)((N + 127) / 128 * 128);
-  dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  dim3 grid((unsigned)(tiles < sm_count ? tiles : sm_count));  // persistent: one CTA per SM
   cudaError_t e;
   if (mx) {
     e = cudaFuncSetAttribute(k_qqmm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
@@ -455,7 +539,6 @@ inline nvfp4_status qqmm_launch(bool mx, int64_t M, int64_t N, int64_t K, const 
     return NVFP4_ERR_CUDA;
   }
   msg[0] = '\0';
-  (void)sm_count;
   return NVFP4_OK;
 }
 
