@@ -282,6 +282,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(Args a) {
       mma_commit(smem_u32(&accum_bar));
     }
   }
+  __syncwarp();  // lanes that skipped a one-lane role loop wait for it before the CTA barrier
   tc_fence_before();
   __syncthreads();
   if (warp == 4) {

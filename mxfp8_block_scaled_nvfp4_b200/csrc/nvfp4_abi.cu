@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "quantize.cuh"
 #include "qmv.cuh"
+#include "qmv_tc.cuh"
 #include "qqmm_sm100.cuh"
 #include "gather_qmm.cuh"
 
@@ -334,26 +335,47 @@ nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32
   nvfp4_status st = device_info("qmv", &d);
   if (st != NVFP4_OK) return st;
   if (N == 0) return ok();
-  const size_t smem = (size_t)M * K * sizeof(float);
-  // one CTA of 16 warps per SM; each warp owns whole weight rows
-  uint64_t grid = ((uint64_t)N + (kQmvThreads / 32) - 1) / (kQmvThreads / 32);
-  if (grid > (uint64_t)d.sm_count) grid = d.sm_count;
   cudaError_t e = cudaSuccess;
-  dispatch_dt(x_dt, [&](auto tag_t) {
-    using T = decltype(tag_t);
-    auto x_t = [](const void* p) { return static_cast<const T*>(p); };
-    auto y_t = [](void* p) { return static_cast<T*>(p); };
-    auto go = [&](auto kern) {
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess)
-        kern<<<(unsigned)grid, kQmvThreads, smem, stream>>>(x_t(x), g_x, w_codes, w_scales, g_w, (int)M, (int)N,
-                                                           (int)K, y_t(y));
-    };
-    if (M == 1) go(k_qmv<T, 1>);
-    else if (M == 2) go(k_qmv<T, 2>);
-    else if (M <= 4) go(k_qmv<T, 4>);
-    else go(k_qmv<T, 8>);
-  });
+  const uint32_t stages = qtc::pick_stages(M, K);
+  if (stages > 0) {
+    // tensor-core path: one CTA per 128 weight rows
+    CUtensorMap mw, ms;
+    if (!qtc::make_maps(&mw, &ms, w_codes, w_scales, (uint64_t)N, (uint64_t)K))
+      return fail(NVFP4_ERR_CUDA, "[qmv] cuTensorMapEncodeTiled failed");
+    qtc::Args a{x, g_x, w_codes, w_scales, g_w, y, (uint32_t)M, (uint32_t)N, (uint32_t)K, stages};
+    const uint32_t MM = M == 1 ? 1u : 2u;
+    const size_t smem = qtc::smem_needed(stages, MM, (uint32_t)K);
+    const unsigned grid = (unsigned)((N + qtc::BM - 1) / qtc::BM);
+    dispatch_dt(x_dt, [&](auto tag_t) {
+      using T = decltype(tag_t);
+      auto go = [&](auto kern) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess) kern<<<grid, qtc::THREADS, smem, stream>>>(mw, ms, a);
+      };
+      if (M == 1) go(qtc::k_qmv_tc<T, 1>);
+      else go(qtc::k_qmv_tc<T, 2>);
+    });
+  } else {
+    const size_t smem = (size_t)M * K * sizeof(float);
+    // one CTA of 16 warps per SM; each warp owns whole weight rows
+    uint64_t grid = ((uint64_t)N + (kQmvThreads / 32) - 1) / (kQmvThreads / 32);
+    if (grid > (uint64_t)d.sm_count) grid = d.sm_count;
+    dispatch_dt(x_dt, [&](auto tag_t) {
+      using T = decltype(tag_t);
+      auto x_t = [](const void* p) { return static_cast<const T*>(p); };
+      auto y_t = [](void* p) { return static_cast<T*>(p); };
+      auto go = [&](auto kern) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess)
+          kern<<<(unsigned)grid, kQmvThreads, smem, stream>>>(x_t(x), g_x, w_codes, w_scales, g_w, (int)M, (int)N,
+                                                             (int)K, y_t(y));
+      };
+      if (M == 1) go(k_qmv<T, 1>);
+      else if (M == 2) go(k_qmv<T, 2>);
+      else if (M <= 4) go(k_qmv<T, 4>);
+      else go(k_qmv<T, 8>);
+    });
+  }
   if (e != cudaSuccess) return fail(NVFP4_ERR_CUDA, "[qmv] %s", cudaGetErrorString(e));
   return check_launch("qmv");
 }

@@ -38,78 +38,74 @@ __device__ __forceinline__ uint32_t xs_index(uint32_t m, uint32_t K, uint32_t k)
   return m * K + (c << 5) + ((seg ^ (c & 7u)) << 2) + (k & 3u);
 }
 
-template <typename T, int MM>
-__global__ void __launch_bounds__(kQmvThreads) k_qmv(
-    const T* __restrict__ x, const float* __restrict__ g_x, const uint32_t* __restrict__ wc,
-    const uint8_t* __restrict__ ws, const float* __restrict__ g_w, int M_, int N, int K,
-    T* __restrict__ y) {
-  extern __shared__ float4 xs4[];
+// x_hat = quantize-dequantize(x, g_x) ("fp_quantize_dequantize") for all M
+// rows into shared memory (fp32, swizzled chunks).
+template <typename T>
+__device__ __forceinline__ void qmv_prologue(const T* __restrict__ x, const float* __restrict__ g_x, uint32_t M,
+                                             uint32_t K, float4* xs4, uint32_t thread, uint32_t nthreads) {
   const uint32_t lane = threadIdx.x & 31u;
-  const uint32_t M = (uint32_t)M_;
-
-  // --- prologue: x_hat = quantize-dequantize(x, g_x) ("fp_quantize_dequantize")
-  {
-    const float E = g_x ? kGlobalEncode / __ldg(g_x) : 1.0f;
-    const float d = g_x ? __ldg(g_x) / kGlobalEncode : 1.0f;
-    const uint32_t n_half = M * (uint32_t)K / 8u;
-    for (uint32_t base = (threadIdx.x & ~31u); base < n_half; base += blockDim.x) {
-      const uint32_t hb = base + lane;
-      float v[8];
-      if (hb < n_half) {
-        load8<T>(x + (size_t)hb * 8, v);
-      } else {
+  const float E = g_x ? kGlobalEncode / __ldg(g_x) : 1.0f;
+  const float d = g_x ? __ldg(g_x) / kGlobalEncode : 1.0f;
+  const uint32_t n_half = M * K / 8u;
+  for (uint32_t base = (thread & ~31u); base < n_half; base += nthreads) {
+    const uint32_t hb = base + lane;
+    float v[8];
+    if (hb < n_half) {
+      load8<T>(x + (size_t)hb * 8, v);
+    } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = 0.0f;
-      }
-      float a = 0.0f;
+      for (int j = 0; j < 8; ++j) v[j] = 0.0f;
+    }
+    float a = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[j]));
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-      float t = a / kE2M1Max;
-      t = t * E;
-      const uint32_t s = f32_to_e4m3(t);
-      const float fs = e4m3_to_f32(s);
-      float dq[8];
-      if (fs != 0.0f) {
-        const float k = E / fs;
-        float q[8];
+    for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[j]));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    float t = a / kE2M1Max;
+    t = t * E;
+    const uint32_t s = f32_to_e4m3(t);
+    const float fs = e4m3_to_f32(s);
+    float dq[8];
+    const float sd = fs * d;
+    if (fs != 0.0f) {
+      const float k = E / fs;
+      float q[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) q[j] = v[j] * k;
-        const uint32_t w = f32x8_to_e2m1x8(q);
-        const float sd = fs * d;
+      for (int j = 0; j < 8; ++j) q[j] = v[j] * k;
+      const uint32_t w = f32x8_to_e2m1x8(q);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) dq[j] = Elem<T>::to_f(Elem<T>::from_f(e2m1_value(w >> (4 * j)) * sd));
-      } else {
+      for (int j = 0; j < 8; ++j) dq[j] = Elem<T>::to_f(Elem<T>::from_f(e2m1_value(w >> (4 * j)) * sd));
+    } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) dq[j] = 0.0f;
-      }
-      if (hb < n_half) {
-        const uint32_t m = (hb * 8u) / (uint32_t)K, k0 = hb * 8u - m * (uint32_t)K;
-        const uint32_t i0 = xs_index(m, K, k0), i1 = xs_index(m, K, k0 + 4);
-        xs4[i0 >> 2] = make_float4(dq[0], dq[1], dq[2], dq[3]);
-        xs4[i1 >> 2] = make_float4(dq[4], dq[5], dq[6], dq[7]);
-      }
+      for (int j = 0; j < 8; ++j) dq[j] = 0.0f;
+    }
+    if (hb < n_half) {
+      const uint32_t m = (hb * 8u) / K, k0 = hb * 8u - m * K;
+      const uint32_t i0 = xs_index(m, K, k0), i1 = xs_index(m, K, k0 + 4);
+      xs4[i0 >> 2] = make_float4(dq[0], dq[1], dq[2], dq[3]);
+      xs4[i1 >> 2] = make_float4(dq[4], dq[5], dq[6], dq[7]);
     }
   }
-  __syncthreads();
+}
 
-  // --- main loop
-  const float dw = g_w ? __ldg(g_w) / kGlobalEncode : 1.0f;
-  const uint32_t chunks = (uint32_t)K >> 5;  // 32 codes (16 bytes) per chunk
+// y rows n = first, first + step, ... < end (one warp per row) from x_hat in
+// shared memory: coalesced 128-bit code loads with register double buffering.
+template <typename T, int MM>
+__device__ __forceinline__ void qmv_simt_rows(const float4* xs4, const uint32_t* __restrict__ wc,
+                                              const uint8_t* __restrict__ ws, float dw, uint32_t M, uint32_t N,
+                                              uint32_t K, T* __restrict__ y, uint32_t first, uint32_t step,
+                                              uint32_t end) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t chunks = K >> 5;  // 32 codes (16 bytes) per chunk
   const uint32_t groups = (chunks + 32u * kQmvCH - 1) / (32u * kQmvCH);
-  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
   const uint4* wc4 = reinterpret_cast<const uint4*>(wc);
-
-  // units of this warp: (row n, group g) for n = warp + i * nwarps
-  uint32_t un = warp, ug = 0;
+  uint32_t un = first, ug = 0;
   uint4 qb[kQmvCH];
   uint32_t sb[kQmvCH];
   auto load_unit = [&](uint32_t n, uint32_t g) {
 #pragma unroll
     for (int i = 0; i < kQmvCH; ++i) {
       const uint32_t c = g * 32u * kQmvCH + (uint32_t)i * 32u + lane;
-      if (n < (uint32_t)N && c < chunks) {
+      if (n < end && c < chunks) {
         qb[i] = __ldg(wc4 + (size_t)n * chunks + c);
         sb[i] = __ldg(reinterpret_cast<const unsigned short*>(ws + (size_t)n * (chunks * 2u) + 2u * c));
       } else {
@@ -122,7 +118,7 @@ __global__ void __launch_bounds__(kQmvThreads) k_qmv(
   float acc[MM];
 #pragma unroll
   for (int m = 0; m < MM; ++m) acc[m] = 0.0f;
-  while (un < (uint32_t)N) {
+  while (un < end) {
     uint4 q[kQmvCH];
     uint32_t s[kQmvCH];
 #pragma unroll
@@ -133,7 +129,7 @@ __global__ void __launch_bounds__(kQmvThreads) k_qmv(
     const uint32_t cn = un, cg = ug;
     if (++ug == groups) {
       ug = 0;
-      un += nwarps;
+      un += step;
     }
     load_unit(un, ug);  // next unit's loads in flight while this one computes
 #pragma unroll
@@ -158,7 +154,7 @@ __global__ void __launch_bounds__(kQmvThreads) k_qmv(
 #pragma unroll
             for (int m = 0; m < MM; ++m) {
               if ((uint32_t)m < M) {
-                const float4 xv = xs4[(m * (uint32_t)K + off) >> 2];
+                const float4 xv = xs4[(m * K + off) >> 2];
                 bs[m] = fmaf(xv.x, v0, bs[m]);
                 bs[m] = fmaf(xv.y, v1, bs[m]);
                 bs[m] = fmaf(xv.z, v2, bs[m]);
@@ -184,6 +180,20 @@ __global__ void __launch_bounds__(kQmvThreads) k_qmv(
       }
     }
   }
+}
+
+template <typename T, int MM>
+__global__ void __launch_bounds__(kQmvThreads) k_qmv(
+    const T* __restrict__ x, const float* __restrict__ g_x, const uint32_t* __restrict__ wc,
+    const uint8_t* __restrict__ ws, const float* __restrict__ g_w, int M_, int N, int K,
+    T* __restrict__ y) {
+  extern __shared__ float4 xs4[];
+  qmv_prologue<T>(x, g_x, (uint32_t)M_, (uint32_t)K, xs4, threadIdx.x, blockDim.x);
+  __syncthreads();
+  const float dw = g_w ? __ldg(g_w) / kGlobalEncode : 1.0f;
+  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  qmv_simt_rows<T, MM>(xs4, wc, ws, dw, (uint32_t)M_, (uint32_t)N, (uint32_t)K, y, warp, nwarps, (uint32_t)N);
 }
 
 }  // namespace nvfp4

@@ -1,0 +1,456 @@
+// qmv on the tensor cores: the NVFP4 weight goes to tcgen05 block-scaled
+// MMAs in its stored form (e2m1 codes by TMA, e4m3 block scales through
+// tensor memory); nothing is decoded per weight on the SIMT cores.
+//
+// Same result as k_qmv (qmv.cuh):  y[m, n] = T( sum_b sd[n,b] * sum_{k in b}
+// x_hat[m,k] * e2m1(q[n,k]) ),  sd = f8(s) * g_w / 2688.
+//
+// x_hat is written exactly as two e2m1 "planes" per 16-block:
+//   x_hat_k = A_b * e2m1(pA_k) + B_b * e2m1(pB_k),
+//   A_b = T(sdx_b), B_b = T(1.5 * sdx_b)  (sdx = f8(sx) * g_x / 2688),
+// because T(v * sdx) = 2^i * T(u * sdx) for v = 2^i * u, u in {1, 1.5},
+// whenever 0.5 |sdx| and 6 |sdx| lie in T's normal range (rounding to a
+// binary format commutes with scaling by a power of two there, and the fp32
+// product before the rounding to T scales the same way).  The prologue
+// checks that range per block; if any block of x falls outside it (x_hat
+// subnormal or overflowing), the CTA computes its rows with the SIMT loop
+// instead, from an fp32 x_hat written over the plane tiles.  One MMA (M = 128 weight rows, N = 8 per x row, K = 64)
+// per k-step then yields, for each of the k-step's 4 blocks and 2 planes,
+//   D[n, (m, b, p)] = f8(sw[n, b]) * sum_{k in b} e2m1(q[n, k]) * e2m1(p_k)
+// (x-side scales 1), written to fresh TMEM columns; the epilogue warps
+// accumulate y[m, n] += U_(b,p) * D with U = A_b or B_b, and finally scale
+// by g_w / 2688.
+//
+// CTA = 128 weight rows; warps: 0 TMA producer (codes [128 x 128 B] and
+// LINEAR scales [128 x 16 B] per stage), 1 TMEM allocator + MMA issuer,
+// 2 scale re-layout (LINEAR [128 rows x 16 B] -> four 128x4 tiles for
+// tcgen05.cp), 4-7 epilogue (TMEM lane quarters).  All warps compute the
+// x_hat planes first, while the producer's first loads are in flight.
+// TMEM: a 256-column ring of MMA outputs drained in 128-column halves, the
+// weight scale tiles of every stage, one column of unit x-side scales.
+//
+// Every mbarrier wait of the MMA thread costs about as much as several of
+// these small MMAs (its shared-memory access queues behind the tensor
+// core's operand reads), so the MMA thread waits once per group of stages:
+// the re-layout warp handles stages in order, so the barrier of a group's
+// last stage covers the whole group; ring halves that were never used are
+// not waited on.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "qmv.cuh"
+#include "qqmm_sm100.cuh"
+
+namespace nvfp4 {
+namespace qtc {
+
+constexpr int THREADS = 256;
+constexpr int BM = 128;            // weight rows per CTA
+constexpr int MAX_STAGES = 8;
+constexpr int A_STAGE = BM * 128;  // 16 KiB of codes (256 K)
+constexpr int S_STAGE = BM * 16;   // 2 KiB of LINEAR scales
+constexpr int T_STAGE = 4 * 512;   // four 128x4 scale tiles
+constexpr int STAGE_BYTES = A_STAGE + S_STAGE + T_STAGE;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t D_RING = 256;     // MMA output columns [0, 256)
+constexpr uint32_t T_SFB = 256;      // unit x-side scales
+constexpr uint32_t T_SFA = 260;      // weight scale tiles: 16 columns per stage
+
+// shared memory carve-up (bytes, from a 1024-aligned base)
+struct Layout {
+  uint32_t stages, M, K;
+  uint32_t ring, planes, uplane, ones, total;
+  __host__ __device__ void init(uint32_t st, uint32_t m, uint32_t k) {
+    stages = st;
+    M = m;
+    K = k;
+    ring = 0;
+    planes = stages * STAGE_BYTES;                 // 4 * M * K bytes (fp32 x_hat in the SIMT fallback)
+    uplane = planes + 4u * M * K;                  // 2 * (K / 16) * M floats
+    ones = uplane + 2u * (K / 16u) * M * 4u;       // 512 bytes of e4m3 1.0
+    total = ones + 512u;
+  }
+};
+
+__host__ __device__ inline uint32_t smem_needed(uint32_t stages, uint32_t M, uint32_t K) {
+  Layout L;
+  L.init(stages, M, K);
+  return L.total + 1024u;
+}
+
+struct Args {
+  const void* x;
+  const float* g_x;
+  const uint32_t* wc;
+  const uint8_t* wsc;
+  const float* g_w;
+  void* y;
+  uint32_t M, N, K, stages;
+};
+
+// K-major operand without swizzle: 8-row x 16-byte core matrices, `lbo`
+// bytes between core matrices along K, `sbo` between 8-row groups.
+__device__ __forceinline__ uint64_t kmajor_plain_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return tc::smem_desc(addr, lbo, sbo, 0);
+}
+
+// Normal range of T: the plane form of x_hat is exact for a block whose
+// decode scale sdx has 0.5 |sdx| >= kMinNormal and 6 |sdx| <= kMaxFinite.
+template <typename T> struct Range;
+template <> struct Range<float> {
+  static constexpr float kMinNormal = 0x1p-126f, kMaxFinite = 0x1.fffffep127f;
+};
+template <> struct Range<__half> {
+  static constexpr float kMinNormal = 0x1p-14f, kMaxFinite = 65504.0f;
+};
+template <> struct Range<__nv_bfloat16> {
+  static constexpr float kMinNormal = 0x1p-126f, kMaxFinite = 0x1.fep127f;
+};
+
+// x_hat = quantize-dequantize(x, g_x) of all M rows as plane codes and
+// plane scales (layout in the header comment).  One lane per half-block;
+// returns false on a thread that met a block outside the exact range.
+// x values of this thread's first half-block, loaded at kernel start.
+template <typename T>
+__device__ __forceinline__ void x_first(const T* __restrict__ x, uint32_t M, uint32_t K, float (&v)[8]) {
+  if (threadIdx.x < M * K / 8u) {
+    load8<T>(x + (size_t)threadIdx.x * 8, v);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = 0.0f;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ bool x_planes(const T* __restrict__ x, float gx, uint32_t M, uint32_t K, float (&cur)[8],
+                                         uint8_t* planes, float* uplane) {
+  const float E = kGlobalEncode / gx;
+  const float d = gx / kGlobalEncode;
+  const uint32_t n_half = M * K / 8u;  // a multiple of 32: whole warps take part in the pair shuffle
+  const uint32_t nb = K / 16u;
+  bool exact = true;
+  for (uint32_t hb = threadIdx.x; hb < n_half; hb += blockDim.x) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = cur[j];
+    const uint32_t hn = hb + blockDim.x;  // next half-block's loads in flight during this one
+    if (hn < n_half) load8<T>(x + (size_t)hn * 8, cur);
+    float a = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[j]));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    const float t = (a / kE2M1Max) * E;
+    const float fs = e4m3_to_f32(f32_to_e4m3(t));
+    const float sd = fs * d;
+    uint32_t w = 0;
+    if (fs != 0.0f) {
+      const float k = E / fs;
+      float q[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) q[j] = v[j] * k;
+      w = f32x8_to_e2m1x8(q);
+    }
+    const float asd = fabsf(sd);
+    exact = exact && (sd == 0.0f || (0.5f * asd >= Range<T>::kMinNormal && 6.0f * asd <= Range<T>::kMaxFinite));
+    // codes of magnitude 1.5, 3, 6 (odd magnitude code >= 3) go to plane B
+    // as 1, 2, 4 (the code minus one); all others stay in plane A
+    const uint32_t odd3 = w & 0x11111111u & ((w >> 1) | (w >> 2));
+    const uint32_t mask = odd3 * 15u;
+    const uint32_t pa = w & ~mask, pbw = (w - odd3) & mask;
+    // plane tile of k-step g = k0/64, block bl = (k0/16)%4, half hf of the block
+    const uint32_t m = (hb * 8u) / K, k0 = hb * 8u - m * K;
+    const uint32_t g = k0 >> 6, bl = (k0 >> 4) & 3u, hf = (k0 >> 3) & 1u;
+    uint8_t* tile = planes + (size_t)g * 256u * M;  // [h][row group][8 rows][16 B], rows = m*8 + bl*2 + p
+    const uint32_t h = bl >> 1, byte = 8u * (bl & 1u) + 4u * hf;
+    const uint32_t rowA = m * 8u + bl * 2u, rowB = rowA + 1u;
+    *reinterpret_cast<uint32_t*>(tile + h * 128u * M + (rowA >> 3) * 128u + (rowA & 7u) * 16u + byte) = pa;
+    *reinterpret_cast<uint32_t*>(tile + h * 128u * M + (rowB >> 3) * 128u + (rowB & 7u) * 16u + byte) = pbw;
+    if (hf == 0) {
+      const uint32_t b = k0 >> 4;
+      uplane[m * 2u * nb + 2u * b] = Elem<T>::to_f(Elem<T>::from_f(sd));
+      uplane[m * 2u * nb + 2u * b + 1u] = Elem<T>::to_f(Elem<T>::from_f(1.5f * sd));
+    }
+  }
+  return exact;
+}
+
+template <typename T, int MM>
+__global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ CUtensorMap tmap_w,
+                                                       const __grid_constant__ CUtensorMap tmap_s, Args a) {
+  using namespace tc;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[MAX_STAGES];
+  __shared__ __align__(8) uint64_t sf_bar[MAX_STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[MAX_STAGES];
+  __shared__ __align__(8) uint64_t dfull_bar[2];
+  __shared__ __align__(8) uint64_t dempty_bar[2];
+  __shared__ uint32_t tmem_holder;
+  __shared__ int abort_flag;
+
+  // x and g_x first: these loads must not queue behind the weight stream
+  float xv[8];
+  x_first<T>(static_cast<const T*>(a.x), a.M, a.K, xv);
+  const float gx = a.g_x ? __ldg(a.g_x) : kGlobalEncode;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  Layout L;
+  L.init(a.stages, MM, a.K);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t row0 = blockIdx.x * BM;
+  const uint32_t S = a.stages;
+  const uint32_t kb_count = a.K / 256u;   // stages of 256 K
+  const uint32_t ksteps = a.K / 64u;      // MMAs
+  const uint32_t ncols = 8u * MM;         // MMA N
+  const uint32_t steps_per_half = 128u / ncols;
+  const uint32_t nb = a.K / 16u;
+
+  if (threadIdx.x == 0) {
+    for (uint32_t s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&sf_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(smem_u32(&dfull_bar[h]), 1);
+      mbar_init(smem_u32(&dempty_bar[h]), 4);
+    }
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // zero the plane tiles (a plane row is nonzero only inside its own
+  // 16-block: the prologue writes those bytes alone), fill the unit scale tile
+  {
+    uint4* z = reinterpret_cast<uint4*>(smem + L.planes);
+    const uint32_t nz = (L.uplane - L.planes) / 16u;
+    for (uint32_t i = threadIdx.x; i < nz; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+    uint4* o = reinterpret_cast<uint4*>(smem + L.ones);
+    if (threadIdx.x < 32) o[threadIdx.x] = make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to tcgen05.cp
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_holder;
+
+  // the producer starts streaming the weight before the prologue runs
+  uint32_t issued = 0;
+  if (threadIdx.x == 0) {
+    for (; issued < S && issued < kb_count; ++issued) {
+      const uint32_t bar = smem_u32(&full_bar[issued]);
+      mbar_expect_tx(bar, A_STAGE + S_STAGE);
+      tma_load_2d(sbase + L.ring + issued * STAGE_BYTES, &tmap_w, (int)(issued * 128u), (int)row0, bar);
+      tma_load_2d(sbase + L.ring + issued * STAGE_BYTES + A_STAGE, &tmap_s, (int)(issued * 16u), (int)row0, bar);
+    }
+  }
+  const bool mine = x_planes<T>(static_cast<const T*>(a.x), gx, a.M, a.K, xv, smem + L.planes,
+                                reinterpret_cast<float*>(smem + L.uplane));
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // planes are read by the tensor core
+  const bool exact = __syncthreads_and(mine) != 0;
+  const float dw = a.g_w ? __ldg(a.g_w) / kGlobalEncode : 1.0f;
+
+  if (!exact) {
+    // x_hat outside the planes' exact range: fp32 x_hat over the plane tiles
+    // and SIMT rows for this CTA, after the loads in flight have landed
+    float4* xs4 = reinterpret_cast<float4*>(smem + L.planes);
+    qmv_prologue<T>(static_cast<const T*>(a.x), a.g_x, a.M, a.K, xs4, threadIdx.x, blockDim.x);
+    if (threadIdx.x == 0)
+      for (uint32_t i = 0; i < issued; ++i) mbar_wait(smem_u32(&full_bar[i]), 0);
+    __syncthreads();
+    const uint32_t end = min(row0 + BM, a.N);
+    qmv_simt_rows<T, MM>(xs4, a.wc, a.wsc, dw, a.M, a.N, a.K, static_cast<T*>(a.y), row0 + warp,
+                         THREADS / 32, end);
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      for (uint32_t kb = issued; kb < kb_count; ++kb) {
+        const uint32_t s = kb % S;
+        if (!mbar_wait(smem_u32(&empty_bar[s]), ((kb / S) & 1u) ^ 1u) || *(volatile int*)&abort_flag) {
+          abort_flag = 1;
+          break;
+        }
+        const uint32_t bar = smem_u32(&full_bar[s]);
+        mbar_expect_tx(bar, A_STAGE + S_STAGE);
+        tma_load_2d(sbase + L.ring + s * STAGE_BYTES, &tmap_w, (int)(kb * 128u), (int)row0, bar);
+        tma_load_2d(sbase + L.ring + s * STAGE_BYTES + A_STAGE, &tmap_s, (int)(kb * 16u), (int)row0, bar);
+        issued = kb + 1;
+      }
+      const uint32_t first = issued > S ? issued - S : 0;
+      for (uint32_t i = first; i < issued; ++i) mbar_wait(smem_u32(&full_bar[i % S]), (i / S) & 1u);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ scale re-layout
+    // tile j (k-step j of the stage), row r: the 4 block scales of weight
+    // rows r, r+32, r+64, r+96 (the 128x4 tile order tcgen05.cp expects)
+    for (uint32_t kb = 0; kb < kb_count; ++kb) {
+      const uint32_t s = kb % S;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full_bar[s]), (kb / S) & 1u)) ||
+          *(volatile int*)&abort_flag) {
+        abort_flag = 1;
+        break;
+      }
+      const uint8_t* raw = smem + L.ring + s * STAGE_BYTES + A_STAGE;
+      uint8_t* tiles = smem + L.ring + s * STAGE_BYTES + A_STAGE + S_STAGE;
+      const uint4 q0 = *reinterpret_cast<const uint4*>(raw + 16u * lane);
+      const uint4 q1 = *reinterpret_cast<const uint4*>(raw + 16u * (lane + 32));
+      const uint4 q2 = *reinterpret_cast<const uint4*>(raw + 16u * (lane + 64));
+      const uint4 q3 = *reinterpret_cast<const uint4*>(raw + 16u * (lane + 96));
+      *reinterpret_cast<uint4*>(tiles + 0 * 512 + 16u * lane) = make_uint4(q0.x, q1.x, q2.x, q3.x);
+      *reinterpret_cast<uint4*>(tiles + 1 * 512 + 16u * lane) = make_uint4(q0.y, q1.y, q2.y, q3.y);
+      *reinterpret_cast<uint4*>(tiles + 2 * 512 + 16u * lane) = make_uint4(q0.z, q1.z, q2.z, q3.z);
+      *reinterpret_cast<uint4*>(tiles + 3 * 512 + 16u * lane) = make_uint4(q0.w, q1.w, q2.w, q3.w);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sf_bar[s])) : "memory");
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    // The whole warp runs the loop and one elected lane issues.  The wait
+    // for a drained ring half sits at a stage boundary (a half holds a
+    // multiple of 4 k-steps), so each stage issues straight-line code.
+    const bool leader = elect_one();
+    if (leader) tmem_cp_sf(tmem + T_SFB, sf_tile_desc(sbase + L.ones));
+    const uint32_t idesc = (1u << 7) | (1u << 10) | ((ncols >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    const uint64_t a_base = kmajor_sw128_desc(sbase + L.ring);
+    const uint64_t b_base = kmajor_plain_desc(sbase + L.planes, 128u * MM, 128u);
+    const uint64_t t_base = sf_tile_desc(sbase + L.ring + A_STAGE + S_STAGE);
+    const uint32_t a_hi = (uint32_t)(a_base >> 32), b_hi = (uint32_t)(b_base >> 32), t_hi = (uint32_t)(t_base >> 32);
+    auto mk = [](uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; };
+    const uint32_t G = S >= 2 ? S / 2 : 1;  // stages per wait
+    uint32_t g = 0;  // global k-step
+    bool ok = true;
+    for (uint32_t kb0 = 0; kb0 < kb_count && ok; kb0 += G) {
+      const uint32_t kb1 = min(kb0 + G, kb_count), last = kb1 - 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sf_bar[last % S]), (last / S) & 1u)) ||
+          *(volatile int*)&abort_flag) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      for (uint32_t kb = kb0; kb < kb1; ++kb) {
+        const uint32_t s = kb % S;
+        const uint32_t hf = (g / steps_per_half) & 1u;  // ring half of this stage
+        const uint32_t use = g / (2u * steps_per_half);   // times this half was used before
+        if (g % steps_per_half == 0 && use > 0) {         // reuse: wait until the half is drained
+          if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&dempty_bar[hf]), (use & 1u) ^ 1u))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        if (leader) {
+          const uint32_t tsfa = tmem + T_SFA + 16u * s;
+#pragma unroll
+          for (uint32_t j = 0; j < 4; ++j)
+            tmem_cp_sf(tsfa + 4u * j, mk((uint32_t)t_base + ((s * STAGE_BYTES + 512u * j) >> 4), t_hi));
+          const uint32_t dcol = (g % (2u * steps_per_half)) * ncols;
+#pragma unroll
+          for (uint32_t j = 0; j < 4; ++j)
+            mma_block_scaled<false>(tmem + dcol + j * ncols,
+                                    mk((uint32_t)a_base + ((s * STAGE_BYTES + 32u * j) >> 4), a_hi),
+                                    mk((uint32_t)b_base + (((g + j) * 256u * MM) >> 4), b_hi), idesc, tsfa + 4u * j,
+                                    tmem + T_SFB, 0u);
+          if ((g + 4) % steps_per_half == 0 || g + 4 == ksteps) mma_commit(smem_u32(&dfull_bar[hf]));
+          mma_commit(smem_u32(&empty_bar[s]));
+        }
+        __syncwarp();
+        g += 4;
+      }
+    }
+    if (!ok && leader) abort_flag = 1;
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t q = warp & 3;
+    const float* U = reinterpret_cast<const float*>(smem + L.uplane);
+    float acc[MM];
+#pragma unroll
+    for (int m = 0; m < MM; ++m) acc[m] = 0.0f;
+    const uint32_t halves = (ksteps + steps_per_half - 1) / steps_per_half;
+    bool ok = true;
+    for (uint32_t h = 0; h < halves; ++h) {
+      const uint32_t hf = h & 1u;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&dfull_bar[hf]), (h >> 1) & 1u)) && !*(volatile int*)&abort_flag;
+      tc_fence_after();
+      if (!ok) break;
+      const uint32_t g0 = h * steps_per_half;
+      const uint32_t nsteps = min(steps_per_half, ksteps - g0);
+      for (uint32_t c = 0; c < nsteps * ncols; c += 32) {
+        float v[32];
+        tmem_ld32(tmem + ((q * 32u) << 16) + hf * 128u + c, v);
+        const uint32_t gc = g0 + c / (8u * MM);  // k-step of column c (32 is a multiple of 8 * MM)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          constexpr int NC = 8 * MM;
+          const int m = (i % NC) >> 3, bp = i & 7;  // compile-time after unrolling
+          const uint32_t gg = gc + (uint32_t)(i / NC);
+          if (c + i < nsteps * ncols) acc[m] = fmaf(U[(uint32_t)m * 2u * nb + 8u * gg + (uint32_t)bp], v[i], acc[m]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&dempty_bar[hf])) : "memory");
+    }
+    const uint32_t row = row0 + q * 32u + lane;
+    if (ok && row < a.N) {
+#pragma unroll
+      for (int m = 0; m < MM; ++m)
+        if ((uint32_t)m < a.M) static_cast<T*>(a.y)[(size_t)m * a.N + row] = Elem<T>::from_f(acc[m] * dw);
+    }
+  }
+  __syncwarp();  // lanes that skipped a one-lane role loop wait for it before the CTA barrier
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// Tensor maps of the weight codes [N, K/2 bytes] (box 128 B x 128 rows,
+// 128-byte swizzle) and LINEAR scales [N, K/16 bytes] (box 16 B x 128 rows).
+inline bool make_maps(CUtensorMap* mw, CUtensorMap* ms, const uint32_t* wc, const uint8_t* wsc, uint64_t N,
+                      uint64_t K) {
+  auto fn = tc::encode_fn();
+  if (!fn) return false;
+  {
+    cuuint64_t dims[2] = {K / 2, N};
+    cuuint64_t strides[1] = {K / 2};
+    cuuint32_t box[2] = {128, BM};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint32_t*>(wc), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  {
+    cuuint64_t dims[2] = {K / 16, N};
+    cuuint64_t strides[1] = {K / 16};
+    cuuint32_t box[2] = {16, BM};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(ms, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(wsc), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  return true;
+}
+
+// Stages that fit next to the plane tiles, plane scales and x_hat; 0 if the
+// tensor-core path does not apply (then the caller runs the SIMT kernel).
+inline uint32_t pick_stages(int64_t M, int64_t K) {
+  if (M < 1 || M > 2 || K % 256 != 0 || K < 256) return 0;
+  const uint32_t MM = M == 1 ? 1u : 2u;
+  for (uint32_t st = MAX_STAGES; st >= 3; --st)
+    if (smem_needed(st, MM, (uint32_t)K) <= 227u * 1024u) return st;
+  return 0;
+}
+
+}  // namespace qtc
+}  // namespace nvfp4

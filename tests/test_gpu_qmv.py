@@ -69,3 +69,32 @@ def test_qmv_rejects_K_not_multiple_of_32(nv):
     ws = torch.zeros(4, 3, dtype=torch.uint8).cuda()
     with pytest.raises(nv.Nvfp4Error):
         nv.qmv(x, wc, ws)
+
+
+# Shapes that take the tensor-core path (M <= 2, K % 256 == 0): the weight
+# goes to block-scaled MMAs in its stored form, x_hat as two e2m1 planes.
+@pytest.mark.parametrize("dt", ["bf16", "f16", "f32"])
+@pytest.mark.parametrize("M,N,K", [(1, 130, 4096), (2, 257, 2048), (1, 128, 8192), (2, 384, 256), (1, 1, 512)])
+@pytest.mark.parametrize("use_g", [True, False])
+def test_qmv_tensor_path_parity(nv, orc, dt, M, N, K, use_g):
+    run_case(nv, orc, M, N, K, dt, use_g, seed=7 * M + N + K)
+
+
+def test_qmv_tensor_path_falls_back_on_subnormal_x_hat(nv, orc):
+    """fp16 x around 1e-6 with g_x = amax(x): x_hat lands in fp16's subnormal
+    range, where the two-plane form is not exact, so the kernel computes
+    these rows on the SIMT cores; the result still matches the oracle."""
+    from mxfp8_block_scaled_nvfp4_b200 import workloads
+    M, N, K = 1, 256, 1024
+    x = (workloads.normal((M, K), 1.0, 5, torch.float32) * 1e-6).to(torch.float16)
+    w = workloads.normal((N, K), 0.02, 6, torch.float16)
+    xg, wg = x.cuda(), w.cuda()
+    g_x, g_w = nv.amax(xg), nv.amax(wg)
+    wc, ws = nv.nvfp4_quantize(wg, g_w, "linear")
+    y = nv.qmv(xg, wc, ws, g_x, g_w)
+    owc, ows = orc.nvfp4_quantize(raw(w), "f16", g_w.item())
+    r = orc.qmv(raw(x), "f16", g_x.item(), owc, ows, g_w.item())
+    # the two-plane form really is inexact for this input
+    xh = orc.to_f64(orc.nvfp4_quantize_dequantize(raw(x), "f16", g_x.item()), "f16")
+    assert np.any((np.abs(xh) < 2.0 ** -14) & (xh != 0))
+    check_gemm_output(raw(y), r, "f16", orc)
