@@ -18,7 +18,8 @@
 //            tiles as plain bulk copies (the 128x4 scale-tile layout of the
 //            operands is already the order the MMA's scale tensor memory
 //            expects, so the copies are contiguous 512-byte blocks).
-//   warp 1   TMEM allocator and MMA issuer: one thread moves the stage's
+//   warp 1   TMEM allocator and MMA issuer: one elected lane of the
+//            converged warp moves the stage's
 //            scale tiles into tensor memory (tcgen05.cp 32x128b.warpx4) and
 //            issues the block-scaled MMAs (M=128, N=256, K=64 NVFP4 / 32
 //            MXFP8 per instruction) into a 128 x 256 fp32 accumulator in TMEM;
@@ -336,11 +337,13 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // One thread issues everything, so the loop is kept lean: descriptors
-    // are built once and advanced by adding byte offsets >> 4 to their low
-    // 32-bit word (start address field); stage offsets advance
-    // incrementally.
-    if (lane == 0) {
+    // The whole warp runs the loop (its values stay warp-uniform) and one
+    // elected lane issues the tensor-core instructions.  The loop is kept
+    // lean: descriptors are built once and advanced by adding byte offsets
+    // >> 4 to their low 32-bit word (start address field); stage offsets
+    // advance incrementally.
+    {
+      const bool leader = elect_one();
       const uint64_t a_base = kmajor_sw128_desc(sbase + SMEM_A), b_base = kmajor_sw128_desc(sbase + SMEM_B);
       const uint64_t sfa_base = sf_tile_desc(sbase + SMEM_SFA), sfb_base = sf_tile_desc(sbase + SMEM_SFB);
       const uint32_t a_hi = (uint32_t)(a_base >> 32), b_hi = (uint32_t)(b_base >> 32);
@@ -354,18 +357,20 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
         tile_coords(t, mt, nt, tm, tn);
         const bool b_second = (uint32_t)(tn * BN + 128) < p.rows_b_pad;
         // the epilogue has drained the previous tile's accumulator
-        if (!mbar_wait(smem_u32(&accum_empty), (tile_i & 1u) ^ 1u) || *(volatile int*)&abort_flag) {
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&accum_empty), (tile_i & 1u) ^ 1u)) ||
+            *(volatile int*)&abort_flag) {
           abort_flag = 1;
           break;
         }
         tc_fence_after();
         for (uint32_t kb = 0; kb < p.kb_count; ++kb, ++it) {
-          if (!mbar_wait(smem_u32(&full_bar[s]), ph)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full_bar[s]), ph))) {
             abort_flag = 1;
             ok = false;
             break;
           }
           tc_fence_after();
+          if (leader) {
           const uint32_t tsfa = tmem + TMEM_SF + s * TMEM_SF_STAGE, tsfb = tsfa + 16;
           const uint32_t sfa_lo = (uint32_t)sfa_base + s * (SFA_STAGE >> 4);
           const uint32_t sfb_lo = (uint32_t)sfb_base + s * (SFB_STAGE >> 4);
@@ -412,13 +417,16 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
                                         tsfb + 8 * j, (kb | j) != 0);
             }
           }
-          mma_commit(smem_u32(&empty_bar[s]));
+            mma_commit(smem_u32(&empty_bar[s]));
+          }
+          __syncwarp();
           if (++s == STAGES) {
             s = 0;
             ph ^= 1u;
           }
         }
-        mma_commit(smem_u32(&accum_full));  // arrives when this tile's MMAs are done
+        if (leader) mma_commit(smem_u32(&accum_full));  // arrives when this tile's MMAs are done
+        __syncwarp();
       }
     }
   } else {
