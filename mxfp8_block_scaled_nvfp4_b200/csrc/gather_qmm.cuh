@@ -12,17 +12,29 @@
 //     row of the expert's run, rows) and the permutation of pair ids grouped
 //     by expert.  Expert ids outside [0, E) set the device error word and
 //     their output rows are written as zeros.
-//  2. k_gather_mma: one CTA per (tile, 256 output columns).  Warps 0-3 gather
-//     the tile's 128 x rows with cp.async into the 128-byte-swizzled K-major
-//     shared layout and dequantize the expert's weight tile [256 rows x 64 K]
-//     to bf16 into the same layout (the weight is rounded to bf16 exactly as
-//     the dequantize kernel does); warp 4 issues tcgen05 kind::f16 MMAs
-//     (M=128 pairs, N=256 columns, K=16) into a TMEM fp32 accumulator; warps
-//     0-3 then read the accumulator and scatter each row to y[t, j, :].
+//  2. k_gather_mma, persistent (one CTA per SM): work units are (128-pair
+//     tile, 256 output columns), handed out round-robin, the column tiles of
+//     a pair tile adjacent so that CTAs running together share x rows and the
+//     expert's weight in L2.  Warp roles:
+//       warp 0     gathers the tile's x rows with TMA tile::gather4 (4 rows
+//                  per copy) into 128-byte-swizzled K-major stages;
+//       warp 1     streams the expert's NVFP4 codes [256 rows x 32 B] per
+//                  k-step with TMA;
+//       warp 2     allocates TMEM and issues tcgen05 kind::f16 MMAs (M = 128
+//                  pairs, N = 256 columns, K = 16) from one elected lane into
+//                  one of two fp32 accumulators;
+//       warps 4-11 dequantize the codes to bf16 (one weight row per thread,
+//                  block scale from global memory one k-step ahead) into the
+//                  swizzled B stages, rounding exactly as the dequantize
+//                  kernel does;
+//       warps 12-15 drain an accumulator (one TMEM lane quarter each) and
+//                  scatter each pair row to y[t, j, :] while the MMAs of the
+//                  next unit run on the other accumulator.
 // The contraction is on the bf16 tensor pipe: both operands are bf16, as
-// the method requires of the materialized weight.
+// the method requires of the materialized weight.  Every wait is bounded.
 #pragma once
 
+#include <cuda.h>
 #include <cstdio>
 
 #include "common.cuh"
@@ -32,17 +44,24 @@
 namespace nvfp4 {
 namespace gq {
 
-constexpr int BM = 128;           // pairs per tile
-constexpr int BN = 256;           // output columns per CTA
-constexpr int BK = 64;            // K elements per stage (128 bytes of bf16)
-constexpr int STAGES = 4;
-constexpr int PRODUCERS = 128;    // warps 0-3
-constexpr int THREADS = 160;      // + MMA warp
-constexpr int A_STAGE = BM * 128;  // 16 KiB
-constexpr int B_STAGE = BN * 128;  // 32 KiB
-constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE);
+constexpr int BM = 128;            // pairs per tile
+constexpr int BN = 256;            // output columns per unit
+constexpr int BK = 64;             // K elements per k-step (128 bytes of bf16)
+constexpr int XS = 4;              // x stages
+constexpr int WS = 3;              // bf16 weight stages
+constexpr int RS = 6;              // raw code stages
+constexpr int DEQ_WARPS = 8;
+constexpr int EPI_WARPS = 4;
+constexpr int THREADS = 32 * (4 + DEQ_WARPS + EPI_WARPS);  // 512
+constexpr int X_STAGE = BM * 128;  // 16 KiB
+constexpr int W_STAGE = BN * 128;  // 32 KiB
+constexpr int R_STAGE = BN * 32;   // 8 KiB of codes
+constexpr int SMEM_X = 0;
+constexpr int SMEM_W = SMEM_X + XS * X_STAGE;
+constexpr int SMEM_R = SMEM_W + WS * W_STAGE;
+constexpr int SMEM_BYTES = SMEM_R + RS * R_STAGE;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
-constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TMEM_COLS = 512;  // two 256-column accumulators
 
 // Workspace: [0] number of tiles; then tile_expert, tile_row0, tile_rows
 // (max_tiles each) and the permutation (P entries), all int32.
@@ -123,11 +142,6 @@ __global__ void __launch_bounds__(ROUTE_THREADS) k_route(const int32_t* __restri
 // K-major tile (rows of 128 bytes, 8-row atoms of 1024 bytes).
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t c) { return r * 128u + ((c ^ (r & 7u)) << 4); }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool pred) {
-  const uint32_t n = pred ? 16u : 0u;  // zero-fill when the source row does not exist
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
-}
-
 // kind::f16 instruction descriptor: fp32 accumulate (bits 4-5 = 1), A and B
 // bf16 (bits 7-9, 10-12 = 1), K-major, N >> 3 (bits 17-22), M >> 4 (24-28).
 __host__ __device__ constexpr uint32_t f16_idesc() {
@@ -142,45 +156,87 @@ __device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uin
       : "memory");
 }
 
+// Four rows (r0..r3) of 64 bf16 of x at column c0 into 512 consecutive
+// bytes of a 128-byte-swizzled stage.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int c0, int r0, int r1, int r2,
+                                            int r3, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Eight e2m1 codes times the fp32 block scale, rounded to bf16 (two per
+// 32-bit word): the same arithmetic as the dequantize kernel.
+__device__ __forceinline__ uint4 dequant8_bf16(uint32_t w, float sd) {
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float lo, hi;
+    e2m1x2_to_f32((w >> (8 * i)) & 0xFFu, lo, hi);
+    o[i] = pack_bf16x2(lo * sd, hi * sd);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 struct Args {
-  const __nv_bfloat16* x;
-  const uint32_t* wc;
   const uint8_t* wsc;
   const float* g;
   __nv_bfloat16* y;
   Workspace ws;
   int N, K, topk;
+  int n_tiles_n;  // column tiles per pair tile
 };
 
-__global__ void __launch_bounds__(THREADS, 1) k_gather_mma(Args a) {
+// Unit u -> (pair tile, first output column).
+__device__ __forceinline__ void unit_coords(uint32_t u, uint32_t n_tiles_n, uint32_t& tile, uint32_t& n0) {
+  tile = u / n_tiles_n;
+  n0 = (u - tile * n_tiles_n) * (uint32_t)BN;
+}
+
+__global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant__ CUtensorMap tmap_x,
+                                                           const __grid_constant__ CUtensorMap tmap_w, Args a) {
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[STAGES];
-  __shared__ __align__(8) uint64_t empty_bar[STAGES];
-  __shared__ __align__(8) uint64_t accum_bar;
+  __shared__ __align__(8) uint64_t x_full[XS], x_empty[XS];
+  __shared__ __align__(8) uint64_t w_full[WS], w_empty[WS];
+  __shared__ __align__(8) uint64_t r_full[RS], r_empty[RS];
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
   __shared__ uint32_t tmem_holder;
-  __shared__ int rows_pair[BM];
-
-  const int tile = blockIdx.x;
-  const int ntiles = *a.ws.ntiles;
-  if (tile >= ntiles) return;  // uniform per CTA, before any barrier or TMEM use
-  const int e = a.ws.tile_expert[tile], row0 = a.ws.tile_row0[tile], nrows = a.ws.tile_rows[tile];
-  const int n0 = blockIdx.y * BN;
+  __shared__ int abort_flag;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t units = (uint32_t)(*a.ws.ntiles) * (uint32_t)a.n_tiles_n;
+  const uint32_t kb_count = (uint32_t)a.K / BK;
 
-  if (threadIdx.x < BM) rows_pair[threadIdx.x] = threadIdx.x < nrows ? a.ws.perm[row0 + threadIdx.x] : -1;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(smem_u32(&full_bar[s]), PRODUCERS);
-      mbar_init(smem_u32(&empty_bar[s]), 1);
+    for (int s = 0; s < XS; ++s) {
+      mbar_init(smem_u32(&x_full[s]), 1);
+      mbar_init(smem_u32(&x_empty[s]), 1);
     }
-    mbar_init(smem_u32(&accum_bar), 1);
+    for (int s = 0; s < WS; ++s) {
+      mbar_init(smem_u32(&w_full[s]), DEQ_WARPS);
+      mbar_init(smem_u32(&w_empty[s]), 1);
+    }
+    for (int s = 0; s < RS; ++s) {
+      mbar_init(smem_u32(&r_full[s]), 1);
+      mbar_init(smem_u32(&r_empty[s]), DEQ_WARPS);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&acc_full[s]), 1);
+      mbar_init(smem_u32(&acc_empty[s]), EPI_WARPS);
+    }
+    abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 4) {
+  if (warp == 2) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_holder)),
                  "r"(TMEM_COLS)
                  : "memory");
@@ -190,105 +246,240 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(Args a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
-  const int kb_count = a.K / BK;
-  bool ok = true;
 
-  if (warp < 4) {
-    // ------------------------------------------------------------ producers
-    const int t = threadIdx.x;  // 0..127
-    const float d = a.g ? __ldg(a.g + e) / kGlobalEncode : 1.0f;
-    const uint32_t kwords = (uint32_t)a.K / 8u;    // code words per weight row
-    const uint32_t kscales = (uint32_t)a.K / 16u;  // scale bytes per weight row
-    const size_t wrow_base = (size_t)e * a.N;
-    for (int kb = 0; kb < kb_count && ok; ++kb) {
-      const int s = kb % STAGES;
-      if (!mbar_wait(smem_u32(&empty_bar[s]), ((kb / STAGES) & 1) ^ 1)) {
-        ok = false;
+  if (warp == 0) {
+    // ------------------------------------------------------------ x gather
+    // lane l owns pair rows 4l..4l+3 of the tile; rows past the tile's end
+    // gather token 0 (their accumulator rows are never stored)
+    uint32_t it = 0;
+    for (uint32_t u = blockIdx.x; u < units; u += gridDim.x) {
+      uint32_t tile, n0;
+      unit_coords(u, (uint32_t)a.n_tiles_n, tile, n0);
+      const int row0 = a.ws.tile_row0[tile], nrows = a.ws.tile_rows[tile];
+      int tok[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 4 * lane + i;
+        tok[i] = r < nrows ? a.ws.perm[row0 + r] / a.topk : 0;
+      }
+      bool ok = true;
+      for (uint32_t kb = 0; kb < kb_count; ++kb, ++it) {
+        const uint32_t s = it % XS;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&x_empty[s]), ((it / XS) & 1u) ^ 1u)) ||
+            *(volatile int*)&abort_flag) {
+          ok = false;
+          break;
+        }
+        const uint32_t bar = smem_u32(&x_full[s]);
+        if (lane == 0) mbar_expect_tx(bar, X_STAGE);
+        __syncwarp();
+        tma_gather4(sbase + SMEM_X + s * X_STAGE + 512u * lane, &tmap_x, (int)(kb * BK), tok[0], tok[1], tok[2], tok[3],
+                    bar);
+      }
+      if (!ok) {
+        if (lane == 0) abort_flag = 1;
         break;
       }
-      const uint32_t sa = sbase + s * A_STAGE, sb = sbase + STAGES * A_STAGE + s * B_STAGE;
-      // x rows of the tile: 128 rows x 8 chunks of 16 bytes
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int u = t + i * PRODUCERS;  // 0..1023
-        const int r = u >> 3, c = u & 7;
-        const int pid = rows_pair[r];
-        const int tok = pid >= 0 ? pid / a.topk : 0;
-        const __nv_bfloat16* src = a.x + (size_t)tok * a.K + kb * BK + c * 8;
-        cp_async16(sa + sw128(r, c), src, pid >= 0);
-      }
-      // weight tile: 256 rows x 4 blocks of 16, dequantized to bf16
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int u = t + i * PRODUCERS;  // 0..1023
-        const int r = u >> 2, blk = u & 3;
-        const int n = n0 + r;
-        uint32_t out[8];
-        if (n < a.N) {
-          const size_t wr = wrow_base + n;
-          const uint2 cw = __ldg(reinterpret_cast<const uint2*>(a.wc + wr * kwords + (kb * BK) / 8) + blk);
-          const float sd = e4m3_to_f32(__ldg(a.wsc + wr * kscales + (kb * BK) / 16 + blk)) * d;
-          const uint32_t words[2] = {cw.x, cw.y};
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t c0 = words[h] >> (8 * j), c1 = c0 >> 4;
-              out[h * 4 + j] = pack_bf16x2(e2m1_value(c0) * sd, e2m1_value(c1) * sd);
-            }
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) out[j] = 0u;
+    }
+    // the last stages must land before the CTA exits
+    const uint32_t first = it > (uint32_t)XS ? it - XS : 0;
+    for (uint32_t i = first; i < it; ++i) mbar_wait(smem_u32(&x_full[i % XS]), (i / XS) & 1u);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ code stream
+    const bool leader = elect_one();
+    uint32_t it = 0;
+    for (uint32_t u = blockIdx.x; u < units; u += gridDim.x) {
+      uint32_t tile, n0;
+      unit_coords(u, (uint32_t)a.n_tiles_n, tile, n0);
+      const int wrow = a.ws.tile_expert[tile] * a.N + (int)n0;
+      bool ok = true;
+      for (uint32_t kb = 0; kb < kb_count; ++kb, ++it) {
+        const uint32_t s = it % RS;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&r_empty[s]), ((it / RS) & 1u) ^ 1u)) ||
+            *(volatile int*)&abort_flag) {
+          ok = false;
+          break;
         }
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sb + sw128(r, 2 * blk)), "r"(out[0]),
-                     "r"(out[1]), "r"(out[2]), "r"(out[3])
-                     : "memory");
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sb + sw128(r, 2 * blk + 1)), "r"(out[4]),
-                     "r"(out[5]), "r"(out[6]), "r"(out[7])
-                     : "memory");
+        if (leader) {
+          const uint32_t bar = smem_u32(&r_full[s]);
+          mbar_expect_tx(bar, R_STAGE);
+          tma_load_2d(sbase + SMEM_R + s * R_STAGE, &tmap_w, (int)(kb * 32u), wrow, bar);
+        }
+        __syncwarp();
       }
-      asm volatile("cp.async.wait_all;" ::: "memory");
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // make st.shared / cp.async visible to tcgen05
-      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&full_bar[s])) : "memory");
-    }
-    // ------------------------------------------------------------ epilogue
-    const bool acc_ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&accum_bar), 0) && ok);
-    tc_fence_after();
-    if (acc_ok) {
-      const int r = warp * 32 + lane;  // TMEM lane = pair row of the tile
-      const int pid = rows_pair[r];
-      for (int c = 0; c < BN; c += 32) {
-        float v[32];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
-        const int col = n0 + c;
-        if (pid >= 0 && col < a.N) store_out<__nv_bfloat16>(a.y + (size_t)pid * a.N + col, v, min(32, a.N - col));
+      if (!ok) {
+        if (lane == 0) abort_flag = 1;
+        break;
       }
     }
-  } else {
+    const uint32_t first = it > (uint32_t)RS ? it - RS : 0;
+    if (leader)
+      for (uint32_t i = first; i < it; ++i) mbar_wait(smem_u32(&r_full[i % RS]), (i / RS) & 1u);
+    __syncwarp();
+  } else if (warp == 2) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = f16_idesc();
-      for (int kb = 0; kb < kb_count; ++kb) {
-        const int s = kb % STAGES;
-        if (!mbar_wait(smem_u32(&full_bar[s]), (kb / STAGES) & 1)) break;
+    const bool leader = elect_one();
+    const uint32_t idesc = f16_idesc();
+    const uint64_t x_base = kmajor_sw128_desc(sbase + SMEM_X), w_base = kmajor_sw128_desc(sbase + SMEM_W);
+    const uint32_t x_hi = (uint32_t)(x_base >> 32), w_hi = (uint32_t)(w_base >> 32);
+    auto mk = [](uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; };
+    uint32_t xit = 0, wit = 0, ui = 0;
+    bool ok = true;
+    for (uint32_t u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
+      const uint32_t acc = ui & 1u;
+      if (ui >= 2) {  // the epilogue has drained this accumulator's previous unit
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_empty[acc]), ((ui >> 1) - 1u) & 1u))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t sa = sbase + s * A_STAGE, sb = sbase + STAGES * A_STAGE + s * B_STAGE;
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          mma_bf16(tmem, kmajor_sw128_desc(sa + 32 * j), kmajor_sw128_desc(sb + 32 * j), idesc, (kb | j) != 0);
-        mma_commit(smem_u32(&empty_bar[s]));
       }
-      mma_commit(smem_u32(&accum_bar));
+      for (uint32_t kb = 0; kb < kb_count; ++kb, ++xit, ++wit) {
+        const uint32_t xs = xit % XS, ws = wit % WS;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&x_full[xs]), (xit / XS) & 1u) &&
+                                         mbar_wait(smem_u32(&w_full[ws]), (wit / WS) & 1u)) ||
+            *(volatile int*)&abort_flag) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (leader) {
+          const uint32_t xl = (uint32_t)x_base + xs * (X_STAGE >> 4), wl = (uint32_t)w_base + ws * (W_STAGE >> 4);
+#pragma unroll
+          for (uint32_t j = 0; j < 4; ++j)
+            mma_bf16(tmem + acc * 256u, mk(xl + 2 * j, x_hi), mk(wl + 2 * j, w_hi), idesc, (kb | j) != 0);
+          mma_commit(smem_u32(&x_empty[xs]));
+          mma_commit(smem_u32(&w_empty[ws]));
+          if (kb + 1 == kb_count) mma_commit(smem_u32(&acc_full[acc]));
+        }
+        __syncwarp();
+      }
+    }
+    if (!ok && lane == 0) abort_flag = 1;
+  } else if (warp >= 4 && warp < 4 + DEQ_WARPS) {
+    // ------------------------------------------------------------ dequantize
+    const uint32_t t = threadIdx.x - 128u;  // weight row of the unit, 0..255
+    const uint32_t kscales = (uint32_t)a.K / 16u;
+    uint32_t rit = 0, wit = 0;
+    bool ok = true;
+    for (uint32_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      uint32_t tile, n0;
+      unit_coords(u, (uint32_t)a.n_tiles_n, tile, n0);
+      const int e = a.ws.tile_expert[tile];
+      const bool valid = n0 + t < (uint32_t)a.N;
+      const float d = a.g ? __ldg(a.g + e) / kGlobalEncode : 1.0f;
+      const uint32_t* srow = reinterpret_cast<const uint32_t*>(a.wsc + ((size_t)e * a.N + n0 + t) * kscales);
+      uint32_t sc = valid ? __ldg(srow) : 0u;  // four block scales of k-step 0
+      for (uint32_t kb = 0; kb < kb_count; ++kb, ++rit, ++wit) {
+        const uint32_t rs = rit % RS, ws = wit % WS;
+        const uint32_t sc_next = (valid && kb + 1 < kb_count) ? __ldg(srow + kb + 1) : 0u;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&r_full[rs]), (rit / RS) & 1u) &&
+                                         mbar_wait(smem_u32(&w_empty[ws]), ((wit / WS) & 1u) ^ 1u)) ||
+            *(volatile int*)&abort_flag) {
+          ok = false;
+          break;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(smem + SMEM_R + rs * R_STAGE + t * 32u);
+        const uint4 c0 = src[0], c1 = src[1];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&r_empty[rs]));  // codes are in registers
+        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const uint32_t dst = sbase + SMEM_W + ws * W_STAGE;
+#pragma unroll
+        for (uint32_t c = 0; c < 8; ++c) {  // 16-byte chunk c holds K elements 8c..8c+7 (block c/2)
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (valid) v = dequant8_bf16(words[c], e4m3_to_f32((sc >> (8 * (c >> 1))) & 0xFFu) * d);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + sw128(t, c)), "r"(v.x), "r"(v.y),
+                       "r"(v.z), "r"(v.w)
+                       : "memory");
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // st.shared visible to tcgen05.mma
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&w_full[ws]));
+        sc = sc_next;
+      }
+    }
+    if (!ok && lane == 0) abort_flag = 1;
+  } else if (warp >= 4 + DEQ_WARPS) {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t q = warp & 3u;  // TMEM lane quarter
+    const uint32_t r = q * 32u + lane;
+    uint32_t ui = 0;
+    for (uint32_t u = blockIdx.x; u < units; u += gridDim.x, ++ui) {
+      uint32_t tile, n0;
+      unit_coords(u, (uint32_t)a.n_tiles_n, tile, n0);
+      const int row0 = a.ws.tile_row0[tile], nrows = a.ws.tile_rows[tile];
+      const int pid = (int)r < nrows ? a.ws.perm[row0 + r] : -1;
+      const uint32_t acc = ui & 1u;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[acc]), (ui >> 1) & 1u));
+      tc_fence_after();
+      if (!ok || *(volatile int*)&abort_flag) {
+        if (lane == 0) abort_flag = 1;
+        break;
+      }
+      for (uint32_t c = 0; c < (uint32_t)BN; c += 32) {
+        float v[32];
+        tmem_ld32(tmem + ((q * 32u) << 16) + acc * 256u + c, v);
+        const int col = (int)(n0 + c);
+        if (pid >= 0 && col < a.N) {  // N % 16 == 0: a chunk has 32 or 16 columns
+          __nv_bfloat16* dst = a.y + (size_t)pid * a.N + col;
+          const uint4 h0 = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                      pack_bf16x2(v[6], v[7]));
+          const uint4 h1 = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
+                                      pack_bf16x2(v[14], v[15]));
+          reinterpret_cast<uint4*>(dst)[0] = h0;
+          reinterpret_cast<uint4*>(dst)[1] = h1;
+          if (col + 32 <= a.N) {
+            const uint4 h2 = make_uint4(pack_bf16x2(v[16], v[17]), pack_bf16x2(v[18], v[19]),
+                                        pack_bf16x2(v[20], v[21]), pack_bf16x2(v[22], v[23]));
+            const uint4 h3 = make_uint4(pack_bf16x2(v[24], v[25]), pack_bf16x2(v[26], v[27]),
+                                        pack_bf16x2(v[28], v[29]), pack_bf16x2(v[30], v[31]));
+            reinterpret_cast<uint4*>(dst)[2] = h2;
+            reinterpret_cast<uint4*>(dst)[3] = h3;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
     }
   }
   __syncwarp();  // lanes that skipped a one-lane role loop wait for it before the CTA barrier
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 2) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
   }
+}
+
+// x [T, K] bf16: box 64 x 1 rows (tile::gather4 takes four rows of it),
+// 128-byte swizzle.  Codes [E*N rows, K/2 bytes]: box 32 B x 256 rows.
+inline bool make_maps(CUtensorMap* mx, CUtensorMap* mw, const void* x, const uint32_t* wc, uint64_t T, uint64_t K,
+                      uint64_t EN) {
+  auto fn = tc::encode_fn();
+  if (!fn) return false;
+  {
+    cuuint64_t dims[2] = {K, T};
+    cuuint64_t strides[1] = {K * 2};
+    cuuint32_t box[2] = {64, 1};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  {
+    cuuint64_t dims[2] = {K / 2, EN};
+    cuuint64_t strides[1] = {K / 2};
+    cuuint32_t box[2] = {32, (cuuint32_t)BN};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint32_t*>(wc), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  return true;
 }
 
 }  // namespace gq
@@ -306,13 +497,16 @@ inline nvfp4_status gather_qmm_launch(const void* x, const uint32_t* w_codes, co
   }
   const int64_t P = T * topk;
   Workspace ws = carve(workspace, P, E);
+  CUtensorMap mx, mw;
+  if (!make_maps(&mx, &mw, x, w_codes, (uint64_t)T, (uint64_t)K, (uint64_t)(E * N))) {
+    snprintf(msg, msg_len, "[gather_qmm] cuTensorMapEncodeTiled failed");
+    return NVFP4_ERR_CUDA;
+  }
   k_route<<<1, ROUTE_THREADS, 0, stream>>>(idx, (int)P, (int)E, (int)N, ws, static_cast<__nv_bfloat16*>(y));
   cudaError_t err = cudaGetLastError();
   if (err == cudaSuccess) err = cudaFuncSetAttribute(k_gather_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
   if (err == cudaSuccess) {
     Args a;
-    a.x = static_cast<const __nv_bfloat16*>(x);
-    a.wc = w_codes;
     a.wsc = w_scales;
     a.g = g;
     a.y = static_cast<__nv_bfloat16*>(y);
@@ -320,8 +514,10 @@ inline nvfp4_status gather_qmm_launch(const void* x, const uint32_t* w_codes, co
     a.N = (int)N;
     a.K = (int)K;
     a.topk = (int)topk;
-    dim3 grid((unsigned)max_tiles(P, E), (unsigned)((N + BN - 1) / BN));
-    k_gather_mma<<<grid, THREADS, SMEM_ALLOC, stream>>>(a);
+    a.n_tiles_n = (int)((N + BN - 1) / BN);
+    const int64_t max_units = max_tiles(P, E) * a.n_tiles_n;
+    const unsigned grid = (unsigned)(max_units < sm_count ? max_units : sm_count);
+    k_gather_mma<<<grid, THREADS, SMEM_ALLOC, stream>>>(mx, mw, a);
     err = cudaGetLastError();
   }
   if (err != cudaSuccess) {
@@ -329,7 +525,6 @@ inline nvfp4_status gather_qmm_launch(const void* x, const uint32_t* w_codes, co
     return NVFP4_ERR_CUDA;
   }
   msg[0] = '\0';
-  (void)sm_count;
   return NVFP4_OK;
 }
 
