@@ -8,28 +8,31 @@
 //
 // Two kernels:
 //  1. k_route (one CTA): histogram of the T*topk (token, slot) pairs by
-//     expert, exclusive prefix sum, a list of 128-pair tiles (expert, first
+//     expert, exclusive prefix sum, a list of 256-pair tiles (expert, first
 //     row of the expert's run, rows) and the permutation of pair ids grouped
 //     by expert.  Expert ids outside [0, E) set the device error word and
 //     their output rows are written as zeros.
-//  2. k_gather_mma, persistent (one CTA per SM): work units are (128-pair
+//  2. k_gather_mma, persistent (one CTA per SM): work units are (256-pair
 //     tile, 256 output columns), handed out round-robin, the column tiles of
 //     a pair tile adjacent so that CTAs running together share x rows and the
-//     expert's weight in L2.  Warp roles:
-//       warp 0     gathers the tile's x rows with TMA tile::gather4 (4 rows
-//                  per copy) into 128-byte-swizzled K-major stages;
-//       warp 1     streams the expert's NVFP4 codes [256 rows x 32 B] per
+//     expert's weight in L2.  Each dequantized weight stage feeds the MMAs of
+//     both 128-pair halves of the tile (two accumulators), which halves the
+//     dequantization per MMA.  Warp roles:
+//       warps 0-7  gather the tile's x rows with TMA tile::gather4 (4 rows
+//                  per copy, 4 copies per warp and k-step: one issuing warp
+//                  cannot keep up with the tensor core) into
+//                  128-byte-swizzled K-major stages;
+//       warp 8     streams the expert's NVFP4 codes [256 rows x 32 B] per
 //                  k-step with TMA;
-//       warp 2     allocates TMEM and issues tcgen05 kind::f16 MMAs (M = 128
-//                  pairs, N = 256 columns, K = 16) from one elected lane into
-//                  one of two fp32 accumulators;
-//       warps 4-11 dequantize the codes to bf16 (one weight row per thread,
-//                  block scale from global memory one k-step ahead) into the
-//                  swizzled B stages, rounding exactly as the dequantize
-//                  kernel does;
-//       warps 12-15 drain an accumulator (one TMEM lane quarter each) and
-//                  scatter each pair row to y[t, j, :] while the MMAs of the
-//                  next unit run on the other accumulator.
+//       warp 9     allocates TMEM and issues tcgen05 kind::f16 MMAs (M = 128
+//                  pairs, N = 256 columns, K = 16) from one elected lane, one
+//                  fp32 accumulator per 128-pair half;
+//       warps 12-15 drain the accumulators (one TMEM lane quarter each) and
+//                  scatter each pair row to y[t, j, :];
+//       warps 16-31 dequantize the codes to bf16 (two threads per weight
+//                  row, block scales from global memory one k-step ahead)
+//                  into the swizzled B stages, rounding exactly as the
+//                  dequantize kernel does.
 // The contraction is on the bf16 tensor pipe: both operands are bf16, as
 // the method requires of the materialized weight.  Every wait is bounded.
 #pragma once
@@ -44,16 +47,19 @@
 namespace nvfp4 {
 namespace gq {
 
-constexpr int BM = 128;            // pairs per tile
+constexpr int BM = 256;            // pairs per tile
+constexpr int MMA_M = 128;         // pairs per MMA (one accumulator per half tile)
 constexpr int BN = 256;            // output columns per unit
 constexpr int BK = 64;             // K elements per k-step (128 bytes of bf16)
-constexpr int XS = 4;              // x stages
+constexpr int XS = 3;              // x stages
 constexpr int WS = 3;              // bf16 weight stages
-constexpr int RS = 6;              // raw code stages
-constexpr int DEQ_WARPS = 8;
+constexpr int RS = 4;              // raw code stages
+constexpr int GATHER_WARPS = 8;
+constexpr int DEQ_WARPS = 16;
 constexpr int EPI_WARPS = 4;
-constexpr int THREADS = 32 * (4 + DEQ_WARPS + EPI_WARPS);  // 512
-constexpr int X_STAGE = BM * 128;  // 16 KiB
+constexpr int W_CODES = 8, W_MMA = 9, W_EPI = 12, W_DEQ = 16;  // first warp of each role
+constexpr int THREADS = 32 * (W_DEQ + DEQ_WARPS);                  // 1024
+constexpr int X_STAGE = BM * 128;  // 32 KiB: two 16 KiB MMA operands
 constexpr int W_STAGE = BN * 128;  // 32 KiB
 constexpr int R_STAGE = BN * 32;   // 8 KiB of codes
 constexpr int SMEM_X = 0;
@@ -61,7 +67,7 @@ constexpr int SMEM_W = SMEM_X + XS * X_STAGE;
 constexpr int SMEM_R = SMEM_W + WS * W_STAGE;
 constexpr int SMEM_BYTES = SMEM_R + RS * R_STAGE;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
-constexpr uint32_t TMEM_COLS = 512;  // two 256-column accumulators
+constexpr uint32_t TMEM_COLS = 512;  // two 256-column accumulators (one per half tile)
 
 // Workspace: [0] number of tiles; then tile_expert, tile_row0, tile_rows
 // (max_tiles each) and the permutation (P entries), all int32.
@@ -96,42 +102,118 @@ __host__ __device__ inline Workspace carve(void* base, int64_t P, int64_t E) {
 // 1. routing
 // ---------------------------------------------------------------------------
 constexpr int ROUTE_THREADS = 1024;
-constexpr int MAX_E = 1024;
+constexpr int ROUTE_WARPS = ROUTE_THREADS / 32;
+constexpr int ROUTE_CHUNK = 16;  // expert ids each lane loads before it processes them
+constexpr int MAX_E = 1024;      // one expert per thread in the scans
 
+// Dynamic shared memory of k_route: per-warp expert histograms [32][E],
+// then expert offsets and first tile indices [E] each.
+__host__ __device__ inline size_t route_smem_bytes(int64_t E) { return (size_t)(ROUTE_WARPS + 2) * E * 4; }
+
+// Exclusive prefix sum of one value per thread over the CTA (1024 threads);
+// also returns the total.  `tmp` holds ROUTE_WARPS ints.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* tmp, int& total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += t;
+  }
+  if (lane == 31) tmp[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int y = tmp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, y, o);
+      if (lane >= o) y += t;
+    }
+    tmp[lane] = y;  // inclusive over warps
+  }
+  __syncthreads();
+  total = tmp[ROUTE_WARPS - 1];
+  const int r = x - v + (w > 0 ? tmp[w - 1] : 0);
+  __syncthreads();  // tmp may be reused by the caller
+  return r;
+}
+
+// Pass 1 counts the pairs of each expert per warp (shared-memory atomics on
+// the warp's own histogram); the per-warp counts become per-warp bases
+// inside each expert's run; pass 2 gives every pair a slot with an atomic
+// on its warp's base.  The order of the pairs inside an expert's run is not
+// part of the result (each output row depends on its own pair only).
 __global__ void __launch_bounds__(ROUTE_THREADS) k_route(const int32_t* __restrict__ idx, int P, int E, int N,
                                                          Workspace ws, __nv_bfloat16* __restrict__ y) {
-  __shared__ int cnt[MAX_E];
-  __shared__ int cursor[MAX_E];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  extern __shared__ int rsm[];
+  __shared__ int scan_tmp[ROUTE_WARPS];
+  int* whist = rsm;                     // [ROUTE_WARPS][E]
+  int* off = rsm + ROUTE_WARPS * E;     // [E] first row of each expert's run
+  int* tile0 = off + E;                 // [E] first tile of each expert
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < ROUTE_WARPS * E; i += blockDim.x) whist[i] = 0;
   __syncthreads();
-  for (int p = threadIdx.x; p < P; p += blockDim.x) {
-    const int e = __ldg(idx + p);
-    if (e >= 0 && e < E) {
-      atomicAdd(&cnt[e], 1);
-    } else {
-      atomicOr(&g_device_error, (unsigned)kDevErrIndex);
-      for (int n = 0; n < N; ++n) y[(size_t)p * N + n] = __float2bfloat16_rn(0.0f);
+  for (int base0 = w * 32; base0 < P; base0 += ROUTE_THREADS * ROUTE_CHUNK) {
+    int ev[ROUTE_CHUNK];
+#pragma unroll
+    for (int i = 0; i < ROUTE_CHUNK; ++i) {
+      const int p = base0 + i * ROUTE_THREADS + lane;
+      ev[i] = p < P ? __ldg(idx + p) : -1;
     }
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int off = 0, nt = 0;
-    for (int e = 0; e < E; ++e) {
-      cursor[e] = off;
-      for (int r = 0; r < cnt[e]; r += BM) {
-        ws.tile_expert[nt] = e;
-        ws.tile_row0[nt] = off + r;
-        ws.tile_rows[nt] = min(BM, cnt[e] - r);
-        ++nt;
+#pragma unroll
+    for (int i = 0; i < ROUTE_CHUNK; ++i) {
+      const int p = base0 + i * ROUTE_THREADS + lane;
+      const int e = ev[i];
+      if (e >= 0 && e < E) {
+        atomicAdd(&whist[w * E + e], 1);
+      } else if (p < P) {
+        atomicOr(&g_device_error, (unsigned)kDevErrIndex);
+        for (int n = 0; n < N; ++n) y[(size_t)p * N + n] = __float2bfloat16_rn(0.0f);
       }
-      off += cnt[e];
     }
-    *ws.ntiles = nt;
   }
   __syncthreads();
-  for (int p = threadIdx.x; p < P; p += blockDim.x) {
-    const int e = __ldg(idx + p);
-    if (e >= 0 && e < E) ws.perm[atomicAdd(&cursor[e], 1)] = p;
+  // thread e: per-warp bases inside expert e's run, its count and tile count
+  int cnt = 0, ntl = 0;
+  if (threadIdx.x < E) {
+    const int e = threadIdx.x;
+    for (int k = 0; k < ROUTE_WARPS; ++k) {
+      const int c = whist[k * E + e];
+      whist[k * E + e] = cnt;
+      cnt += c;
+    }
+    ntl = (cnt + BM - 1) / BM;
+  }
+  int total_rows, total_tiles;
+  const int o = block_exclusive_scan(cnt, scan_tmp, total_rows);
+  const int t0 = block_exclusive_scan(ntl, scan_tmp, total_tiles);
+  if (threadIdx.x < E) {
+    const int e = threadIdx.x;
+    off[e] = o;
+    tile0[e] = t0;
+    for (int k = 0; k < ntl; ++k) {
+      ws.tile_expert[t0 + k] = e;
+      ws.tile_row0[t0 + k] = o + k * BM;
+      ws.tile_rows[t0 + k] = min(BM, cnt - k * BM);
+    }
+  }
+  if (threadIdx.x == 0) *ws.ntiles = total_tiles;
+  __syncthreads();
+  for (int i = threadIdx.x; i < ROUTE_WARPS * E; i += blockDim.x) whist[i] += off[i % E];
+  __syncthreads();
+  for (int base0 = w * 32; base0 < P; base0 += ROUTE_THREADS * ROUTE_CHUNK) {
+    int ev[ROUTE_CHUNK];
+#pragma unroll
+    for (int i = 0; i < ROUTE_CHUNK; ++i) {
+      const int p = base0 + i * ROUTE_THREADS + lane;
+      ev[i] = p < P ? __ldg(idx + p) : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < ROUTE_CHUNK; ++i) {
+      const int p = base0 + i * ROUTE_THREADS + lane;
+      const int e = ev[i];
+      if (e >= 0 && e < E) ws.perm[atomicAdd(&whist[w * E + e], 1)] = p;
+    }
   }
 }
 
@@ -145,7 +227,7 @@ __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t c) { return r * 1
 // kind::f16 instruction descriptor: fp32 accumulate (bits 4-5 = 1), A and B
 // bf16 (bits 7-9, 10-12 = 1), K-major, N >> 3 (bits 17-22), M >> 4 (24-28).
 __host__ __device__ constexpr uint32_t f16_idesc() {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(MMA_M >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
@@ -179,7 +261,12 @@ __device__ __forceinline__ uint4 dequant8_bf16(uint32_t w, float sd) {
   for (int i = 0; i < 4; ++i) {
     float lo, hi;
     e2m1x2_to_f32((w >> (8 * i)) & 0xFFu, lo, hi);
-    o[i] = pack_bf16x2(lo * sd, hi * sd);
+    // both products in one packed fp32x2 multiply (round-to-nearest per lane)
+    uint64_t p;
+    asm("{\n\t.reg .b64 a, b;\n\tmov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %3};\n\tmul.rn.f32x2 %0, a, b;\n\t}"
+        : "=l"(p)
+        : "f"(lo), "f"(hi), "f"(sd));
+    o[i] = pack_bf16x2(__uint_as_float((uint32_t)p), __uint_as_float((uint32_t)(p >> 32)));
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -206,7 +293,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
   __shared__ __align__(8) uint64_t x_full[XS], x_empty[XS];
   __shared__ __align__(8) uint64_t w_full[WS], w_empty[WS];
   __shared__ __align__(8) uint64_t r_full[RS], r_empty[RS];
-  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2];
+  __shared__ __align__(8) uint64_t acc_full, acc_empty;
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_flag;
 
@@ -218,7 +305,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < XS; ++s) {
-      mbar_init(smem_u32(&x_full[s]), 1);
+      mbar_init(smem_u32(&x_full[s]), GATHER_WARPS);
       mbar_init(smem_u32(&x_empty[s]), 1);
     }
     for (int s = 0; s < WS; ++s) {
@@ -229,14 +316,12 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
       mbar_init(smem_u32(&r_full[s]), 1);
       mbar_init(smem_u32(&r_empty[s]), DEQ_WARPS);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(smem_u32(&acc_full[s]), 1);
-      mbar_init(smem_u32(&acc_empty[s]), EPI_WARPS);
-    }
+    mbar_init(smem_u32(&acc_full), 1);
+    mbar_init(smem_u32(&acc_empty), EPI_WARPS);
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 2) {
+  if (warp == W_MMA) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_holder)),
                  "r"(TMEM_COLS)
                  : "memory");
@@ -247,10 +332,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
 
-  if (warp == 0) {
+  if (warp < GATHER_WARPS) {
     // ------------------------------------------------------------ x gather
-    // lane l owns pair rows 4l..4l+3 of the tile; rows past the tile's end
-    // gather token 0 (their accumulator rows are never stored)
+    // lane l < 8 of warp w owns pair rows 4q..4q+3, q = 8w + l; rows past the
+    // tile's end gather token 0 (their accumulator rows are never stored)
+    const uint32_t q = 8u * warp + (lane & 7u);
     uint32_t it = 0;
     for (uint32_t u = blockIdx.x; u < units; u += gridDim.x) {
       uint32_t tile, n0;
@@ -259,7 +345,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
       int tok[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int r = 4 * lane + i;
+        const int r = 4 * (int)q + i;
         tok[i] = r < nrows ? a.ws.perm[row0 + r] / a.topk : 0;
       }
       bool ok = true;
@@ -271,10 +357,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
           break;
         }
         const uint32_t bar = smem_u32(&x_full[s]);
-        if (lane == 0) mbar_expect_tx(bar, X_STAGE);
+        if (lane == 0) mbar_expect_tx(bar, X_STAGE / GATHER_WARPS);  // this warp's share of the stage
         __syncwarp();
-        tma_gather4(sbase + SMEM_X + s * X_STAGE + 512u * lane, &tmap_x, (int)(kb * BK), tok[0], tok[1], tok[2], tok[3],
-                    bar);
+        if (lane < 8)
+          tma_gather4(sbase + SMEM_X + s * X_STAGE + 512u * q, &tmap_x, (int)(kb * BK), tok[0], tok[1], tok[2], tok[3],
+                      bar);
       }
       if (!ok) {
         if (lane == 0) abort_flag = 1;
@@ -284,7 +371,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
     // the last stages must land before the CTA exits
     const uint32_t first = it > (uint32_t)XS ? it - XS : 0;
     for (uint32_t i = first; i < it; ++i) mbar_wait(smem_u32(&x_full[i % XS]), (i / XS) & 1u);
-  } else if (warp == 1) {
+  } else if (warp == W_CODES) {
     // ------------------------------------------------------------ code stream
     const bool leader = elect_one();
     uint32_t it = 0;
@@ -316,7 +403,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
     if (leader)
       for (uint32_t i = first; i < it; ++i) mbar_wait(smem_u32(&r_full[i % RS]), (i / RS) & 1u);
     __syncwarp();
-  } else if (warp == 2) {
+  } else if (warp == W_MMA) {
     // ------------------------------------------------------------ MMA issuer
     const bool leader = elect_one();
     const uint32_t idesc = f16_idesc();
@@ -326,9 +413,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
     uint32_t xit = 0, wit = 0, ui = 0;
     bool ok = true;
     for (uint32_t u = blockIdx.x; u < units && ok; u += gridDim.x, ++ui) {
-      const uint32_t acc = ui & 1u;
-      if (ui >= 2) {  // the epilogue has drained this accumulator's previous unit
-        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_empty[acc]), ((ui >> 1) - 1u) & 1u))) {
+      if (ui >= 1) {  // the epilogue has drained the previous unit's accumulators
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_empty), (ui - 1u) & 1u))) {
           ok = false;
           break;
         }
@@ -346,19 +432,25 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
         if (leader) {
           const uint32_t xl = (uint32_t)x_base + xs * (X_STAGE >> 4), wl = (uint32_t)w_base + ws * (W_STAGE >> 4);
 #pragma unroll
-          for (uint32_t j = 0; j < 4; ++j)
-            mma_bf16(tmem + acc * 256u, mk(xl + 2 * j, x_hi), mk(wl + 2 * j, w_hi), idesc, (kb | j) != 0);
+          for (uint32_t hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (uint32_t j = 0; j < 4; ++j)
+              mma_bf16(tmem + hh * 256u, mk(xl + hh * ((MMA_M * 128) >> 4) + 2 * j, x_hi), mk(wl + 2 * j, w_hi), idesc,
+                       (kb | j) != 0);
           mma_commit(smem_u32(&x_empty[xs]));
           mma_commit(smem_u32(&w_empty[ws]));
-          if (kb + 1 == kb_count) mma_commit(smem_u32(&acc_full[acc]));
+          if (kb + 1 == kb_count) mma_commit(smem_u32(&acc_full));
         }
         __syncwarp();
       }
     }
     if (!ok && lane == 0) abort_flag = 1;
-  } else if (warp >= 4 && warp < 4 + DEQ_WARPS) {
+  } else if (warp >= W_DEQ) {
     // ------------------------------------------------------------ dequantize
-    const uint32_t t = threadIdx.x - 128u;  // weight row of the unit, 0..255
+    // thread pair (2t, 2t+1) owns weight row t of the unit; half h takes K
+    // elements 32h..32h+31 of each k-step (blocks 2h, 2h+1)
+    const uint32_t tt = threadIdx.x - 32u * W_DEQ;
+    const uint32_t t = tt >> 1, h = tt & 1u;
     const uint32_t kscales = (uint32_t)a.K / 16u;
     uint32_t rit = 0, wit = 0;
     bool ok = true;
@@ -368,29 +460,30 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
       const int e = a.ws.tile_expert[tile];
       const bool valid = n0 + t < (uint32_t)a.N;
       const float d = a.g ? __ldg(a.g + e) / kGlobalEncode : 1.0f;
-      const uint32_t* srow = reinterpret_cast<const uint32_t*>(a.wsc + ((size_t)e * a.N + n0 + t) * kscales);
-      uint32_t sc = valid ? __ldg(srow) : 0u;  // four block scales of k-step 0
+      const unsigned short* srow =
+          reinterpret_cast<const unsigned short*>(a.wsc + ((size_t)e * a.N + n0 + t) * kscales) + h;
+      uint32_t sc = valid ? __ldg(srow) : 0u;  // this half's two block scales of k-step 0
       for (uint32_t kb = 0; kb < kb_count; ++kb, ++rit, ++wit) {
         const uint32_t rs = rit % RS, ws = wit % WS;
-        const uint32_t sc_next = (valid && kb + 1 < kb_count) ? __ldg(srow + kb + 1) : 0u;
+        const uint32_t sc_next = (valid && kb + 1 < kb_count) ? __ldg(srow + 2 * (kb + 1)) : 0u;
         if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&r_full[rs]), (rit / RS) & 1u) &&
                                          mbar_wait(smem_u32(&w_empty[ws]), ((wit / WS) & 1u) ^ 1u)) ||
             *(volatile int*)&abort_flag) {
           ok = false;
           break;
         }
-        const uint4* src = reinterpret_cast<const uint4*>(smem + SMEM_R + rs * R_STAGE + t * 32u);
-        const uint4 c0 = src[0], c1 = src[1];
+        const uint4 c0 = *reinterpret_cast<const uint4*>(smem + SMEM_R + rs * R_STAGE + t * 32u + h * 16u);
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&r_empty[rs]));  // codes are in registers
-        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const uint32_t words[4] = {c0.x, c0.y, c0.z, c0.w};
         const uint32_t dst = sbase + SMEM_W + ws * W_STAGE;
+        const float sd0 = e4m3_to_f32(sc & 0xFFu) * d, sd1 = e4m3_to_f32((sc >> 8) & 0xFFu) * d;
 #pragma unroll
-        for (uint32_t c = 0; c < 8; ++c) {  // 16-byte chunk c holds K elements 8c..8c+7 (block c/2)
+        for (uint32_t c = 0; c < 4; ++c) {  // chunk 4h + c holds K elements 8(4h+c).. (block 2h + c/2)
           uint4 v = make_uint4(0, 0, 0, 0);
-          if (valid) v = dequant8_bf16(words[c], e4m3_to_f32((sc >> (8 * (c >> 1))) & 0xFFu) * d);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + sw128(t, c)), "r"(v.x), "r"(v.y),
-                       "r"(v.z), "r"(v.w)
+          if (valid) v = dequant8_bf16(words[c], c < 2 ? sd0 : sd1);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + sw128(t, 4u * h + c)), "r"(v.x),
+                       "r"(v.y), "r"(v.z), "r"(v.w)
                        : "memory");
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // st.shared visible to tcgen05.mma
@@ -400,54 +493,56 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
       }
     }
     if (!ok && lane == 0) abort_flag = 1;
-  } else if (warp >= 4 + DEQ_WARPS) {
+  } else if (warp >= W_EPI && warp < W_EPI + EPI_WARPS) {
     // ------------------------------------------------------------ epilogue
     const uint32_t q = warp & 3u;  // TMEM lane quarter
-    const uint32_t r = q * 32u + lane;
     uint32_t ui = 0;
     for (uint32_t u = blockIdx.x; u < units; u += gridDim.x, ++ui) {
       uint32_t tile, n0;
       unit_coords(u, (uint32_t)a.n_tiles_n, tile, n0);
       const int row0 = a.ws.tile_row0[tile], nrows = a.ws.tile_rows[tile];
-      const int pid = (int)r < nrows ? a.ws.perm[row0 + r] : -1;
-      const uint32_t acc = ui & 1u;
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full[acc]), (ui >> 1) & 1u));
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&acc_full), ui & 1u));
       tc_fence_after();
       if (!ok || *(volatile int*)&abort_flag) {
         if (lane == 0) abort_flag = 1;
         break;
       }
-      for (uint32_t c = 0; c < (uint32_t)BN; c += 32) {
-        float v[32];
-        tmem_ld32(tmem + ((q * 32u) << 16) + acc * 256u + c, v);
-        const int col = (int)(n0 + c);
-        if (pid >= 0 && col < a.N) {  // N % 16 == 0: a chunk has 32 or 16 columns
-          __nv_bfloat16* dst = a.y + (size_t)pid * a.N + col;
-          const uint4 h0 = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                                      pack_bf16x2(v[6], v[7]));
-          const uint4 h1 = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]), pack_bf16x2(v[12], v[13]),
-                                      pack_bf16x2(v[14], v[15]));
-          reinterpret_cast<uint4*>(dst)[0] = h0;
-          reinterpret_cast<uint4*>(dst)[1] = h1;
-          if (col + 32 <= a.N) {
-            const uint4 h2 = make_uint4(pack_bf16x2(v[16], v[17]), pack_bf16x2(v[18], v[19]),
-                                        pack_bf16x2(v[20], v[21]), pack_bf16x2(v[22], v[23]));
-            const uint4 h3 = make_uint4(pack_bf16x2(v[24], v[25]), pack_bf16x2(v[26], v[27]),
-                                        pack_bf16x2(v[28], v[29]), pack_bf16x2(v[30], v[31]));
-            reinterpret_cast<uint4*>(dst)[2] = h2;
-            reinterpret_cast<uint4*>(dst)[3] = h3;
+#pragma unroll 1
+      for (uint32_t hh = 0; hh < 2; ++hh) {
+        const int r = (int)(hh * MMA_M + q * 32u + lane);  // pair row of the tile
+        const int pid = r < nrows ? a.ws.perm[row0 + r] : -1;
+        for (uint32_t c = 0; c < (uint32_t)BN; c += 32) {
+          float v[32];
+          tmem_ld32(tmem + ((q * 32u) << 16) + hh * 256u + c, v);
+          const int col = (int)(n0 + c);
+          if (pid >= 0 && col < a.N) {  // N % 16 == 0: a chunk has 32 or 16 columns
+            __nv_bfloat16* dst = a.y + (size_t)pid * a.N + col;
+            const uint4 h0 = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                        pack_bf16x2(v[6], v[7]));
+            const uint4 h1 = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                                        pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+            reinterpret_cast<uint4*>(dst)[0] = h0;
+            reinterpret_cast<uint4*>(dst)[1] = h1;
+            if (col + 32 <= a.N) {
+              const uint4 h2 = make_uint4(pack_bf16x2(v[16], v[17]), pack_bf16x2(v[18], v[19]),
+                                          pack_bf16x2(v[20], v[21]), pack_bf16x2(v[22], v[23]));
+              const uint4 h3 = make_uint4(pack_bf16x2(v[24], v[25]), pack_bf16x2(v[26], v[27]),
+                                          pack_bf16x2(v[28], v[29]), pack_bf16x2(v[30], v[31]));
+              reinterpret_cast<uint4*>(dst)[2] = h2;
+              reinterpret_cast<uint4*>(dst)[3] = h3;
+            }
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[acc]));
+      if (lane == 0) mbar_arrive(smem_u32(&acc_empty));
     }
   }
   __syncwarp();  // lanes that skipped a one-lane role loop wait for it before the CTA barrier
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == W_MMA) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
   }
@@ -502,8 +597,12 @@ inline nvfp4_status gather_qmm_launch(const void* x, const uint32_t* w_codes, co
     snprintf(msg, msg_len, "[gather_qmm] cuTensorMapEncodeTiled failed");
     return NVFP4_ERR_CUDA;
   }
-  k_route<<<1, ROUTE_THREADS, 0, stream>>>(idx, (int)P, (int)E, (int)N, ws, static_cast<__nv_bfloat16*>(y));
-  cudaError_t err = cudaGetLastError();
+  const size_t rsmem = route_smem_bytes(E);
+  cudaError_t err = cudaFuncSetAttribute(k_route, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem);
+  if (err == cudaSuccess) {
+    k_route<<<1, ROUTE_THREADS, rsmem, stream>>>(idx, (int)P, (int)E, (int)N, ws, static_cast<__nv_bfloat16*>(y));
+    err = cudaGetLastError();
+  }
   if (err == cudaSuccess) err = cudaFuncSetAttribute(k_gather_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
   if (err == cudaSuccess) {
     Args a;
