@@ -16,10 +16,13 @@ One step = one pass over every row of the hot path, each on its workload
 The headline ``value`` is the prefill qqmm op in TFLOP/s (2*M*N*K over the
 whole op: amaxes, quantizes and GEMM); every row's own metric, time and
 roofline are under ``rows``.  L2 (126 MB) is flushed before every row by
-writing a 256 MiB buffer, outside the row's timed window.  Every ABI call of
-a row is captured into its own CUDA graph; the timed step replays them back
-to back behind the flush, with CUDA events between them on the launching
-stream, so host-side call overhead is not inside any kernel's window.
+writing a 256 MiB buffer and then reading another 256 MiB buffer (the read
+evicts the flush's dirty lines, so their write-back to HBM is not charged to
+the row's first kernel), outside the row's timed window.  The calls of a row
+are captured as one CUDA graph with timing events recorded inside the graph
+before the first call and after every call; each timed step replays its own
+copy of the graph behind the flush, so neither host-side call overhead nor
+the graph's launch latency is inside any window.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs the same step on
 its own GPU (independent problems, no data-path collective): weak scaling;
@@ -115,36 +118,53 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 class Row:
     """One row of the hot path.  ``calls()`` lists its ABI calls as
-    (label, fn) with every output preallocated, so each call can be captured
-    into a CUDA graph; the timed step replays the graphs back to back, with
-    CUDA events between them on the launching stream."""
+    (label, fn) with every output preallocated.  The row is captured as one
+    CUDA graph with a timing event recorded inside the graph before the
+    first call and after every call (external events: the graph records
+    them each replay), so per-call and whole-row device times exclude the
+    graph's launch latency.  Each timed step replays its own copy of the
+    graph, so no event is overwritten before it is read."""
     name = ""
     launches = 0  # our kernels per run
 
     def __init__(self, nv, wl, dev, seed_offset):
         self.nv, self.wl, self.dev, self.off = nv, wl, dev, seed_offset
-        self.timers = []  # (label, start_event, end_event) of the timed steps
-        self.graphs = []  # (label, CUDAGraph)
+        self.copies = []  # (CUDAGraph, labels, events)
+        self.used = []    # copies replayed in the timed region
 
     def run(self):
         for _, fn in self.calls():
             fn()
 
-    def capture(self):
-        self.graphs = []
-        for label, fn in self.calls():
+    def capture(self, copies):
+        self.copies = []
+        for _ in range(copies):
+            calls = self.calls()
+            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(calls) + 1)]
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, capture_error_mode="thread_local"):
-                fn()
-            self.graphs.append((label, g))
+                evs[0].record()
+                for i, (_, fn) in enumerate(calls):
+                    fn()
+                    evs[i + 1].record()
+            self.copies.append((g, [label for label, _ in calls], evs))
 
-    def replay_timed(self):
-        for label, g in self.graphs:
-            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s.record()
-            g.replay()
-            e.record()
-            self.timers.append((label, s, e))
+    def replay(self, k, timed):
+        g = self.copies[k % len(self.copies)][0]
+        g.replay()
+        if timed:
+            self.used.append(k % len(self.copies))
+
+    def times(self):
+        """Mean ms per call and per row over the timed replays."""
+        per, row = {}, 0.0
+        for k in self.used:
+            _, labels, evs = self.copies[k]
+            for i, label in enumerate(labels):
+                per[label] = per.get(label, 0.0) + evs[i].elapsed_time(evs[i + 1])
+            row += evs[0].elapsed_time(evs[-1])
+        n = max(1, len(self.used))
+        return {k: v / n for k, v in per.items()}, row / n
 
 
 def _gen(wl, name, dev, off):
@@ -169,7 +189,7 @@ class Quant1G(Row):
         return [("amax", lambda: self.nv.amax(self.x, self.g)),
                 ("quantize", lambda: self.nv.nvfp4_quantize(self.x, self.g, "swizzled", self.codes, self.scales))]
 
-    def report(self, ms, peaks):
+    def report(self, ms, row_ms, peaks):
         q = ms["quantize"]
         return {"metric": "nvfp4 quantize GB/s", "unit": "GB/s", "value": self.bytes_q / q / 1e6,
                 "ms": ms, "roofline": {"bound": "hbm", "kernel": "k_nvfp4_quantize", "achieved": self.bytes_q / q / 1e6,
@@ -197,7 +217,7 @@ class Gemv(Row):
         return [("amax", lambda: self.nv.amax(self.x, self.g_x)),
                 ("qmv", lambda: self.nv.qmv(self.x, self.wc, self.ws, self.g_x, self.g_w, self.y))]
 
-    def report(self, ms, peaks):
+    def report(self, ms, row_ms, peaks):
         q = ms["qmv"]
         gbs = self.bytes / q / 1e6
         return {"metric": "qmv GB/s", "unit": "GB/s", "value": gbs, "ms": ms,
@@ -222,7 +242,7 @@ class Dequant(Row):
         return [("dequantize", lambda: self.nv.nvfp4_dequantize(self.wc, self.ws, self.g, "linear",
                                                                 torch.bfloat16, out=self.out))]
 
-    def report(self, ms, peaks):
+    def report(self, ms, row_ms, peaks):
         q = ms["dequantize"]
         gbs = self.bytes / q / 1e6
         return {"metric": "nvfp4 dequantize GB/s", "unit": "GB/s", "value": gbs, "ms": ms,
@@ -262,8 +282,8 @@ class Prefill(Row):
                 ("gemm", lambda: nv.qqmm(self.xc, self.xs, self.wc, self.ws, self.K, "nvfp4", self.g_x, self.g_w,
                                          out=self.y))]
 
-    def report(self, ms, peaks):
-        total = sum(ms.values())
+    def report(self, ms, row_ms, peaks):
+        total = row_ms  # the whole op: quantize x and W, GEMM, as one graph
         fp4_peak = peaks["bf16_tflops"] * 4.0  # nominal dense fp4 : bf16 = 9 : 2.25
         tf = self.flop / ms["gemm"] / 1e9
         return {"metric": "qqmm FP4 TFLOP/s", "unit": "TFLOP/s", "value": self.flop / total / 1e9, "ms": ms,
@@ -300,7 +320,7 @@ class Moe(Row):
         return [("gather_qmm", lambda: self.nv.gather_qmm(self.x, self.wc, self.ws, self.g, self.idx,
                                                           self.ws_buf, self.y))]
 
-    def report(self, ms, peaks):
+    def report(self, ms, row_ms, peaks):
         t = ms["gather_qmm"]
         tf = self.flop / t / 1e9
         return {"metric": "gather_qmm TFLOP/s", "unit": "TFLOP/s", "value": tf, "ms": ms,
@@ -334,10 +354,10 @@ class Mxfp8(Row):
                 ("quantize_w", lambda: nv.mxfp8_quantize(self.w, "swizzled", self.wc, self.ws)),
                 ("gemm", lambda: nv.qqmm(self.xc, self.xs, self.wc, self.ws, self.K, "mxfp8", out=self.y))]
 
-    def report(self, ms, peaks):
+    def report(self, ms, row_ms, peaks):
         fp8_peak = peaks["bf16_tflops"] * 2.0
         tf = self.flop / ms["gemm"] / 1e9
-        return {"metric": "mxfp8 qqmm TFLOP/s", "unit": "TFLOP/s", "value": self.flop / sum(ms.values()) / 1e9,
+        return {"metric": "mxfp8 qqmm TFLOP/s", "unit": "TFLOP/s", "value": self.flop / row_ms / 1e9,
                 "ms": ms, "roofline": {"bound": "tensor", "kernel": "qqmm_sm100 (mxfp8)", "achieved": tf,
                                        "peak": fp8_peak, "unit": "TFLOP/s", "frac": tf / fp8_peak,
                                        "peak_note": "measured bf16 burst x 2 (nominal fp8:bf16 ratio)"}}
@@ -480,6 +500,12 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     peaks = load_peaks()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_sum = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        flush.fill_(1.0)                       # write a buffer larger than L2
+        torch.sum(flush_rd, dim=0, out=flush_sum)  # read one: L2 holds clean lines only
     rows, unavailable = [], {}
     for cls in ROWS:
         if args.rows and cls.name not in args.rows:
@@ -500,18 +526,16 @@ def run_ours(args):
             r.run()
     torch.cuda.synchronize()
     for r in rows:
-        r.capture()
+        r.capture(args.steps)
     torch.cuda.synchronize()
 
-    def step():
+    def step(k, timed):
         for r in rows:
-            flush.fill_(1.0)  # L2 flush, outside the rows' timed windows
-            r.replay_timed()
+            flush_l2()  # outside the rows' timed windows
+            r.replay(k, timed)
 
-    for _ in range(args.warmup):
-        step()
-    for r in rows:
-        r.timers = []
+    for k in range(args.warmup):
+        step(k, False)
     torch.cuda.synchronize()
     barrier(world)
     clk = ClockSampler(local)
@@ -521,8 +545,8 @@ def run_ours(args):
     s_all, e_all = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.nvtx.range_push("timed")
     s_all.record()
-    for _ in range(args.steps):
-        step()
+    for k in range(args.steps):
+        step(k, True)
     e_all.record()
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
@@ -531,11 +555,11 @@ def run_ours(args):
     ms_step = max_over_ranks(world, s_all.elapsed_time(e_all) / args.steps)
     reports = {}
     for r in rows:
-        per = {}
-        for label, s, e in r.timers:
-            per[label] = per.get(label, 0.0) + s.elapsed_time(e)
-        per = {k: max_over_ranks(world, v / args.steps) for k, v in per.items()}
-        reports[r.name] = r.report(per, peaks)
+        per, row_ms = r.times()
+        per = {k: max_over_ranks(world, v) for k, v in per.items()}
+        row_ms = max_over_ranks(world, row_ms)
+        reports[r.name] = r.report(per, row_ms, peaks)
+        reports[r.name]["row_ms"] = row_ms
     head_row = "prefill" if "prefill" in reports else ("gemv" if "gemv" in reports else rows[0].name)
     head = reports[head_row]
     e2e = None
@@ -566,8 +590,9 @@ def run_ours(args):
                 "prefill": "nvfp4 qqmm op, x [4096,4096] bf16 N(0,1), W [4096,4096] bf16 N(0,0.02) with 1% x50 "
                            "outliers, g = amax, SWIZZLED scales, y bf16",
                 "gemv": "nvfp4 qmv, x [1,4096] bf16, W [14336,4096] pre-quantized"}.get(head_row, head_row),
-                "rows_per_step": [r.name for r in rows], "l2": "flushed (256 MiB write) before every row",
-                "timing": "each ABI call replayed as a CUDA graph; events on the launching stream",
+                "rows_per_step": [r.name for r in rows], "l2": "flushed before every row: 256 MiB write, then 256 MiB read",
+                "timing": "each row's ABI calls replayed as one CUDA graph per step; device time from events "
+                          "recorded inside the graph before and after every call",
                 "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
             "roofline": roof,
             "cpu_baseline": cpu,
