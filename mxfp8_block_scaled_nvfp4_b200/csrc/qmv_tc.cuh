@@ -23,18 +23,20 @@
 //
 // CTA = 128 weight rows; warps: 0 TMA producer (codes [128 x 128 B] and
 // LINEAR scales [128 x 16 B] per stage), 1 TMEM allocator + MMA issuer,
-// 2 scale re-layout (LINEAR [128 rows x 16 B] -> four 128x4 tiles for
-// tcgen05.cp), 4-7 epilogue (TMEM lane quarters).  All warps compute the
-// x_hat planes first, while the producer's first loads are in flight.
+// 4-7 epilogue (TMEM lane quarters), 8-11 scale re-layout (LINEAR [128 rows
+// x 16 B] -> four 128x4 tiles for tcgen05.cp; stage kb on warp 8 + kb % 4).
+// Warps 1-11 compute the x_hat planes first, while warp 0 starts the
+// weight stream.
 // TMEM: a 256-column ring of MMA outputs drained in 128-column halves, the
 // weight scale tiles of every stage, one column of unit x-side scales.
 //
 // Every mbarrier wait of the MMA thread costs about as much as several of
 // these small MMAs (its shared-memory access queues behind the tensor
 // core's operand reads), so the MMA thread waits once per group of stages:
-// the re-layout warp handles stages in order, so the barrier of a group's
-// last stage covers the whole group; ring halves that were never used are
-// not waited on.
+// the re-layout warps arrive on one barrier per group of stages (two such
+// barriers alternate; the ring holds two groups, so a group barrier is not
+// reused before the MMA warp has passed its previous phase); ring halves
+// that were never used are not waited on.
 #pragma once
 
 #include <cuda.h>
@@ -46,7 +48,9 @@
 namespace nvfp4 {
 namespace qtc {
 
-constexpr int THREADS = 256;
+constexpr int THREADS = 384;
+constexpr int RELAYOUT_WARPS = 4;     // warps 8-11
+constexpr int FIRST_RELAYOUT_WARP = 8;
 constexpr int BM = 128;            // weight rows per CTA
 constexpr int MAX_STAGES = 8;
 constexpr int A_STAGE = BM * 128;  // 16 KiB of codes (256 K)
@@ -113,10 +117,12 @@ template <> struct Range<__nv_bfloat16> {
 // plane scales (layout in the header comment).  One lane per half-block;
 // returns false on a thread that met a block outside the exact range.
 // x values of this thread's first half-block, loaded at kernel start.
+// Threads 32.. (warps 1 and up) take part; warp 0 streams the weight.
 template <typename T>
 __device__ __forceinline__ void x_first(const T* __restrict__ x, uint32_t M, uint32_t K, float (&v)[8]) {
-  if (threadIdx.x < M * K / 8u) {
-    load8<T>(x + (size_t)threadIdx.x * 8, v);
+  const uint32_t t = threadIdx.x - 32u;
+  if (threadIdx.x >= 32u && t < M * K / 8u) {
+    load8<T>(x + (size_t)t * 8, v);
   } else {
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = 0.0f;
@@ -131,11 +137,12 @@ __device__ __forceinline__ bool x_planes(const T* __restrict__ x, float gx, uint
   const uint32_t n_half = M * K / 8u;  // a multiple of 32: whole warps take part in the pair shuffle
   const uint32_t nb = K / 16u;
   bool exact = true;
-  for (uint32_t hb = threadIdx.x; hb < n_half; hb += blockDim.x) {
+  const uint32_t nthr = blockDim.x - 32u;  // warps 1 and up (a multiple of 32)
+  for (uint32_t hb = threadIdx.x - 32u; threadIdx.x >= 32u && hb < n_half; hb += nthr) {
     float v[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = cur[j];
-    const uint32_t hn = hb + blockDim.x;  // next half-block's loads in flight during this one
+    const uint32_t hn = hb + nthr;  // next half-block's loads in flight during this one
     if (hn < n_half) load8<T>(x + (size_t)hn * 8, cur);
     float a = 0.0f;
 #pragma unroll
@@ -182,7 +189,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[MAX_STAGES];
-  __shared__ __align__(8) uint64_t sf_bar[MAX_STAGES];
+  __shared__ __align__(8) uint64_t sf_grp[2];  // scale tiles of a group of stages ready
   __shared__ __align__(8) uint64_t empty_bar[MAX_STAGES];
   __shared__ __align__(8) uint64_t dfull_bar[2];
   __shared__ __align__(8) uint64_t dempty_bar[2];
@@ -206,18 +213,28 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
   const uint32_t steps_per_half = 128u / ncols;
   const uint32_t nb = a.K / 16u;
 
+  const uint32_t G = S / 2;  // stages per group (S is even)
+  uint32_t issued = 0;       // weight stages issued (thread 0)
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < S; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
-      mbar_init(smem_u32(&sf_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
+    mbar_init(smem_u32(&sf_grp[0]), G);
+    mbar_init(smem_u32(&sf_grp[1]), G);
     for (int h = 0; h < 2; ++h) {
       mbar_init(smem_u32(&dfull_bar[h]), 1);
       mbar_init(smem_u32(&dempty_bar[h]), 4);
     }
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    // the weight stream starts before TMEM allocation and the prologue
+    for (; issued < S && issued < kb_count; ++issued) {
+      const uint32_t bar = smem_u32(&full_bar[issued]);
+      mbar_expect_tx(bar, A_STAGE + S_STAGE);
+      tma_load_2d(sbase + L.ring + issued * STAGE_BYTES, &tmap_w, (int)(issued * 128u), (int)row0, bar);
+      tma_load_2d(sbase + L.ring + issued * STAGE_BYTES + A_STAGE, &tmap_s, (int)(issued * 16u), (int)row0, bar);
+    }
   }
   // zero the plane tiles (a plane row is nonzero only inside its own
   // 16-block: the prologue writes those bytes alone), fill the unit scale tile
@@ -240,16 +257,6 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
 
-  // the producer starts streaming the weight before the prologue runs
-  uint32_t issued = 0;
-  if (threadIdx.x == 0) {
-    for (; issued < S && issued < kb_count; ++issued) {
-      const uint32_t bar = smem_u32(&full_bar[issued]);
-      mbar_expect_tx(bar, A_STAGE + S_STAGE);
-      tma_load_2d(sbase + L.ring + issued * STAGE_BYTES, &tmap_w, (int)(issued * 128u), (int)row0, bar);
-      tma_load_2d(sbase + L.ring + issued * STAGE_BYTES + A_STAGE, &tmap_s, (int)(issued * 16u), (int)row0, bar);
-    }
-  }
   const bool mine = x_planes<T>(static_cast<const T*>(a.x), gx, a.M, a.K, xv, smem + L.planes,
                                 reinterpret_cast<float*>(smem + L.uplane));
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // planes are read by the tensor core
@@ -285,11 +292,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
       const uint32_t first = issued > S ? issued - S : 0;
       for (uint32_t i = first; i < issued; ++i) mbar_wait(smem_u32(&full_bar[i % S]), (i / S) & 1u);
     }
-  } else if (warp == 2) {
+  } else if (warp >= FIRST_RELAYOUT_WARP && warp < FIRST_RELAYOUT_WARP + RELAYOUT_WARPS) {
     // ------------------------------------------------------------ scale re-layout
     // tile j (k-step j of the stage), row r: the 4 block scales of weight
     // rows r, r+32, r+64, r+96 (the 128x4 tile order tcgen05.cp expects)
-    for (uint32_t kb = 0; kb < kb_count; ++kb) {
+    for (uint32_t kb = (uint32_t)(warp - FIRST_RELAYOUT_WARP); kb < kb_count; kb += RELAYOUT_WARPS) {
       const uint32_t s = kb % S;
       if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full_bar[s]), (kb / S) & 1u)) ||
           *(volatile int*)&abort_flag) {
@@ -308,7 +315,14 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
       *reinterpret_cast<uint4*>(tiles + 3 * 512 + 16u * lane) = make_uint4(q0.w, q1.w, q2.w, q3.w);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
-      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sf_bar[s])) : "memory");
+      if (lane == 0) {
+        // the last stage of a short final group also arrives for the stages it lacks
+        const uint32_t grp = kb / G;
+        const uint32_t in_grp = min(G, kb_count - grp * G);
+        const uint32_t cnt = (kb == grp * G + in_grp - 1) ? 1u + (G - in_grp) : 1u;
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&sf_grp[grp & 1u])), "r"(cnt)
+                     : "memory");
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -323,12 +337,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
     const uint64_t t_base = sf_tile_desc(sbase + L.ring + A_STAGE + S_STAGE);
     const uint32_t a_hi = (uint32_t)(a_base >> 32), b_hi = (uint32_t)(b_base >> 32), t_hi = (uint32_t)(t_base >> 32);
     auto mk = [](uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; };
-    const uint32_t G = S >= 2 ? S / 2 : 1;  // stages per wait
     uint32_t g = 0;  // global k-step
     bool ok = true;
     for (uint32_t kb0 = 0; kb0 < kb_count && ok; kb0 += G) {
-      const uint32_t kb1 = min(kb0 + G, kb_count), last = kb1 - 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sf_bar[last % S]), (last / S) & 1u)) ||
+      const uint32_t kb1 = min(kb0 + G, kb_count), grp = kb0 / G;
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sf_grp[grp & 1u]), (grp >> 1) & 1u)) ||
           *(volatile int*)&abort_flag) {
         ok = false;
         break;
@@ -447,7 +460,7 @@ inline bool make_maps(CUtensorMap* mw, CUtensorMap* ms, const uint32_t* wc, cons
 inline uint32_t pick_stages(int64_t M, int64_t K) {
   if (M < 1 || M > 2 || K % 256 != 0 || K < 256) return 0;
   const uint32_t MM = M == 1 ? 1u : 2u;
-  for (uint32_t st = MAX_STAGES; st >= 3; --st)
+  for (uint32_t st = MAX_STAGES; st >= 2; st -= 2)  // even: two groups of st / 2 stages
     if (smem_needed(st, MM, (uint32_t)K) <= 227u * 1024u) return st;
   return 0;
 }
