@@ -11,6 +11,7 @@ One step = one pass over every row of the hot path, each on its workload
   dequant   a5      NVFP4 dequantize of W [14336,4096] to bf16
   prefill   a1-a4,a8-a9  qqmm op: amax x2, quantize x2 (SWIZZLED), FP4 GEMM 4096^3 -> bf16
   moe       a10     gather_qmm: 64 experts [1408,2048], 4096 tokens, top-8 -> bf16
+  moe_decode f2     gather_qmm decode (gather_qmv): the same experts, 4 tokens, top-8
   mxfp8     a11-a12 mxfp8 quantize x2 + FP8 GEMM 8192^3 -> bf16
 
 The headline ``value`` is the prefill qqmm op in TFLOP/s (2*M*N*K over the
@@ -339,6 +340,48 @@ class Moe(Row):
                              "hbm_frac": self.bytes / t / 1e6 / peaks["hbm_gbs"], "algorithmic_bytes": self.bytes}}
 
 
+class MoeDecode(Row):
+    """Decode-time MoE (the gather_qmv path): the MoE config's 64 experts
+    [1408, 2048], 4 tokens routed top-8 (tokens 0-3 of the MoE routing)."""
+    name, launches = "moe_decode", 2
+
+    def setup(self):
+        d = self.wl.make("moe", device=self.dev)
+        x, w, idx = d["x"], d["w"], d["idx"]
+        E, N, K = w.shape
+        self.E, self.N, self.K = E, N, K
+        self.g = torch.stack([self.nv.amax(w[e]) for e in range(E)]).view(E)
+        wc, ws = [], []
+        for e in range(E):
+            c, s = self.nv.nvfp4_quantize(w[e], self.g[e:e + 1], "linear")
+            wc.append(c)
+            ws.append(s)
+        self.wc, self.ws = torch.stack(wc), torch.stack(ws)
+        del w, wc, ws
+        self.T = 4
+        self.x = x[:self.T].contiguous()
+        self.idx = idx[:self.T].contiguous()
+        self.topk = self.idx.shape[1]
+        self.ws_buf = torch.empty(self.nv.gather_qmm_workspace_size(self.T, self.topk, E), dtype=torch.uint8,
+                                  device=self.dev)
+        self.y = torch.empty(self.T, self.topk, N, dtype=torch.bfloat16, device=self.dev)
+        used = int(torch.unique(self.idx).numel())  # each routed expert's weight is read once
+        self.experts_read = used
+        self.bytes = used * (N * K // 2 + N * K // 16) + self.x.numel() * 2 + self.y.numel() * 2 + self.idx.numel() * 4
+
+    def calls(self):
+        return [("gather_qmm", lambda: self.nv.gather_qmm(self.x, self.wc, self.ws, self.g, self.idx,
+                                                          self.ws_buf, self.y))]
+
+    def report(self, ms, row_ms, peaks):
+        t = ms["gather_qmm"]
+        gbs = self.bytes / t / 1e6
+        return {"metric": "gather_qmm decode GB/s", "unit": "GB/s", "value": gbs, "ms": ms,
+                "experts_read": self.experts_read,
+                "roofline": {"bound": "hbm", "kernel": "k_gather_qmv", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes": self.bytes}}
+
+
 class Mxfp8(Row):
     name, launches = "mxfp8", 3
 
@@ -372,7 +415,7 @@ class Mxfp8(Row):
                                        "peak_note": "measured bf16 burst x 2 (nominal fp8:bf16 ratio)"}}
 
 
-ROWS = [Quant1G, Gemv, Dequant, Prefill, Moe, Mxfp8]
+ROWS = [Quant1G, Gemv, Dequant, Prefill, Moe, MoeDecode, Mxfp8]
 
 
 # ---------------------------------------------------------------------------

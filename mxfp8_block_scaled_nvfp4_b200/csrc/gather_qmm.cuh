@@ -35,6 +35,13 @@
 //                  dequantize kernel does.
 // The contraction is on the bf16 tensor pipe: both operands are bf16, as
 // the method requires of the materialized weight.  Every wait is bounded.
+//
+// Decode (T <= kQmvTokens tokens; the pages' "gather_qmv"): few pairs per
+// expert, so 256-pair MMA tiles would mostly compute padding.  k_gather_qmv
+// instead streams each routed expert's weight rows once per tile of pairs:
+// a warp per weight row, 128-bit coalesced code loads, the same bf16
+// rounding of the dequantized weight as above, fp32 dot products with up to
+// kQmvPairs routed x rows held in shared memory at a time.
 #pragma once
 
 #include <cuda.h>
@@ -42,6 +49,7 @@
 
 #include "common.cuh"
 #include "nvfp4.h"
+#include "qmv.cuh"
 #include "qqmm_sm100.cuh"
 
 namespace nvfp4 {
@@ -548,6 +556,138 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
   }
 }
 
+// ---------------------------------------------------------------------------
+// 3. decode: gather_qmv
+// ---------------------------------------------------------------------------
+constexpr int kQmvTokens = 16;   // T at or below which gather_qmm runs k_gather_qmv
+constexpr int kQmvPairs = 4;     // routed x rows per pass
+constexpr int QV_THREADS = 256;
+constexpr int QV_ROWS = 16;      // weight rows per CTA (2 per warp)
+
+// CTA (row block, tile): weight rows n0..n0+15 of the tile's expert against
+// every pair of the tile, kQmvPairs pairs per pass; x of those pairs in
+// shared memory as fp32 [kQmvPairs][K] in qmv's swizzled 32-element chunks
+// (xs_index): lane l reads chunk l, and the swizzle puts the 8 lanes of a
+// 128-bit load phase on distinct banks.
+__global__ void __launch_bounds__(QV_THREADS) k_gather_qmv(const __nv_bfloat16* __restrict__ x,
+                                                           const uint32_t* __restrict__ wc, Args a) {
+  extern __shared__ float xs[];  // [kQmvPairs][K]
+  const int tile = blockIdx.y;
+  if (tile >= *a.ws.ntiles) return;  // uniform per CTA
+  const int e = a.ws.tile_expert[tile], row0 = a.ws.tile_row0[tile], nrows = a.ws.tile_rows[tile];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K = a.K, N = a.N;
+  const uint32_t chunks = (uint32_t)K / 32u;  // 32 codes (16 bytes) per lane and chunk
+  const float d = a.g ? __ldg(a.g + e) / kGlobalEncode : 1.0f;
+  // units (row, chunk group): a lane loads chunks g*128 + 32i + lane (i < 4)
+  // of a weight row; the next unit's loads are in flight while this one
+  // computes, and a pass's first loads are issued before x is staged
+  const uint32_t groups = (chunks + 127u) / 128u;
+  const int nr = min(QV_ROWS, N - (int)blockIdx.x * QV_ROWS);
+  uint4 qb[4];
+  uint32_t sb[4];
+  auto load_unit = [&](int r, uint32_t g) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t c = g * 128u + (uint32_t)i * 32u + (uint32_t)lane;
+      if (r < nr && c < chunks) {
+        const size_t wrow = (size_t)e * N + blockIdx.x * QV_ROWS + r;
+        qb[i] = __ldg(reinterpret_cast<const uint4*>(wc + wrow * (size_t)(K / 8)) + c);
+        sb[i] = __ldg(reinterpret_cast<const unsigned short*>(a.wsc + wrow * (size_t)(K / 16)) + c);
+      } else {
+        qb[i] = make_uint4(0, 0, 0, 0);
+        sb[i] = 0;
+      }
+    }
+  };
+  for (int q0 = 0; q0 < nrows; q0 += kQmvPairs) {
+    const int nq = min(kQmvPairs, nrows - q0);
+    int ur = warp;
+    uint32_t ug = 0;
+    load_unit(ur, ug);
+    __syncthreads();  // the previous pass is done with xs
+    for (int q = 0; q < nq; ++q) {
+      const int tok = a.ws.perm[row0 + q0 + q] / a.topk;
+      const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tok * K);
+      for (int i = threadIdx.x; i < K / 8; i += blockDim.x) {
+        float v[8];
+        load8<__nv_bfloat16>(reinterpret_cast<const __nv_bfloat16*>(src + i), v);
+        *reinterpret_cast<float4*>(xs + xs_index((uint32_t)q, (uint32_t)K, (uint32_t)(i * 8))) =
+            make_float4(v[0], v[1], v[2], v[3]);
+        *reinterpret_cast<float4*>(xs + xs_index((uint32_t)q, (uint32_t)K, (uint32_t)(i * 8 + 4))) =
+            make_float4(v[4], v[5], v[6], v[7]);
+      }
+    }
+    __syncthreads();
+    float acc[kQmvPairs];
+#pragma unroll
+    for (int q = 0; q < kQmvPairs; ++q) acc[q] = 0.0f;
+    while (ur < nr) {
+      uint4 qc[4];
+      uint32_t sc4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        qc[i] = qb[i];
+        sc4[i] = sb[i];
+      }
+      const int cr = ur;
+      const uint32_t cg = ug;
+      if (++ug == groups) {
+        ug = 0;
+        ur += QV_THREADS / 32;
+      }
+      load_unit(ur, ug);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t c = cg * 128u + (uint32_t)i * 32u + (uint32_t)lane;
+        if (c < chunks) {
+          const uint32_t words[4] = {qc[i].x, qc[i].y, qc[i].z, qc[i].w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {  // 8 weights per word, block h / 2 of the chunk
+            const uint4 wb = dequant8_bf16(words[h], e4m3_to_f32((sc4[i] >> (8 * (h >> 1))) & 0xFFu) * d);
+            const uint32_t pw[4] = {wb.x, wb.y, wb.z, wb.w};
+            float wv[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              wv[2 * j] = __uint_as_float(pw[j] << 16);
+              wv[2 * j + 1] = __uint_as_float(pw[j] & 0xFFFF0000u);
+            }
+            const uint32_t k0 = c * 32u + (uint32_t)h * 8u;
+#pragma unroll
+            for (int q = 0; q < kQmvPairs; ++q) {
+              if (q < nq) {
+                const float4 xa = *reinterpret_cast<const float4*>(xs + xs_index((uint32_t)q, (uint32_t)K, k0));
+                const float4 xb = *reinterpret_cast<const float4*>(xs + xs_index((uint32_t)q, (uint32_t)K, k0 + 4u));
+                float t = acc[q];
+                t = fmaf(wv[0], xa.x, t);
+                t = fmaf(wv[1], xa.y, t);
+                t = fmaf(wv[2], xa.z, t);
+                t = fmaf(wv[3], xa.w, t);
+                t = fmaf(wv[4], xb.x, t);
+                t = fmaf(wv[5], xb.y, t);
+                t = fmaf(wv[6], xb.z, t);
+                t = fmaf(wv[7], xb.w, t);
+                acc[q] = t;
+              }
+            }
+          }
+        }
+      }
+      if (cg + 1 == groups) {  // row finished: reduce across the warp and store
+        const int n = (int)blockIdx.x * QV_ROWS + cr;
+#pragma unroll
+        for (int q = 0; q < kQmvPairs; ++q) {
+          float t = acc[q];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+          if (lane == 0 && q < nq) a.y[(size_t)a.ws.perm[row0 + q0 + q] * N + n] = __float2bfloat16_rn(t);
+          acc[q] = 0.0f;
+        }
+      }
+    }
+  }
+}
+
 // x [T, K] bf16: box 64 x 1 rows (tile::gather4 takes four rows of it),
 // 128-byte swizzle.  Codes [E*N rows, K/2 bytes]: box 32 B x 256 rows.
 inline bool make_maps(CUtensorMap* mx, CUtensorMap* mw, const void* x, const uint32_t* wc, uint64_t T, uint64_t K,
@@ -602,6 +742,32 @@ inline nvfp4_status gather_qmm_launch(const void* x, const uint32_t* w_codes, co
   if (err == cudaSuccess) {
     k_route<<<1, ROUTE_THREADS, rsmem, stream>>>(idx, (int)P, (int)E, (int)N, ws, static_cast<__nv_bfloat16*>(y));
     err = cudaGetLastError();
+  }
+  const size_t qv_smem = (size_t)kQmvPairs * (size_t)K * sizeof(float);
+  if (err == cudaSuccess && T <= kQmvTokens && qv_smem <= 200u * 1024u) {
+    // decode: gather_qmv
+    err = cudaFuncSetAttribute(k_gather_qmv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qv_smem);
+    if (err == cudaSuccess) {
+      Args a;
+      a.wsc = w_scales;
+      a.g = g;
+      a.y = static_cast<__nv_bfloat16*>(y);
+      a.ws = ws;
+      a.N = (int)N;
+      a.K = (int)K;
+      a.topk = (int)topk;
+      a.n_tiles_n = 0;
+      const int64_t mt = max_tiles(P, E);
+      dim3 grid((unsigned)((N + QV_ROWS - 1) / QV_ROWS), (unsigned)(P < mt ? P : mt));  // every tile holds >= 1 pair
+      k_gather_qmv<<<grid, QV_THREADS, qv_smem, stream>>>(static_cast<const __nv_bfloat16*>(x), w_codes, a);
+      err = cudaGetLastError();
+    }
+    if (err != cudaSuccess) {
+      snprintf(msg, msg_len, "[gather_qmm] launch failed: %s", cudaGetErrorString(err));
+      return NVFP4_ERR_CUDA;
+    }
+    msg[0] = '\0';
+    return NVFP4_OK;
   }
   if (err == cudaSuccess) err = cudaFuncSetAttribute(k_gather_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
   if (err == cudaSuccess) {

@@ -121,3 +121,43 @@ def test_moe_config_sampled_tokens(nv, orc):
     oc, os_, gs = oracle_operands(orc, w, g)
     r = orc.gather_qmm(raw(x), oc, os_, gs, idx.numpy(), tokens=tokens)
     check_gemm_output(raw(y)[tokens], r, "bf16", orc)
+
+
+# Decode: T <= 16 tokens take the gather_qmv kernel (a warp per expert weight
+# row, the same bf16 rounding of the dequantized weight); same oracle.
+@pytest.mark.parametrize("T,topk,E,N,K", [(1, 8, 64, 192, 256), (2, 4, 8, 272, 512), (4, 8, 16, 128, 2048),
+                                          (16, 2, 5, 64, 128), (3, 3, 7, 1408, 192)])
+@pytest.mark.parametrize("use_g", [True, False])
+def test_gather_qmv_decode_parity(nv, orc, T, topk, E, N, K, use_g):
+    x, w, idx, g, wc, ws = make_case(nv, T, topk, E, N, K, use_g, seed=3 * T + E + N)
+    y = nv.gather_qmm(x.cuda(), wc, ws, g, idx.cuda())
+    nv.check_device_errors()
+    oc, os_, gs = oracle_operands(orc, w, g)
+    r = orc.gather_qmm(raw(x), oc, os_, gs, idx.numpy())
+    check_gemm_output(raw(y), r, "bf16", orc)
+
+
+def test_gather_qmv_decode_full_size_experts(nv, orc):
+    """64 experts W_e [1408, 2048] N(0,0.02), g_e = amax(W_e), 4 tokens, top-8:
+    every output element compared."""
+    x, w, idx, g, wc, ws = make_case(nv, 4, 8, 64, 1408, 2048, True, seed=41)
+    y = nv.gather_qmm(x.cuda(), wc, ws, g, idx.cuda())
+    nv.check_device_errors()
+    oc, os_, gs = oracle_operands(orc, w, g)
+    r = orc.gather_qmm(raw(x), oc, os_, gs, idx.numpy())
+    check_gemm_output(raw(y), r, "bf16", orc)
+
+
+def test_gather_qmv_repeated_expert_and_boundary(nv, orc):
+    """A token routed twice to the same expert (more pairs per expert than
+    tokens), and T = 16 (decode kernel) vs T = 17 (MMA kernel) on the same
+    weights: both match the oracle."""
+    E, N, K, topk = 6, 96, 256, 3
+    idx = torch.tensor([[2, 2, 5]] + [[i % E, (i + 1) % E, 2] for i in range(16)], dtype=torch.int32)
+    x, w, _, g, wc, ws = make_case(nv, 17, topk, E, N, K, True, seed=77, idx=idx)
+    oc, os_, gs = oracle_operands(orc, w, g)
+    for T in (16, 17):
+        y = nv.gather_qmm(x[:T].cuda(), wc, ws, g, idx[:T].cuda())
+        nv.check_device_errors()
+        r = orc.gather_qmm(raw(x[:T]), oc, os_, gs, idx[:T].numpy())
+        check_gemm_output(raw(y), r, "bf16", orc)
