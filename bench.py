@@ -10,6 +10,8 @@ One step = one pass over every row of the hot path, each on its workload
   gemv      a1,a6-a7  amax(x) + qmv: x [1,4096] bf16, W [14336,4096] pre-quantized
   dequant   a5      NVFP4 dequantize of W [14336,4096] to bf16
   prefill   a1-a4,a8-a9  qqmm op: amax x2, quantize x2 (SWIZZLED), FP4 GEMM 4096^3 -> bf16
+  prefill_bwd f1    qqmm backward: amax + quantize of the gradient, column-wise
+                    quantizes of W, x and the gradient, dx and dw GEMMs 4096^3
   moe       a10     gather_qmm: 64 experts [1408,2048], 4096 tokens, top-8 -> bf16
   moe_decode f2     gather_qmm decode (gather_qmv): the same experts, 4 tokens, top-8
   mxfp8     a11-a12 mxfp8 quantize x2 + FP8 GEMM 8192^3 -> bf16
@@ -302,6 +304,51 @@ class Prefill(Row):
                              "peak_note": "measured bf16 burst x 4 (nominal fp4:bf16 ratio)"}}
 
 
+class PrefillBwd(Row):
+    """Backward pass of the prefill qqmm (QQMatmul::vjp, NVFP4 with global
+    scales): amax of the upstream gradient, its row-wise and column-wise
+    quantization, column-wise quantization of W and x, and the dx and dw
+    GEMMs (4096^3 each)."""
+    name, launches = "prefill_bwd", 7
+
+    def setup(self):
+        d = self.wl.make("prefill_bwd", device=self.dev)
+        self.x, self.w, self.c = d["x"], d["w"], d["cotan"]
+        M, K = self.x.shape
+        N = self.w.shape[0]
+        self.M, self.N, self.K = M, N, K
+        nv, dev = self.nv, self.dev
+        self.g_x, self.g_w = nv.amax(self.x), nv.amax(self.w)
+        self.g_c = torch.empty(1, dtype=torch.float32, device=dev)
+        q = lambda r, k: (torch.empty(r, k // 8, dtype=torch.int32, device=dev),
+                          torch.empty(nv.scale_shape(r, k // 16, "swizzled"), dtype=torch.uint8, device=dev))
+        self.cq, self.wtq, self.ctq, self.xtq = q(M, N), q(K, N), q(N, M), q(K, M)
+        self.dx = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        self.dw = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+        self.flop = 2 * (2 * M * N * K)
+
+    def calls(self):
+        nv = self.nv
+        return [("amax_cotan", lambda: nv.amax(self.c, self.g_c)),
+                ("quantize_cotan", lambda: nv.nvfp4_quantize(self.c, self.g_c, "swizzled", *self.cq)),
+                ("quantize_wT", lambda: nv.nvfp4_quantize_columnwise(self.w, self.g_w, "swizzled", *self.wtq)),
+                ("gemm_dx", lambda: nv.qqmm(*self.cq, *self.wtq, self.N, "nvfp4", self.g_c, self.g_w, out=self.dx)),
+                ("quantize_cotanT", lambda: nv.nvfp4_quantize_columnwise(self.c, self.g_c, "swizzled", *self.ctq)),
+                ("quantize_xT", lambda: nv.nvfp4_quantize_columnwise(self.x, self.g_x, "swizzled", *self.xtq)),
+                ("gemm_dw", lambda: nv.qqmm(*self.ctq, *self.xtq, self.M, "nvfp4", self.g_c, self.g_x, out=self.dw))]
+
+    def report(self, ms, row_ms, peaks):
+        fp4_peak = peaks["bf16_tflops"] * 4.0
+        col_bytes = 2 * self.M * self.K + self.M * self.K // 2 + self.M * self.K // 16  # one 4096^2 bf16 operand
+        return {"metric": "qqmm backward FP4 TFLOP/s", "unit": "TFLOP/s", "value": self.flop / row_ms / 1e9, "ms": ms,
+                "columnwise_quantize_gbs": col_bytes / ms["quantize_xT"] / 1e6,
+                "roofline": {"bound": "tensor", "kernel": "qqmm_sm100 (nvfp4)",
+                             "achieved": (self.flop / 2) / ms["gemm_dx"] / 1e9, "peak": fp4_peak, "unit": "TFLOP/s",
+                             "frac": (self.flop / 2) / ms["gemm_dx"] / 1e9 / fp4_peak,
+                             "algorithmic_flop": self.flop // 2,
+                             "peak_note": "measured bf16 burst x 4 (nominal fp4:bf16 ratio)"}}
+
+
 class Moe(Row):
     name, launches = "moe", 3
 
@@ -415,7 +462,7 @@ class Mxfp8(Row):
                                        "peak_note": "measured bf16 burst x 2 (nominal fp8:bf16 ratio)"}}
 
 
-ROWS = [Quant1G, Gemv, Dequant, Prefill, Moe, MoeDecode, Mxfp8]
+ROWS = [Quant1G, Gemv, Dequant, Prefill, PrefillBwd, Moe, MoeDecode, Mxfp8]
 
 
 # ---------------------------------------------------------------------------

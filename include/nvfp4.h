@@ -118,6 +118,19 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const uint32_t* codes, const uint8_t* sc
                               nvfp4_layout layout, int64_t rows, int64_t K, const float* g,
                               void* out, nvfp4_dtype out_dt, nvfp4_stream_t stream);
 
+/* f1 -- column-wise NVFP4 quantize ([P2] fp_quantize_columnwise: an M-major
+ * matrix quantized along its last dimension): x [rows, cols] row-major is
+ * quantized as x^T [cols, rows] along rows, block by block exactly as
+ * nvfp4_quantize does (so the result equals nvfp4_quantize of the
+ * transposed, contiguous matrix).  The backward pass of qqmm quantizes w^T,
+ * x^T and the transposed upstream gradient this way ([P1] QQMatmul::vjp).
+ * rows % 16 == 0; codes [cols, rows/8] uint32; scales for [cols, rows/16]
+ * in `layout` (SWIZZLED: [ceil128(cols), ceil4(rows/16)], zero padding);
+ * g as in nvfp4_quantize. */
+NVFP4_API nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, int64_t rows, int64_t cols,
+                                                 const float* g, uint32_t* codes, uint8_t* scales,
+                                                 nvfp4_layout layout, nvfp4_stream_t stream);
+
 /* a11 -- MXFP8 quantize ([P2] fp_quantize_rowwise with 8 bits and the e8m0
  * scale; group size 32, [P1] fp_quantize; the E8M0 scale is rounded up, [P3]
  * mlxcel note).  Per 32-block: s = ue8m0_round_up(amax / 448);

@@ -214,6 +214,40 @@ nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t
   return quantize_common("quantize", false, x, dt, rows, K, g, codes, scales, layout, stream);
 }
 
+nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, int64_t rows, int64_t cols, const float* g,
+                                       uint32_t* codes, uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
+  const char* tag = "quantize_columnwise";
+  if (!valid_dt(dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] dtype must be float32, float16 or bfloat16", tag);
+  if (layout != NVFP4_LAYOUT_LINEAR && layout != NVFP4_LAYOUT_SWIZZLED)
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] unknown scale layout", tag);
+  if (rows < 0 || cols < 0 || rows * cols > kMaxElems || rows > (1 << 30) || cols > (1 << 30))
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] bad shape [%lld, %lld]", tag, (long long)rows, (long long)cols);
+  if (rows % 16 != 0)
+    return fail(NVFP4_ERR_INVALID_ARG,
+                "[%s] The quantized dimension (rows of x, the last dimension of x^T) needs to be divisible by the "
+                "quantization group size 16. However the provided matrix has shape [%lld, %lld]",
+                tag, (long long)rows, (long long)cols);
+  if (rows * cols > 0 && (!x || !codes || !scales)) return fail(NVFP4_ERR_INVALID_ARG, "[%s] null pointer", tag);
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(g) & 3u))
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] tensor pointers must be 16-byte aligned", tag);
+  DeviceInfo d;
+  nvfp4_status st = device_info(tag, &d);
+  if (st != NVFP4_OK) return st;
+  if (rows * cols == 0) return ok();
+  ScaleOut so;
+  so.p = scales;
+  so.blocks_per_row = (uint32_t)(rows / 16);
+  so.Cp = (uint32_t)((rows / 16 + 3) / 4 * 4);
+  so.swizzled = layout == NVFP4_LAYOUT_SWIZZLED;
+  dim3 grid((unsigned)((rows + kColR - 1) / kColR), (unsigned)((cols + kColC - 1) / kColC));
+  dispatch_dt(dt, [&](auto tag_t) {
+    using T = decltype(tag_t);
+    k_nvfp4_quantize_columnwise<T><<<grid, kColThreads, 0, stream>>>(static_cast<const T*>(x), (uint32_t)rows,
+                                                                      (uint32_t)cols, g, codes, so);
+  });
+  return check_launch(tag);
+}
+
 nvfp4_status mxfp8_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K, uint32_t* codes,
                             uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
   return quantize_common("mxfp8_quantize", true, x, dt, rows, K, nullptr, codes, scales, layout, stream);

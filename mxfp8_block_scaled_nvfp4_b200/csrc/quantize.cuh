@@ -147,6 +147,88 @@ __global__ void __launch_bounds__(kEwThreads) k_nvfp4_quantize(
 }
 
 // ---------------------------------------------------------------------------
+// f1: column-wise NVFP4 quantize ("mlx 0.30.7.2 -> 0.30.7.6" diff, page 7,
+// fp_quantize.cu, fp_quantize_columnwise: an M-major [M, K] input quantized
+// along K): x [R, C] row-major is quantized as x^T [C, R] along R, with the
+// same per-block arithmetic as k_nvfp4_quantize.  Codes [C, R/8], scales
+// [C, R/16] (LINEAR or 128x4 tiles).  This is what the backward pass of the
+// dense matmul needs for w^T and x^T and for the transposed upstream
+// gradient.
+//
+// CTA tile: 128 rows x 64 columns of x, staged in shared memory as fp32
+// [64 columns][128 rows + 1] (the padding keeps both the transposing writes
+// and the per-column reads on distinct banks); a thread quantizes one
+// 16-row block of one column; codes go through shared memory so each
+// column's 64 bytes of codes are stored contiguously.
+// ---------------------------------------------------------------------------
+constexpr int kColR = 128, kColC = 64, kColThreads = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kColThreads) k_nvfp4_quantize_columnwise(
+    const T* __restrict__ x, uint32_t R, uint32_t C, const float* __restrict__ g, uint32_t* __restrict__ codes,
+    ScaleOut so) {
+  __shared__ float tile[kColC][kColR + 1];
+  __shared__ uint2 qcodes[kColC][kColR / 16];
+  const float E = g ? kGlobalEncode / __ldg(g) : 1.0f;
+  const uint32_t r0 = blockIdx.x * kColR, c0 = blockIdx.y * kColC;
+  // load: a thread takes 8 consecutive columns of a row (one vector load
+  // when they are in range and C % 8 == 0); for a fixed element the 32 lanes
+  // (8 column groups x 4 rows) write 32 distinct banks of the padded tile
+  for (uint32_t i = threadIdx.x; i < (uint32_t)(kColR * kColC / 8); i += blockDim.x) {
+    const uint32_t rr = i / (kColC / 8), cg = i % (kColC / 8);
+    const uint32_t r = r0 + rr, c = c0 + cg * 8u;
+    float v[8];
+    if (r < R && c + 8u <= C && (C & 7u) == 0) {
+      load8<T>(x + (size_t)r * C + c, v);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = (r < R && c + j < C) ? Elem<T>::to_f(x[(size_t)r * C + c + j]) : 0.0f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) tile[cg * 8u + j][rr] = v[j];
+  }
+  __syncthreads();
+  // quantize: unit (column cc, row block rb), consecutive lanes on consecutive columns
+  for (uint32_t u = threadIdx.x; u < (uint32_t)(kColC * (kColR / 16)); u += blockDim.x) {
+    const uint32_t cc = u % kColC, rb = u / kColC;
+    float v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = tile[cc][rb * 16 + j];
+    float a = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) a = fmaxf(a, fabsf(v[j]));
+    float t = a / kE2M1Max;
+    t = t * E;
+    const uint32_t s = f32_to_e4m3(t);
+    const float fs = e4m3_to_f32(s);
+    uint32_t w0 = 0, w1 = 0;
+    if (fs != 0.0f) {
+      const float k = E / fs;
+      float q0[8], q1[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        q0[j] = v[j] * k;
+        q1[j] = v[8 + j] * k;
+      }
+      w0 = f32x8_to_e2m1x8(q0);
+      w1 = f32x8_to_e2m1x8(q1);
+    }
+    qcodes[cc][rb] = make_uint2(w0, w1);
+    const uint32_t c = c0 + cc, r = r0 + rb * 16;
+    if (c < C && r < R) so.store(c * (R / 16u) + r / 16u, s);
+  }
+  __syncthreads();
+  // store: column cc of the tile is row c of x^T, its 16 blocks 128 contiguous bytes
+  const uint32_t wpr = R / 8u;  // code words per row of x^T
+  for (uint32_t i = threadIdx.x; i < (uint32_t)(kColC * (kColR / 16)); i += blockDim.x) {
+    const uint32_t cc = i / (kColR / 16), rb = i % (kColR / 16);
+    const uint32_t c = c0 + cc, r = r0 + rb * 16;
+    if (c < C && r < R) *reinterpret_cast<uint2*>(codes + (size_t)c * wpr + r / 8u) = qcodes[cc][rb];
+  }
+  zero_scale_padding(so, C);
+}
+
+// ---------------------------------------------------------------------------
 // a11: MXFP8 quantize (fp_quantize_rowwise with bits 8 and the e8m0 scale;
 // the scale is rounded up, as the mlxcel note on the "[Metal] global scale
 // for qmm" page records for CUDA):  per 32-block: v = max|x| / 448;

@@ -33,6 +33,7 @@ SIGNATURES = [
     ("nvfp4_scale_bytes", _SZ, [_I64, _I64, _I]),
     ("nvfp4_amax", _I, [_P, _I, _I64, _P, _P]),
     ("nvfp4_quantize", _I, [_P, _I, _I64, _I64, _P, _P, _P, _I, _P]),
+    ("nvfp4_quantize_columnwise", _I, [_P, _I, _I64, _I64, _P, _P, _P, _I, _P]),
     ("nvfp4_dequantize", _I, [_P, _P, _I, _I64, _I64, _P, _P, _I, _P]),
     ("mxfp8_quantize", _I, [_P, _I, _I64, _I64, _P, _P, _I, _P]),
     ("mxfp8_dequantize", _I, [_P, _P, _I, _I64, _I64, _P, _I, _P]),
@@ -130,6 +131,21 @@ def nvfp4_quantize(x: torch.Tensor, g: torch.Tensor | None = None, layout: str =
     return codes, scales
 
 
+def nvfp4_quantize_columnwise(x: torch.Tensor, g: torch.Tensor | None = None, layout: str = "linear",
+                              codes: torch.Tensor | None = None, scales: torch.Tensor | None = None):
+    """(codes [cols, rows/8], scales) of x^T quantized along the rows of a 2-D x
+    (equal to nvfp4_quantize(x.T.contiguous(), g, layout))."""
+    _need_cuda(x, g)
+    rows, cols = x.shape
+    if codes is None:
+        codes = torch.empty(cols, rows // 8, dtype=torch.int32, device=x.device)
+    if scales is None:
+        scales = torch.empty(scale_shape(cols, rows // 16, layout), dtype=torch.uint8, device=x.device)
+    _check(lib().nvfp4_quantize_columnwise(_ptr(x), DT[x.dtype], rows, cols, _ptr(g), _ptr(codes), _ptr(scales),
+                                           LAYOUT[layout], _stream()))
+    return codes, scales
+
+
 def nvfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, g: torch.Tensor | None = None,
                      layout: str = "linear", dtype=torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
     _need_cuda(codes, scales, g)
@@ -181,6 +197,26 @@ def qqmm(a_codes, a_scales, b_codes, b_scales, K: int, mode: str = "nvfp4", g_x=
     _check(lib().qqmm(MODE[mode], M, N, K, _ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales),
                       _ptr(g_x), _ptr(g_w), _ptr(out), DT[out.dtype], _stream()))
     return out
+
+
+def qqmm_vjp(x: torch.Tensor, w: torch.Tensor, cotan: torch.Tensor, g_x: torch.Tensor, g_w: torch.Tensor):
+    """(dx, dw) of y = qqmm(x, w) ("mlx 0.30.7.2 -> 0.30.7.6" diff, page 8,
+    QQMatmul::vjp, NVFP4 with global scales): with g_c = amax(cotan),
+      dx = qqmm(cotan, w^T)   -- cotan quantized along N with g_c, w^T along N with g_w
+      dw = qqmm(cotan^T, x^T) -- both quantized along M, with g_c and g_x.
+    x [M, K], w [N, K], cotan [M, N] bf16/fp16/fp32; M, N multiples of 32.
+    Every step is one ABI call (amax, quantize, column-wise quantize, qqmm)."""
+    _need_cuda(x, w, cotan, g_x, g_w)
+    M, K = x.shape
+    N = w.shape[0]
+    g_c = amax(cotan)
+    c_codes, c_scales = nvfp4_quantize(cotan, g_c, "swizzled")                # [M, N/8]
+    wt_codes, wt_scales = nvfp4_quantize_columnwise(w, g_w, "swizzled")      # w^T [K, N/8]
+    dx = qqmm(c_codes, c_scales, wt_codes, wt_scales, N, "nvfp4", g_c, g_w, out_dtype=x.dtype)
+    ct_codes, ct_scales = nvfp4_quantize_columnwise(cotan, g_c, "swizzled")  # cotan^T [N, M/8]
+    xt_codes, xt_scales = nvfp4_quantize_columnwise(x, g_x, "swizzled")      # x^T [K, M/8]
+    dw = qqmm(ct_codes, ct_scales, xt_codes, xt_scales, M, "nvfp4", g_c, g_x, out_dtype=w.dtype)
+    return dx, dw
 
 
 def qmv(x: torch.Tensor, w_codes, w_scales, g_x=None, g_w=None, out=None) -> torch.Tensor:

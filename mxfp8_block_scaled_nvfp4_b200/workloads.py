@@ -21,6 +21,8 @@ moe        64 experts W_e [1408,2048] bf16 N(0,0.02); x [4096,2048]    5, 6
            bf16 N(0,1); per token 8 distinct experts (randperm(64))    7
 mxfp8      x, W [8192,8192] bf16 N(0,1)                                8, 9
 quant1g    x [32768,16384] bf16 N(0,1) (1 GiB)                         10
+prefill_bwd  the prefill x and W, upstream gradient [4096,4096] bf16    3, 4, 11
+           N(0,1) (synthetic: no model produces it here)
 =========  ==========================================================  =====
 """
 from __future__ import annotations
@@ -35,6 +37,7 @@ WORKLOADS = {
             "seeds": (5, 6, 7)},
     "mxfp8": {"M": 8192, "N": 8192, "K": 8192, "dtype": torch.bfloat16, "seeds": (8, 9)},
     "quant1g": {"R": 32768, "K": 16384, "dtype": torch.bfloat16, "seeds": (10,)},
+    "prefill_bwd": {"M": 4096, "N": 4096, "K": 4096, "dtype": torch.bfloat16, "seeds": (3, 4, 11)},
 }
 
 
@@ -105,6 +108,11 @@ def make(name: str, device="cpu", scale_down: int = 1) -> dict:
         x = normal((T, K), 1.0, s_x, w["dtype"], device)
         idx = routing(T, E, topk, s_i, device)
         return {"x": x, "w": W, "idx": idx}
+    if name == "prefill_bwd":
+        d = make("prefill", device=device, scale_down=sd)
+        M, N = d["x"].shape[0], d["w"].shape[0]
+        d["cotan"] = normal((M, N), 1.0, w["seeds"][2], w["dtype"], device)
+        return d
     if name == "quant1g":
         R, K = w["R"], w["K"]
         if sd > 1:
