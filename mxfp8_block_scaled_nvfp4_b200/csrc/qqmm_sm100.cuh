@@ -37,6 +37,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cstdio>
+#include <cstring>
 
 #include "common.cuh"
 #include "nvfp4.h"
@@ -58,7 +59,9 @@ constexpr int SMEM_A = 0;
 constexpr int SMEM_B = SMEM_A + STAGES * A_STAGE;
 constexpr int SMEM_SFA = SMEM_B + STAGES * B_STAGE;
 constexpr int SMEM_SFB = SMEM_SFA + STAGES * SFA_STAGE;
-constexpr int SMEM_BYTES = SMEM_SFB + STAGES * SFB_STAGE;
+constexpr int SMEM_EPI = SMEM_SFB + STAGES * SFB_STAGE;
+constexpr int EPI_BUF = 32 * 32;  // per epilogue warp: 32 rows x 32 bytes of output
+constexpr int SMEM_BYTES = SMEM_EPI + EPI_WARPS * EPI_BUF;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_SF = 256;       // scale-factor columns start here
@@ -103,6 +106,20 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
       : "memory");
+}
+
+// Tensor store of a 2-D box from shared memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(src)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
@@ -209,6 +226,7 @@ struct Params {
   uint32_t k_bytes;     // bytes of K per row (K/2 NVFP4, K MXFP8)
   uint32_t sf_groups;   // Cp / 4: scale-tile columns per 128-row block
   uint32_t rows_b_pad;  // ceil128(N)
+  int tma_store;        // 1: y is written through tmap_y (row pitch a multiple of 16 bytes)
 };
 
 template <typename T>
@@ -262,7 +280,8 @@ __device__ __forceinline__ void tile_coords(uint32_t t, uint32_t mt, uint32_t nt
 
 template <bool MX>
 __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUtensorMap tmap_a,
-                                                     const __grid_constant__ CUtensorMap tmap_b, Params p) {
+                                                     const __grid_constant__ CUtensorMap tmap_b,
+                                                     const __grid_constant__ CUtensorMap tmap_y, Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
@@ -454,9 +473,56 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
       tc_fence_before();
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&accum_empty)) : "memory");
-      const int row = (int)(tm * BM) + q * 32 + lane;
+      const int row0 = (int)(tm * BM) + q * 32, row = row0 + lane;
       const int col0 = (int)(tn * BN) + half * 128;
-      if (row < p.M) {
+      if (p.tma_store) {
+        // Stage 32 rows x 32 bytes at a time in this warp's buffer and let
+        // the TMA write the box (whole sectors; rows >= M and columns >= N
+        // of the box are clipped by the tensor map).  Each lane writes its
+        // row's two 16-byte halves in an order that keeps every 8-lane
+        // phase of the shared store free of bank conflicts.
+        const uint32_t buf = sbase + SMEM_EPI + (uint32_t)(warp - 2) * EPI_BUF;
+        const uint32_t rbase = buf + (uint32_t)lane * 32u;
+        const bool swap = (lane >> 2) & 1;
+        auto put = [&](int col, uint4 h0, uint4 h1) {
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          __syncwarp();
+          st_shared_v4(rbase + (swap ? 16u : 0u), swap ? h1 : h0);
+          st_shared_v4(rbase + (swap ? 0u : 16u), swap ? h0 : h1);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) tma_store_2d(&tmap_y, buf, col, row0);
+        };
+        if (row0 < p.M) {
+          if (p.y_dt == NVFP4_DT_F32) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int col = col0 + c * 8;
+              if (col >= p.N) break;
+              const float* o = v + c * 8;
+              put(col,
+                  make_uint4(__float_as_uint(o[0] * alpha), __float_as_uint(o[1] * alpha),
+                             __float_as_uint(o[2] * alpha), __float_as_uint(o[3] * alpha)),
+                  make_uint4(__float_as_uint(o[4] * alpha), __float_as_uint(o[5] * alpha),
+                             __float_as_uint(o[6] * alpha), __float_as_uint(o[7] * alpha)));
+            }
+          } else {
+            const bool bf = p.y_dt == NVFP4_DT_BF16;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int col = col0 + c * 16;
+              if (col >= p.N) break;
+              uint32_t w[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float lo = v[c * 16 + 2 * i] * alpha, hi = v[c * 16 + 2 * i + 1] * alpha;
+                w[i] = bf ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
+              }
+              put(col, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
+            }
+          }
+        }
+      } else if (row < p.M) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int col = col0 + c * 32;
@@ -473,6 +539,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
         }
       }
     }
+    // the tensor stores of this warp are complete before the CTA exits
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
   __syncwarp();  // lanes that skipped a one-lane role loop wait for it before the CTA barrier
   tc_fence_before();
@@ -526,7 +594,27 @@ inline nvfp4_status qqmm_launch(bool mx, int64_t M, int64_t N, int64_t K, const 
     snprintf(msg, msg_len, "[qqmm] cuTensorMapEncodeTiled failed");
     return NVFP4_ERR_CUDA;
   }
+  // Output tensor map: boxes of 32 rows x 32 bytes; usable when the row pitch
+  // is a multiple of 16 bytes (y itself is 16-byte aligned).
+  const uint64_t esz = y_dt == NVFP4_DT_F32 ? 4u : 2u;
+  CUtensorMap ty;
+  memset(&ty, 0, sizeof(ty));
+  bool tma_store = ((uint64_t)N * esz) % 16u == 0;
+  if (tma_store) {
+    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    cuuint64_t strides[1] = {(cuuint64_t)N * esz};
+    cuuint32_t box[2] = {(cuuint32_t)(32u / esz), 32u};
+    cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapDataType dt = y_dt == NVFP4_DT_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : y_dt == NVFP4_DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    auto fn = encode_fn();
+    tma_store = fn && fn(&ty, dt, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
   Params p;
+  p.tma_store = tma_store ? 1 : 0;
   p.sfa = a_scales;
   p.sfb = b_scales;
   p.g_x = g_x;
@@ -546,10 +634,10 @@ inline nvfp4_status qqmm_launch(bool mx, int64_t M, int64_t N, int64_t K, const 
   cudaError_t e;
   if (mx) {
     e = cudaFuncSetAttribute(k_qqmm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-    if (e == cudaSuccess) k_qqmm<true><<<grid, THREADS, SMEM_ALLOC, stream>>>(ta, tb, p);
+    if (e == cudaSuccess) k_qqmm<true><<<grid, THREADS, SMEM_ALLOC, stream>>>(ta, tb, ty, p);
   } else {
     e = cudaFuncSetAttribute(k_qqmm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-    if (e == cudaSuccess) k_qqmm<false><<<grid, THREADS, SMEM_ALLOC, stream>>>(ta, tb, p);
+    if (e == cudaSuccess) k_qqmm<false><<<grid, THREADS, SMEM_ALLOC, stream>>>(ta, tb, ty, p);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
