@@ -12,12 +12,17 @@
 // decoding each block with its global scale.
 //
 // Kernel structure (persistent: one CTA per SM loops over 128 x 256 output
-// tiles; 320 threads):
+// tiles; 352 threads):
 //   warp 0   TMA producer: per K stage, A codes [128 rows x 128 B] and B codes
-//            [256 rows x 128 B] as 128-byte-swizzled tiles, plus the scale
-//            tiles as plain bulk copies (the 128x4 scale-tile layout of the
-//            operands is already the order the MMA's scale tensor memory
-//            expects, so the copies are contiguous 512-byte blocks).
+//            [256 rows x 128 B] as 128-byte-swizzled tiles; it also posts
+//            the stage's expected bytes, scale tiles included.
+//   warp 10  scale producer: the stage's scale tiles as plain bulk copies
+//            (the 128x4 scale-tile layout of the operands is already the
+//            order the MMA's scale tensor memory expects, so the copies are
+//            contiguous 512-byte blocks).  Each TMA issue occupies its thread
+//            for on the order of a hundred cycles; with all five copies of a
+//            stage on one thread the issue loop, not the tensor core, set the
+//            stage rate, so the copies are split over two warps.
 //   warp 1   TMEM allocator and MMA issuer: one elected lane of the
 //            converged warp moves the stage's
 //            scale tiles into tensor memory (tcgen05.cp 32x128b.warpx4) and
@@ -50,7 +55,8 @@ constexpr int BN = 256;
 constexpr int BKB = 128;  // bytes of K per row per stage (256 FP4 / 128 FP8 elements)
 constexpr int STAGES = 4;
 constexpr int EPI_WARPS = 8;
-constexpr int THREADS = 64 + 32 * EPI_WARPS;  // producer, MMA, 8 epilogue warps
+constexpr int W_SCALES = 2 + EPI_WARPS;         // the scale producer warp
+constexpr int THREADS = 96 + 32 * EPI_WARPS;     // producer, MMA, 8 epilogue warps, scale producer
 constexpr int A_STAGE = BM * BKB;    // 16 KiB
 constexpr int B_STAGE = BN * BKB;    // 32 KiB
 constexpr int SFA_STAGE = 4 * 512;   // up to 4 scale tiles (NVFP4)
@@ -266,6 +272,76 @@ __device__ __forceinline__ void store_out<__half>(__half* dst, const float* v, i
   store_out_16<__half>(dst, v, n);
 }
 
+// Epilogue of one warp: its 32 accumulator rows (one per lane, starting at
+// row0) x 128 columns (starting at col0), scaled by alpha and rounded to y's
+// type.  With p.tma_store the warp stages 32 rows x 32 bytes at a time in
+// its 1 KiB shared buffer `buf` and the TMA writes the box (whole sectors;
+// rows >= M and columns >= N of the box are clipped by the tensor map); each
+// lane writes its row's two 16-byte halves in an order that keeps every
+// 8-lane phase of the shared store free of bank conflicts.  Otherwise each
+// lane stores its row directly.
+__device__ __forceinline__ void epilogue_store(const Params& p, const CUtensorMap* tmap_y, uint32_t buf,
+                                               const float (&v)[128], float alpha, int row0, int col0, int lane) {
+  if (row0 >= p.M) return;
+  if (p.tma_store) {
+    const uint32_t rbase = buf + (uint32_t)lane * 32u;
+    const bool swap = (lane >> 2) & 1;
+    auto put = [&](int col, uint4 h0, uint4 h1) {
+      if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      __syncwarp();
+      st_shared_v4(rbase + (swap ? 16u : 0u), swap ? h1 : h0);
+      st_shared_v4(rbase + (swap ? 0u : 16u), swap ? h0 : h1);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) tma_store_2d(tmap_y, buf, col, row0);
+    };
+    if (p.y_dt == NVFP4_DT_F32) {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int col = col0 + c * 8;
+        if (col >= p.N) break;
+        const float* o = v + c * 8;
+        put(col,
+            make_uint4(__float_as_uint(o[0] * alpha), __float_as_uint(o[1] * alpha), __float_as_uint(o[2] * alpha),
+                       __float_as_uint(o[3] * alpha)),
+            make_uint4(__float_as_uint(o[4] * alpha), __float_as_uint(o[5] * alpha), __float_as_uint(o[6] * alpha),
+                       __float_as_uint(o[7] * alpha)));
+      }
+    } else {
+      const bool bf = p.y_dt == NVFP4_DT_BF16;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int col = col0 + c * 16;
+        if (col >= p.N) break;
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float lo = v[c * 16 + 2 * i] * alpha, hi = v[c * 16 + 2 * i + 1] * alpha;
+          w[i] = bf ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
+        }
+        put(col, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
+      }
+    }
+    return;
+  }
+  const int row = row0 + lane;
+  if (row >= p.M) return;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int col = col0 + c * 32;
+    if (col < p.N) {
+      const int n = min(32, p.N - col);
+      float o[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = v[c * 32 + i] * alpha;
+      const size_t off = (size_t)row * p.N + col;
+      if (p.y_dt == NVFP4_DT_F32) store_out<float>(static_cast<float*>(p.y) + off, o, n);
+      else if (p.y_dt == NVFP4_DT_BF16) store_out<__nv_bfloat16>(static_cast<__nv_bfloat16*>(p.y) + off, o, n);
+      else store_out<__half>(static_cast<__half*>(p.y) + off, o, n);
+    }
+  }
+}
+
 // Tile t of the persistent schedule -> (m tile, n tile): groups of 8 M tiles
 // sweep all N tiles, so the CTAs running at the same time share A and B
 // tiles in L2.
@@ -340,14 +416,6 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
           mbar_expect_tx(bar, A_STAGE + B_STAGE + sfa_bytes + sfb_bytes);
           tma_load_2d(sbase + SMEM_A + s * A_STAGE, &tmap_a, (int)(kb * BKB), tile_m, bar);
           tma_load_2d(sbase + SMEM_B + s * B_STAGE, &tmap_b, (int)(kb * BKB), tile_n, bar);
-          if (ntl) {
-            bulk_load(sbase + SMEM_SFA + s * SFA_STAGE, p.sfa + ((size_t)tm * p.sf_groups + g0) * 512u, sfa_bytes, bar);
-            bulk_load(sbase + SMEM_SFB + s * SFB_STAGE, p.sfb + ((size_t)(tile_n / 128) * p.sf_groups + g0) * 512u,
-                      sfa_bytes, bar);
-            if (b_second)
-              bulk_load(sbase + SMEM_SFB + s * SFB_STAGE + 4 * 512,
-                        p.sfb + ((size_t)(tile_n / 128 + 1) * p.sf_groups + g0) * 512u, sfa_bytes, bar);
-          }
         }
       }
       // drain: the last STAGES issued stages must have landed before exit
@@ -448,6 +516,38 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
         __syncwarp();
       }
     }
+  } else if (warp == W_SCALES) {
+    // ------------------------------------------------------------ scale producer
+    // Same stage sequence as warp 0; its copies complete on the stage's full
+    // barrier, whose expected bytes warp 0 has posted (or will post: the
+    // phase cannot complete before warp 0's arrival).
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (uint32_t t = blockIdx.x; t < tiles && !*(volatile int*)&abort_flag; t += gridDim.x) {
+        uint32_t tm, tn;
+        tile_coords(t, mt, nt, tm, tn);
+        const int tile_n = (int)(tn * BN);
+        const bool b_second = (uint32_t)(tile_n + 128) < p.rows_b_pad;
+        for (uint32_t kb = 0; kb < p.kb_count; ++kb, ++it) {
+          const uint32_t s = it % STAGES;
+          if (!mbar_wait(smem_u32(&empty_bar[s]), ((it / STAGES) & 1u) ^ 1u)) {
+            abort_flag = 1;
+            break;
+          }
+          const uint32_t g0 = kb * tiles_per_stage;
+          uint32_t ntl = p.sf_groups > g0 ? p.sf_groups - g0 : 0;
+          if (ntl > tiles_per_stage) ntl = tiles_per_stage;
+          if (ntl == 0) continue;
+          const uint32_t bytes = ntl * 512u, bar = smem_u32(&full_bar[s]);
+          bulk_load(sbase + SMEM_SFA + s * SFA_STAGE, p.sfa + ((size_t)tm * p.sf_groups + g0) * 512u, bytes, bar);
+          bulk_load(sbase + SMEM_SFB + s * SFB_STAGE, p.sfb + ((size_t)(tile_n / 128) * p.sf_groups + g0) * 512u,
+                    bytes, bar);
+          if (b_second)
+            bulk_load(sbase + SMEM_SFB + s * SFB_STAGE + 4 * 512,
+                      p.sfb + ((size_t)(tile_n / 128 + 1) * p.sf_groups + g0) * 512u, bytes, bar);
+        }
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue warps 2..9
     const int q = warp & 3;                // TMEM lane quarter this warp may read
@@ -473,71 +573,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
       tc_fence_before();
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&accum_empty)) : "memory");
-      const int row0 = (int)(tm * BM) + q * 32, row = row0 + lane;
-      const int col0 = (int)(tn * BN) + half * 128;
-      if (p.tma_store) {
-        // Stage 32 rows x 32 bytes at a time in this warp's buffer and let
-        // the TMA write the box (whole sectors; rows >= M and columns >= N
-        // of the box are clipped by the tensor map).  Each lane writes its
-        // row's two 16-byte halves in an order that keeps every 8-lane
-        // phase of the shared store free of bank conflicts.
-        const uint32_t buf = sbase + SMEM_EPI + (uint32_t)(warp - 2) * EPI_BUF;
-        const uint32_t rbase = buf + (uint32_t)lane * 32u;
-        const bool swap = (lane >> 2) & 1;
-        auto put = [&](int col, uint4 h0, uint4 h1) {
-          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-          __syncwarp();
-          st_shared_v4(rbase + (swap ? 16u : 0u), swap ? h1 : h0);
-          st_shared_v4(rbase + (swap ? 0u : 16u), swap ? h0 : h1);
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-          if (lane == 0) tma_store_2d(&tmap_y, buf, col, row0);
-        };
-        if (row0 < p.M) {
-          if (p.y_dt == NVFP4_DT_F32) {
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const int col = col0 + c * 8;
-              if (col >= p.N) break;
-              const float* o = v + c * 8;
-              put(col,
-                  make_uint4(__float_as_uint(o[0] * alpha), __float_as_uint(o[1] * alpha),
-                             __float_as_uint(o[2] * alpha), __float_as_uint(o[3] * alpha)),
-                  make_uint4(__float_as_uint(o[4] * alpha), __float_as_uint(o[5] * alpha),
-                             __float_as_uint(o[6] * alpha), __float_as_uint(o[7] * alpha)));
-            }
-          } else {
-            const bool bf = p.y_dt == NVFP4_DT_BF16;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const int col = col0 + c * 16;
-              if (col >= p.N) break;
-              uint32_t w[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float lo = v[c * 16 + 2 * i] * alpha, hi = v[c * 16 + 2 * i + 1] * alpha;
-                w[i] = bf ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
-              }
-              put(col, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
-            }
-          }
-        }
-      } else if (row < p.M) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int col = col0 + c * 32;
-          if (col < p.N) {
-            const int n = min(32, p.N - col);
-            float o[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = v[c * 32 + i] * alpha;
-            const size_t off = (size_t)row * p.N + col;
-            if (p.y_dt == NVFP4_DT_F32) store_out<float>(static_cast<float*>(p.y) + off, o, n);
-            else if (p.y_dt == NVFP4_DT_BF16) store_out<__nv_bfloat16>(static_cast<__nv_bfloat16*>(p.y) + off, o, n);
-            else store_out<__half>(static_cast<__half*>(p.y) + off, o, n);
-          }
-        }
-      }
+      epilogue_store(p, &tmap_y, sbase + SMEM_EPI + (uint32_t)(warp - 2) * EPI_BUF, v, alpha,
+                     (int)(tm * BM) + q * 32, (int)(tn * BN) + half * 128, lane);
     }
     // the tensor stores of this warp are complete before the CTA exits
     if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -581,6 +618,26 @@ inline bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
+// Output tensor map for the TMA-store epilogue: boxes of 32 rows x 32 bytes.
+// False (direct stores then) unless the row pitch is a multiple of 16 bytes;
+// y itself is 16-byte aligned.
+inline bool make_y_tmap(CUtensorMap* m, void* y, int y_dt, int64_t M, int64_t N) {
+  const uint64_t esz = y_dt == NVFP4_DT_F32 ? 4u : 2u;
+  memset(m, 0, sizeof(*m));
+  if (((uint64_t)N * esz) % 16u != 0) return false;
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+  cuuint64_t strides[1] = {(cuuint64_t)N * esz};
+  cuuint32_t box[2] = {(cuuint32_t)(32u / esz), 32u};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt = y_dt == NVFP4_DT_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : y_dt == NVFP4_DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return fn(m, dt, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace tc
 
 inline nvfp4_status qqmm_launch(bool mx, int64_t M, int64_t N, int64_t K, const uint32_t* a_codes,
@@ -594,25 +651,8 @@ inline nvfp4_status qqmm_launch(bool mx, int64_t M, int64_t N, int64_t K, const 
     snprintf(msg, msg_len, "[qqmm] cuTensorMapEncodeTiled failed");
     return NVFP4_ERR_CUDA;
   }
-  // Output tensor map: boxes of 32 rows x 32 bytes; usable when the row pitch
-  // is a multiple of 16 bytes (y itself is 16-byte aligned).
-  const uint64_t esz = y_dt == NVFP4_DT_F32 ? 4u : 2u;
   CUtensorMap ty;
-  memset(&ty, 0, sizeof(ty));
-  bool tma_store = ((uint64_t)N * esz) % 16u == 0;
-  if (tma_store) {
-    cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
-    cuuint64_t strides[1] = {(cuuint64_t)N * esz};
-    cuuint32_t box[2] = {(cuuint32_t)(32u / esz), 32u};
-    cuuint32_t estr[2] = {1, 1};
-    const CUtensorMapDataType dt = y_dt == NVFP4_DT_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                                   : y_dt == NVFP4_DT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    auto fn = encode_fn();
-    tma_store = fn && fn(&ty, dt, 2, y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-  }
+  const bool tma_store = make_y_tmap(&ty, y, y_dt, M, N);
   Params p;
   p.tma_store = tma_store ? 1 : 0;
   p.sfa = a_scales;
