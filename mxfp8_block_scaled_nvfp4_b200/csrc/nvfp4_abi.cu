@@ -373,8 +373,8 @@ nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32
   const uint32_t stages = qtc::pick_stages(M, K);
   if (stages > 0) {
     // tensor-core path: one CTA per 128 weight rows
-    CUtensorMap mw, ms;
-    if (!qtc::make_maps(&mw, &ms, w_codes, w_scales, (uint64_t)N, (uint64_t)K))
+    CUtensorMap mw;
+    if (!qtc::make_map(&mw, w_codes, (uint64_t)N, (uint64_t)K))
       return fail(NVFP4_ERR_CUDA, "[qmv] cuTensorMapEncodeTiled failed");
     qtc::Args a{x, g_x, w_codes, w_scales, g_w, y, (uint32_t)M, (uint32_t)N, (uint32_t)K, stages};
     const uint32_t MM = M == 1 ? 1u : 2u;
@@ -384,7 +384,7 @@ nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32
       using T = decltype(tag_t);
       auto go = [&](auto kern) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess) kern<<<grid, qtc::THREADS, smem, stream>>>(mw, ms, a);
+        if (e == cudaSuccess) kern<<<grid, qtc::THREADS, smem, stream>>>(mw, a);
       };
       if (M == 1) go(qtc::k_qmv_tc<T, 1>);
       else go(qtc::k_qmv_tc<T, 2>);

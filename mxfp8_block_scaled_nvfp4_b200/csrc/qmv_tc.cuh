@@ -16,27 +16,31 @@
 // subnormal or overflowing), the CTA computes its rows with the SIMT loop
 // instead, from an fp32 x_hat written over the plane tiles.  One MMA (M = 128 weight rows, N = 8 per x row, K = 64)
 // per k-step then yields, for each of the k-step's 4 blocks and 2 planes,
-//   D[n, (m, b, p)] = f8(sw[n, b]) * sum_{k in b} e2m1(q[n, k]) * e2m1(p_k)
-// (x-side scales 1), written to fresh TMEM columns; the epilogue warps
-// accumulate y[m, n] += U_(b,p) * D with U = A_b or B_b, and finally scale
-// by g_w / 2688.
+//   D[n, (m, b, p)] = sum_{k in b} e2m1(q[n, k]) * e2m1(p_k)
+// (unit block scales on both operands), written to fresh TMEM columns; the
+// epilogue warps accumulate y[m, n] += U_(b,p) * (f8(sw[n, b]) * D) with U =
+// A_b or B_b, and finally scale by g_w / 2688.  f8(sw) * D is exact in fp32
+// (a 4-bit by 11-bit significand product: D is a multiple of 1/4 below 2^9),
+// so this equals the block-scaled MMA's own output times U; applying the
+// weight scales in the epilogue removes every per-stage scale copy from the
+// tensor-core instruction stream, which is what bounds a CTA (each tcgen05
+// instruction of these N = 8 shapes costs about as much as a small MMA).
 //
-// CTA = 128 weight rows; warps: 0 TMA producer (codes [128 x 128 B] and
-// LINEAR scales [128 x 16 B] per stage), 1 TMEM allocator + MMA issuer,
-// 4-7 epilogue (TMEM lane quarters), 8-11 scale re-layout (LINEAR [128 rows
-// x 16 B] -> four 128x4 tiles for tcgen05.cp; stage kb on warp 8 + kb % 4).
-// Warps 1-11 compute the x_hat planes first, while warp 0 starts the
-// weight stream.
-// TMEM: a 256-column ring of MMA outputs drained in 128-column halves, the
-// weight scale tiles of every stage, one column of unit x-side scales.
+// CTA = 128 weight rows; warps: 0 TMA producer (codes [128 x 128 B] per
+// stage), 1 TMEM allocator + MMA issuer, 4-7 epilogue (TMEM lane quarters;
+// each lane reads its weight row's LINEAR scale bytes straight from global
+// memory, one ring half ahead).  Warps 1-11 compute the x_hat planes first,
+// while warp 0 starts the weight stream.
+// TMEM: a 256-column ring of MMA outputs drained in 128-column halves and
+// one tile of unit scales used by both operands.
 //
 // Every mbarrier wait of the MMA thread costs about as much as several of
 // these small MMAs (its shared-memory access queues behind the tensor
 // core's operand reads), so the MMA thread waits once per group of stages:
-// the re-layout warps arrive on one barrier per group of stages (two such
-// barriers alternate; the ring holds two groups, so a group barrier is not
-// reused before the MMA warp has passed its previous phase); ring halves
-// that were never used are not waited on.
+// the stages of a group complete on one barrier (the producer posts each
+// stage's bytes on it; two such barriers alternate, and the ring holds two
+// groups, so a group barrier is not reused before the MMA warp has passed
+// its previous phase); ring halves that were never used are not waited on.
 #pragma once
 
 #include <cuda.h>
@@ -49,18 +53,13 @@ namespace nvfp4 {
 namespace qtc {
 
 constexpr int THREADS = 384;
-constexpr int RELAYOUT_WARPS = 4;     // warps 8-11
-constexpr int FIRST_RELAYOUT_WARP = 8;
 constexpr int BM = 128;            // weight rows per CTA
-constexpr int MAX_STAGES = 8;
+constexpr int MAX_STAGES = 12;
 constexpr int A_STAGE = BM * 128;  // 16 KiB of codes (256 K)
-constexpr int S_STAGE = BM * 16;   // 2 KiB of LINEAR scales
-constexpr int T_STAGE = 4 * 512;   // four 128x4 scale tiles
-constexpr int STAGE_BYTES = A_STAGE + S_STAGE + T_STAGE;
+constexpr int STAGE_BYTES = A_STAGE;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t D_RING = 256;     // MMA output columns [0, 256)
-constexpr uint32_t T_SFB = 256;      // unit x-side scales
-constexpr uint32_t T_SFA = 260;      // weight scale tiles: 16 columns per stage
+constexpr uint32_t T_ONES = 256;     // unit block scales (both operands)
 
 // shared memory carve-up (bytes, from a 1024-aligned base)
 struct Layout {
@@ -184,12 +183,10 @@ __device__ __forceinline__ bool x_planes(const T* __restrict__ x, float gx, uint
 }
 
 template <typename T, int MM>
-__global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ CUtensorMap tmap_w,
-                                                       const __grid_constant__ CUtensorMap tmap_s, Args a) {
+__global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ CUtensorMap tmap_w, Args a) {
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[MAX_STAGES];
-  __shared__ __align__(8) uint64_t sf_grp[2];  // scale tiles of a group of stages ready
+  __shared__ __align__(8) uint64_t gfull[2];  // all stages of a group landed
   __shared__ __align__(8) uint64_t empty_bar[MAX_STAGES];
   __shared__ __align__(8) uint64_t dfull_bar[2];
   __shared__ __align__(8) uint64_t dempty_bar[2];
@@ -212,16 +209,36 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
   const uint32_t ncols = 8u * MM;         // MMA N
   const uint32_t steps_per_half = 128u / ncols;
   const uint32_t nb = a.K / 16u;
+  const uint32_t G = S / 2;               // stages per group (S is even)
+  const uint32_t groups = (kb_count + G - 1) / G;
 
-  const uint32_t G = S / 2;  // stages per group (S is even)
-  uint32_t issued = 0;       // weight stages issued (thread 0)
-  if (threadIdx.x == 0) {
-    for (uint32_t s = 0; s < S; ++s) {
-      mbar_init(smem_u32(&full_bar[s]), 1);
-      mbar_init(smem_u32(&empty_bar[s]), 1);
+  // stage kb into ring slot kb % S; its bytes complete on its group's
+  // barrier, and the last stage of a short final group also arrives for the
+  // stages that group lacks
+  auto issue = [&](uint32_t kb) {
+    const uint32_t grp = kb / G, bar = smem_u32(&gfull[grp & 1u]);
+    mbar_expect_tx(bar, A_STAGE);
+    tma_load_2d(sbase + L.ring + (kb % S) * STAGE_BYTES, &tmap_w, (int)(kb * 128u), (int)row0, bar);
+    if (kb + 1 == kb_count) {
+      const uint32_t missing = G - (kb_count - grp * G);
+      if (missing)
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(missing) : "memory");
     }
-    mbar_init(smem_u32(&sf_grp[0]), G);
-    mbar_init(smem_u32(&sf_grp[1]), G);
+  };
+  // the latest phases of both group barriers (all copies still in flight
+  // belong to the last two groups issued)
+  auto drain = [&](uint32_t issued) {
+    if (issued == 0) return;
+    const uint32_t last = (issued - 1) / G;
+    for (uint32_t gr = last > 0 ? last - 1 : 0; gr <= last; ++gr)
+      mbar_wait(smem_u32(&gfull[gr & 1u]), (gr >> 1) & 1u);
+  };
+
+  uint32_t issued = 0;  // weight stages issued (thread 0)
+  if (threadIdx.x == 0) {
+    for (uint32_t s = 0; s < S; ++s) mbar_init(smem_u32(&empty_bar[s]), 1);
+    mbar_init(smem_u32(&gfull[0]), G);
+    mbar_init(smem_u32(&gfull[1]), G);
     for (int h = 0; h < 2; ++h) {
       mbar_init(smem_u32(&dfull_bar[h]), 1);
       mbar_init(smem_u32(&dempty_bar[h]), 4);
@@ -229,12 +246,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     // the weight stream starts before TMEM allocation and the prologue
-    for (; issued < S && issued < kb_count; ++issued) {
-      const uint32_t bar = smem_u32(&full_bar[issued]);
-      mbar_expect_tx(bar, A_STAGE + S_STAGE);
-      tma_load_2d(sbase + L.ring + issued * STAGE_BYTES, &tmap_w, (int)(issued * 128u), (int)row0, bar);
-      tma_load_2d(sbase + L.ring + issued * STAGE_BYTES + A_STAGE, &tmap_s, (int)(issued * 16u), (int)row0, bar);
-    }
+    for (; issued < S && issued < kb_count; ++issued) issue(issued);
   }
   // zero the plane tiles (a plane row is nonzero only inside its own
   // 16-block: the prologue writes those bytes alone), fill the unit scale tile
@@ -268,8 +280,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
     // and SIMT rows for this CTA, after the loads in flight have landed
     float4* xs4 = reinterpret_cast<float4*>(smem + L.planes);
     qmv_prologue<T>(static_cast<const T*>(a.x), a.g_x, a.M, a.K, xs4, threadIdx.x, blockDim.x);
-    if (threadIdx.x == 0)
-      for (uint32_t i = 0; i < issued; ++i) mbar_wait(smem_u32(&full_bar[i]), 0);
+    if (threadIdx.x == 0) drain(issued);
     __syncthreads();
     const uint32_t end = min(row0 + BM, a.N);
     qmv_simt_rows<T, MM>(xs4, a.wc, a.wsc, dw, a.M, a.N, a.K, static_cast<T*>(a.y), row0 + warp,
@@ -283,46 +294,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
           abort_flag = 1;
           break;
         }
-        const uint32_t bar = smem_u32(&full_bar[s]);
-        mbar_expect_tx(bar, A_STAGE + S_STAGE);
-        tma_load_2d(sbase + L.ring + s * STAGE_BYTES, &tmap_w, (int)(kb * 128u), (int)row0, bar);
-        tma_load_2d(sbase + L.ring + s * STAGE_BYTES + A_STAGE, &tmap_s, (int)(kb * 16u), (int)row0, bar);
+        issue(kb);
         issued = kb + 1;
       }
-      const uint32_t first = issued > S ? issued - S : 0;
-      for (uint32_t i = first; i < issued; ++i) mbar_wait(smem_u32(&full_bar[i % S]), (i / S) & 1u);
-    }
-  } else if (warp >= FIRST_RELAYOUT_WARP && warp < FIRST_RELAYOUT_WARP + RELAYOUT_WARPS) {
-    // ------------------------------------------------------------ scale re-layout
-    // tile j (k-step j of the stage), row r: the 4 block scales of weight
-    // rows r, r+32, r+64, r+96 (the 128x4 tile order tcgen05.cp expects)
-    for (uint32_t kb = (uint32_t)(warp - FIRST_RELAYOUT_WARP); kb < kb_count; kb += RELAYOUT_WARPS) {
-      const uint32_t s = kb % S;
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full_bar[s]), (kb / S) & 1u)) ||
-          *(volatile int*)&abort_flag) {
-        abort_flag = 1;
-        break;
-      }
-      const uint8_t* raw = smem + L.ring + s * STAGE_BYTES + A_STAGE;
-      uint8_t* tiles = smem + L.ring + s * STAGE_BYTES + A_STAGE + S_STAGE;
-      const uint4 q0 = *reinterpret_cast<const uint4*>(raw + 16u * lane);
-      const uint4 q1 = *reinterpret_cast<const uint4*>(raw + 16u * (lane + 32));
-      const uint4 q2 = *reinterpret_cast<const uint4*>(raw + 16u * (lane + 64));
-      const uint4 q3 = *reinterpret_cast<const uint4*>(raw + 16u * (lane + 96));
-      *reinterpret_cast<uint4*>(tiles + 0 * 512 + 16u * lane) = make_uint4(q0.x, q1.x, q2.x, q3.x);
-      *reinterpret_cast<uint4*>(tiles + 1 * 512 + 16u * lane) = make_uint4(q0.y, q1.y, q2.y, q3.y);
-      *reinterpret_cast<uint4*>(tiles + 2 * 512 + 16u * lane) = make_uint4(q0.z, q1.z, q2.z, q3.z);
-      *reinterpret_cast<uint4*>(tiles + 3 * 512 + 16u * lane) = make_uint4(q0.w, q1.w, q2.w, q3.w);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) {
-        // the last stage of a short final group also arrives for the stages it lacks
-        const uint32_t grp = kb / G;
-        const uint32_t in_grp = min(G, kb_count - grp * G);
-        const uint32_t cnt = (kb == grp * G + in_grp - 1) ? 1u + (G - in_grp) : 1u;
-        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(&sf_grp[grp & 1u])), "r"(cnt)
-                     : "memory");
-      }
+      drain(issued);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -330,24 +305,23 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
     // for a drained ring half sits at a stage boundary (a half holds a
     // multiple of 4 k-steps), so each stage issues straight-line code.
     const bool leader = elect_one();
-    if (leader) tmem_cp_sf(tmem + T_SFB, sf_tile_desc(sbase + L.ones));
+    if (leader) tmem_cp_sf(tmem + T_ONES, sf_tile_desc(sbase + L.ones));
     const uint32_t idesc = (1u << 7) | (1u << 10) | ((ncols >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
     const uint64_t a_base = kmajor_sw128_desc(sbase + L.ring);
     const uint64_t b_base = kmajor_plain_desc(sbase + L.planes, 128u * MM, 128u);
-    const uint64_t t_base = sf_tile_desc(sbase + L.ring + A_STAGE + S_STAGE);
-    const uint32_t a_hi = (uint32_t)(a_base >> 32), b_hi = (uint32_t)(b_base >> 32), t_hi = (uint32_t)(t_base >> 32);
+    const uint32_t a_hi = (uint32_t)(a_base >> 32), b_hi = (uint32_t)(b_base >> 32);
     auto mk = [](uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; };
     uint32_t g = 0;  // global k-step
     bool ok = true;
-    for (uint32_t kb0 = 0; kb0 < kb_count && ok; kb0 += G) {
-      const uint32_t kb1 = min(kb0 + G, kb_count), grp = kb0 / G;
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sf_grp[grp & 1u]), (grp >> 1) & 1u)) ||
+    for (uint32_t grp = 0; grp < groups && ok; ++grp) {
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&gfull[grp & 1u]), (grp >> 1) & 1u)) ||
           *(volatile int*)&abort_flag) {
         ok = false;
         break;
       }
       tc_fence_after();
-      for (uint32_t kb = kb0; kb < kb1; ++kb) {
+      const uint32_t kb1 = min((grp + 1) * G, kb_count);
+      for (uint32_t kb = grp * G; kb < kb1; ++kb) {
         const uint32_t s = kb % S;
         const uint32_t hf = (g / steps_per_half) & 1u;  // ring half of this stage
         const uint32_t use = g / (2u * steps_per_half);   // times this half was used before
@@ -359,17 +333,13 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
           tc_fence_after();
         }
         if (leader) {
-          const uint32_t tsfa = tmem + T_SFA + 16u * s;
-#pragma unroll
-          for (uint32_t j = 0; j < 4; ++j)
-            tmem_cp_sf(tsfa + 4u * j, mk((uint32_t)t_base + ((s * STAGE_BYTES + 512u * j) >> 4), t_hi));
           const uint32_t dcol = (g % (2u * steps_per_half)) * ncols;
 #pragma unroll
           for (uint32_t j = 0; j < 4; ++j)
             mma_block_scaled<false>(tmem + dcol + j * ncols,
                                     mk((uint32_t)a_base + ((s * STAGE_BYTES + 32u * j) >> 4), a_hi),
-                                    mk((uint32_t)b_base + (((g + j) * 256u * MM) >> 4), b_hi), idesc, tsfa + 4u * j,
-                                    tmem + T_SFB, 0u);
+                                    mk((uint32_t)b_base + (((g + j) * 256u * MM) >> 4), b_hi), idesc, tmem + T_ONES,
+                                    tmem + T_ONES, 0u);
           if ((g + 4) % steps_per_half == 0 || g + 4 == ksteps) mma_commit(smem_u32(&dfull_bar[hf]));
           mma_commit(smem_u32(&empty_bar[s]));
         }
@@ -378,43 +348,69 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
       }
     }
     if (!ok && leader) abort_flag = 1;
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ epilogue
+    constexpr int NC = 8 * MM;              // MMA output columns per k-step
+    constexpr int SPH = 128 / NC;           // k-steps per ring half (16 or 8)
     const uint32_t q = warp & 3;
     const float* U = reinterpret_cast<const float*>(smem + L.uplane);
+    const uint32_t n = row0 + q * 32u + lane;
+    // this lane's weight row of LINEAR scales (a row past N reads row N-1:
+    // its codes were loaded as zeros, so the products vanish)
+    const uint8_t* srow = a.wsc + (size_t)min(n, a.N - 1u) * nb;
     float acc[MM];
 #pragma unroll
     for (int m = 0; m < MM; ++m) acc[m] = 0.0f;
     const uint32_t halves = (ksteps + steps_per_half - 1) / steps_per_half;
+    auto load_scales = [&](uint32_t h, uint4 (&sc)[SPH / 4]) {
+#pragma unroll
+      for (int j = 0; j < SPH / 4; ++j) {
+        const uint32_t off = 4u * h * (uint32_t)SPH + 16u * (uint32_t)j;  // 4 scale bytes per k-step
+        sc[j] = off < nb ? __ldg(reinterpret_cast<const uint4*>(srow + off)) : make_uint4(0, 0, 0, 0);
+      }
+    };
+    uint4 sc[SPH / 4];
+    load_scales(0, sc);
     bool ok = true;
     for (uint32_t h = 0; h < halves; ++h) {
       const uint32_t hf = h & 1u;
+      uint4 cur[SPH / 4];
+#pragma unroll
+      for (int j = 0; j < SPH / 4; ++j) cur[j] = sc[j];
+      if (h + 1 < halves) load_scales(h + 1, sc);  // next half's scales in flight
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&dfull_bar[hf]), (h >> 1) & 1u)) && !*(volatile int*)&abort_flag;
       tc_fence_after();
       if (!ok) break;
       const uint32_t g0 = h * steps_per_half;
       const uint32_t nsteps = min(steps_per_half, ksteps - g0);
-      for (uint32_t c = 0; c < nsteps * ncols; c += 32) {
-        float v[32];
-        tmem_ld32(tmem + ((q * 32u) << 16) + hf * 128u + c, v);
-        const uint32_t gc = g0 + c / (8u * MM);  // k-step of column c (32 is a multiple of 8 * MM)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          constexpr int NC = 8 * MM;
-          const int m = (i % NC) >> 3, bp = i & 7;  // compile-time after unrolling
-          const uint32_t gg = gc + (uint32_t)(i / NC);
-          if (c + i < nsteps * ncols) acc[m] = fmaf(U[(uint32_t)m * 2u * nb + 8u * gg + (uint32_t)bp], v[i], acc[m]);
+      for (int cc = 0; cc < 4; ++cc) {  // 32-column chunks of the half
+        if ((uint32_t)(cc * 32) < nsteps * ncols) {
+          float v[32];
+          tmem_ld32(tmem + ((q * 32u) << 16) + hf * 128u + (uint32_t)(cc * 32), v);
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {  // (plane A, plane B) of one block
+            const int m = (i % NC) >> 3, bl = (i & 7) >> 1;
+            const int kl = cc * 32 / NC + i / NC;  // k-step within the half
+            const int byte = 4 * kl + bl;          // its scale byte within the half
+            const uint4 w4 = cur[byte >> 4];
+            const uint32_t word = ((byte >> 2) & 3) == 0 ? w4.x : ((byte >> 2) & 3) == 1 ? w4.y
+                                  : ((byte >> 2) & 3) == 2 ? w4.z : w4.w;
+            const float sw = e4m3_to_f32(word >> (8 * (byte & 3)));
+            const uint32_t ub = (uint32_t)m * 2u * nb + 8u * (g0 + (uint32_t)kl) + 2u * (uint32_t)bl;
+            acc[m] = fmaf(U[ub], v[i] * sw, acc[m]);
+            acc[m] = fmaf(U[ub + 1u], v[i + 1] * sw, acc[m]);
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&dempty_bar[hf])) : "memory");
     }
-    const uint32_t row = row0 + q * 32u + lane;
-    if (ok && row < a.N) {
+    if (ok && n < a.N) {
 #pragma unroll
       for (int m = 0; m < MM; ++m)
-        if ((uint32_t)m < a.M) static_cast<T*>(a.y)[(size_t)m * a.N + row] = Elem<T>::from_f(acc[m] * dw);
+        if ((uint32_t)m < a.M) static_cast<T*>(a.y)[(size_t)m * a.N + n] = Elem<T>::from_f(acc[m] * dw);
     }
   }
   __syncwarp();  // lanes that skipped a one-lane role loop wait for it before the CTA barrier
@@ -426,33 +422,18 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
   }
 }
 
-// Tensor maps of the weight codes [N, K/2 bytes] (box 128 B x 128 rows,
-// 128-byte swizzle) and LINEAR scales [N, K/16 bytes] (box 16 B x 128 rows).
-inline bool make_maps(CUtensorMap* mw, CUtensorMap* ms, const uint32_t* wc, const uint8_t* wsc, uint64_t N,
-                      uint64_t K) {
+// Tensor map of the weight codes [N, K/2 bytes] (box 128 B x 128 rows,
+// 128-byte swizzle).
+inline bool make_map(CUtensorMap* mw, const uint32_t* wc, uint64_t N, uint64_t K) {
   auto fn = tc::encode_fn();
   if (!fn) return false;
-  {
-    cuuint64_t dims[2] = {K / 2, N};
-    cuuint64_t strides[1] = {K / 2};
-    cuuint32_t box[2] = {128, BM};
-    cuuint32_t estr[2] = {1, 1};
-    if (fn(mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint32_t*>(wc), dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return false;
-  }
-  {
-    cuuint64_t dims[2] = {K / 16, N};
-    cuuint64_t strides[1] = {K / 16};
-    cuuint32_t box[2] = {16, BM};
-    cuuint32_t estr[2] = {1, 1};
-    if (fn(ms, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(wsc), dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return false;
-  }
-  return true;
+  cuuint64_t dims[2] = {K / 2, N};
+  cuuint64_t strides[1] = {K / 2};
+  cuuint32_t box[2] = {128, BM};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint32_t*>(wc), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Stages that fit next to the plane tiles, plane scales and x_hat; 0 if the
