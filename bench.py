@@ -54,8 +54,8 @@ L2_FLUSH_BYTES = 256 << 20
 # dominant kernel, from one ncu capture of that kernel as it is now (the
 # summaries under profiles/ give the commands and the other counters).
 NCU_TRAFFIC_BYTES = {
-    "qqmm_sm100 (nvfp4)": 18950656 + 319232,    # profiles/qqmm_nvfp4_4096x4096x4096.md
-    "k_qmv_tc": 33104384 + 0,                   # profiles/qmv_tc_gemv_14336x4096.md
+    "qqmm_sm100 (nvfp4)": 18958336 + 225536,    # profiles/qqmm_nvfp4_4096x4096x4096.md
+    "k_qmv_tc": 33109760 + 0,                   # profiles/qmv_tc_gemv_14336x4096.md
     "gather_qmm": 90273024 + 3263744,           # profiles/gather_qmm_moe_T4096_top8_E64_N1408_K2048.md
 }
 
