@@ -425,6 +425,71 @@ void orc_mxfp8_decode_exact(const uint32_t* codes, const uint8_t* scales,
 }
 
 /* ------------------------------------------------------------------------ */
+/* 8b. MXFP4 quantize ([P2] fp_quantize_rowwise / fp_quantize_dequantize     */
+/*    with bits = 4 and the mx scale: the e8m0 scale type, no global scale). */
+/*    Per 32-block (the MX block size; the pages' mx scale is the e8m0 one): */
+/*      v   = max|x| / 6.0f                     fp32                          */
+/*      s   = e8m0 of v, rounded up (the conversion that the MXFP8 path uses; */
+/*            [P3] mlxcel note: CUDA rounds the E8M0 scale up)                */
+/*      k   = 1 / 2^(s-127)       fp32 (exact power of two)                  */
+/*      q_i = e2m1_rne_satfinite(x_i * k)      -> 4-bit code                 */
+/*    Codes: element 8w+i of a row in bits 4i..4i+3 of word w (as NVFP4).    */
+/*    Scales: LINEAR layout [rows, K/32].                                    */
+/* ------------------------------------------------------------------------ */
+void orc_mxfp4_quantize(const void* x, int dt, int64_t rows, int64_t K,
+                        uint32_t* codes, uint8_t* scales) {
+  const int64_t nb = K / 32;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t b = 0; b < nb; ++b) {
+      float xv[32];
+      float a = 0.0f;
+      for (int i = 0; i < 32; ++i) {
+        xv[i] = (float)orc_load(x, dt, r * K + b * 32 + i);
+        if (fabsf(xv[i]) > a) a = fabsf(xv[i]);
+      }
+      float v = a / 6.0f;
+      int s = orc_e8m0_ceil(v);
+      scales[r * nb + b] = (uint8_t)s;
+      float k = 1.0f / (float)orc_e8m0_value(s);
+      uint32_t w[4] = {0, 0, 0, 0};
+      for (int i = 0; i < 32; ++i) {
+        uint32_t q = (uint32_t)orc_e2m1_rne_satfinite(xv[i] * k);
+        w[i / 8] |= q << (4 * (i % 8));
+      }
+      for (int j = 0; j < 4; ++j) codes[(r * K + b * 32) / 8 + j] = w[j];
+    }
+  }
+}
+
+/* MXFP4 dequantize ([P1] fp_dequantize fallback, e8m0 branch with 4-bit
+ * codes): w_hat = T( e2m1(q) * 2^(s-127) ), product in fp32. */
+void orc_mxfp4_dequantize(const uint32_t* codes, const uint8_t* scales,
+                          int64_t rows, int64_t K, void* out, int out_dt) {
+  const int64_t nb = K / 32;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t k = 0; k < K; ++k) {
+      int64_t idx = r * K + k;
+      int q = (codes[idx / 8] >> (4 * (idx % 8))) & 15;
+      float v = (float)orc_e2m1_value(q) * (float)orc_e8m0_value(scales[r * nb + k / 32]);
+      orc_store(out, out_dt, idx, v);
+    }
+  }
+}
+
+/* Exact real value of each MXFP4 element, e2m1(q) * 2^(s-127), float64. */
+void orc_mxfp4_decode_exact(const uint32_t* codes, const uint8_t* scales,
+                            int64_t rows, int64_t K, double* out) {
+  const int64_t nb = K / 32;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t k = 0; k < K; ++k) {
+      int64_t idx = r * K + k;
+      int q = (codes[idx / 8] >> (4 * (idx % 8))) & 15;
+      out[idx] = orc_e2m1_value(q) * orc_e8m0_value(scales[r * nb + k / 32]);
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
 /* 9. Scale layout for the block-scaled MMA ([P5] qqmm_utils.cu comment:     */
 /*    tmp = s.reshape(rb, 4, 32, cb, 4); tmp.transpose(0, 3, 2, 1, 4), and   */
 /*    its worked index table; [P1] pad_and_swizzle_scales: pad to 128-row x  */

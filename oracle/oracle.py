@@ -86,6 +86,9 @@ def _L():
                 "orc_mxfp8_quantize": (None, [P, I, I64, I64, P, P]),
                 "orc_mxfp8_dequantize": (None, [P, P, I64, I64, P, I]),
                 "orc_mxfp8_decode_exact": (None, [P, P, I64, I64, P]),
+                "orc_mxfp4_quantize": (None, [P, I, I64, I64, P, P]),
+                "orc_mxfp4_dequantize": (None, [P, P, I64, I64, P, I]),
+                "orc_mxfp4_decode_exact": (None, [P, P, I64, I64, P]),
                 "orc_swizzle_scales": (None, [P, I64, I64, P]),
                 "orc_load_array": (None, [P, I, I64, P]),
                 "orc_store_array": (None, [P, I64, I, P]),
@@ -282,6 +285,40 @@ def mxfp8_decode_exact(codes, scales) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# MXFP4 quantize / dequantize (the 4-bit codes with the mx scale)
+# --------------------------------------------------------------------------
+def mxfp4_quantize(x: np.ndarray, dt: str):
+    """MXFP4 quantize: 32-blocks, E8M0 scale of max|x|/6 rounded up, e2m1
+    codes ([P2] fp_quantize_rowwise with bits 4 and the mx scale).
+    Returns (codes uint32 [rows, K/8], scales uint8 [rows, K/32] LINEAR)."""
+    x = _raw(x, dt)
+    rows, K = x.shape
+    assert K % 32 == 0
+    codes = np.zeros((rows, K // 8), dtype=np.uint32)
+    scales = np.zeros((rows, K // 32), dtype=np.uint8)
+    _L().orc_mxfp4_quantize(_p(x), DT[dt], rows, K, _p(codes), _p(scales))
+    return codes, scales
+
+
+def mxfp4_dequantize(codes, scales, out_dt="bf16") -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, K = codes.shape[0], codes.shape[1] * 8
+    out = np.empty((rows, K), dtype=NP_CONTAINER[out_dt])
+    _L().orc_mxfp4_dequantize(_p(codes), _p(scales), rows, K, _p(out), DT[out_dt])
+    return out
+
+
+def mxfp4_decode_exact(codes, scales) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, K = codes.shape[0], codes.shape[1] * 8
+    out = np.empty((rows, K), dtype=np.float64)
+    _L().orc_mxfp4_decode_exact(_p(codes), _p(scales), rows, K, _p(out))
+    return out
+
+
+# --------------------------------------------------------------------------
 # a8-a9, a12: dense block-scaled matmul y = x_hat . w_hat^T
 # --------------------------------------------------------------------------
 def qqmm(a_codes, a_scales, b_codes, b_scales, mode="nvfp4", g_x=None, g_w=None,
@@ -305,6 +342,10 @@ def qqmm(a_codes, a_scales, b_codes, b_scales, mode="nvfp4", g_x=None, g_w=None,
         assert g_x is None and g_w is None
         xh = mxfp8_decode_exact(a_codes, a_scales)
         wh = mxfp8_decode_exact(b_codes, b_scales)
+    elif mode == "mxfp4":
+        assert g_x is None and g_w is None
+        xh = mxfp4_decode_exact(a_codes, a_scales)
+        wh = mxfp4_decode_exact(b_codes, b_scales)
     else:
         raise ValueError(mode)
     y_ref = xh @ wh.T
