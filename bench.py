@@ -15,6 +15,7 @@ One step = one pass over every row of the hot path, each on its workload
   moe       a10     gather_qmm: 64 experts [1408,2048], 4096 tokens, top-8 -> bf16
   moe_decode f2     gather_qmm decode (gather_qmv): the same experts, 4 tokens, top-8
   mxfp8     a11-a12 mxfp8 quantize x2 + FP8 GEMM 8192^3 -> bf16
+  mxfp4     f3      mxfp4 quantize x2 + FP4 GEMM 8192^3 (mxfp4 mode) -> bf16
 
 The headline ``value`` is the prefill qqmm op in TFLOP/s (2*M*N*K over the
 whole op: amaxes, quantizes and GEMM); every row's own metric, time and
@@ -462,7 +463,45 @@ class Mxfp8(Row):
                                        "peak_note": "measured bf16 burst x 2 (nominal fp8:bf16 ratio)"}}
 
 
-ROWS = [Quant1G, Gemv, Dequant, Prefill, PrefillBwd, Moe, MoeDecode, Mxfp8]
+class Mxfp4(Row):
+    """The MXFP4 mode on the MXFP8 row's operands (x, W [8192, 8192] bf16
+    N(0,1)): two MXFP4 quantizes (e8m0 scales per 32, SWIZZLED) and the
+    block-scaled GEMM on the FP4 tensor pipe."""
+    name, launches = "mxfp4", 3
+
+    def setup(self):
+        d = self.wl.make("mxfp4", device=self.dev)
+        self.x, self.w = d["x"], d["w"]
+        self.M, self.K = self.x.shape
+        self.N = self.w.shape[0]
+        mk = lambda r: (torch.empty(r, self.K // 8, dtype=torch.int32, device=self.dev),
+                        torch.empty(self.nv.scale_shape(r, self.K // 32, "swizzled"), dtype=torch.uint8,
+                                    device=self.dev))
+        self.xc, self.xs = mk(self.M)
+        self.wc, self.ws = mk(self.N)
+        self.y = torch.empty(self.M, self.N, dtype=torch.bfloat16, device=self.dev)
+        self.flop = 2 * self.M * self.N * self.K
+        self.bytes_q = self.M * self.K * 2 + self.M * self.K // 2 + self.M * self.K // 32
+        self.nv.qqmm(self.xc[:128], self.xs[:128], self.wc[:128], self.ws[:128], self.K, "mxfp4",
+                     out=self.y[:128, :128].contiguous())
+
+    def calls(self):
+        nv = self.nv
+        return [("quantize_x", lambda: nv.mxfp4_quantize(self.x, "swizzled", self.xc, self.xs)),
+                ("quantize_w", lambda: nv.mxfp4_quantize(self.w, "swizzled", self.wc, self.ws)),
+                ("gemm", lambda: nv.qqmm(self.xc, self.xs, self.wc, self.ws, self.K, "mxfp4", out=self.y))]
+
+    def report(self, ms, row_ms, peaks):
+        fp4_peak = peaks["bf16_tflops"] * 4.0
+        tf = self.flop / ms["gemm"] / 1e9
+        return {"metric": "mxfp4 qqmm TFLOP/s", "unit": "TFLOP/s", "value": self.flop / row_ms / 1e9,
+                "ms": ms, "quantize_gbs": self.bytes_q / ms["quantize_x"] / 1e6,
+                "roofline": {"bound": "tensor", "kernel": "qqmm_sm100 (mxfp4)", "achieved": tf,
+                             "peak": fp4_peak, "unit": "TFLOP/s", "frac": tf / fp4_peak,
+                             "peak_note": "measured bf16 burst x 4 (nominal fp4:bf16 ratio)"}}
+
+
+ROWS = [Quant1G, Gemv, Dequant, Prefill, PrefillBwd, Moe, MoeDecode, Mxfp8, Mxfp4]
 
 
 # ---------------------------------------------------------------------------

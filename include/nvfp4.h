@@ -72,7 +72,7 @@ typedef enum {
 
 typedef enum { NVFP4_DT_F32 = 0, NVFP4_DT_F16 = 1, NVFP4_DT_BF16 = 2 } nvfp4_dtype;
 typedef enum { NVFP4_LAYOUT_LINEAR = 0, NVFP4_LAYOUT_SWIZZLED = 1 } nvfp4_layout;
-typedef enum { NVFP4_MODE_NVFP4 = 0, NVFP4_MODE_MXFP8 = 1 } nvfp4_mode;
+typedef enum { NVFP4_MODE_NVFP4 = 0, NVFP4_MODE_MXFP8 = 1, NVFP4_MODE_MXFP4 = 2 } nvfp4_mode;
 
 /* Short text of a status code. */
 NVFP4_API const char* nvfp4_status_string(nvfp4_status s);
@@ -147,6 +147,24 @@ NVFP4_API nvfp4_status mxfp8_dequantize(const uint32_t* codes, const uint8_t* sc
                               nvfp4_layout layout, int64_t rows, int64_t K, void* out,
                               nvfp4_dtype out_dt, nvfp4_stream_t stream);
 
+/* f3 -- MXFP4 quantize ([P2] fp_quantize_rowwise with 4 bits and the e8m0
+ * (mx) scale; group size 32; the E8M0 scale rounded up as for MXFP8, [P3]).
+ * Per 32-block: s = ue8m0_round_up(amax / 6);
+ *   q_i = e2m1_rne_satfinite(x_i / 2^(s-127)), 8 codes per uint32 as NVFP4.
+ * x [rows, K] of dt, K % 32 == 0; codes [rows, K/8] uint32; scales e8m0
+ * bytes in `layout`: nvfp4_scale_bytes(rows, K/32, layout).  No global
+ * scale.  Errors as nvfp4_quantize. */
+NVFP4_API nvfp4_status mxfp4_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K,
+                                      uint32_t* codes, uint8_t* scales, nvfp4_layout layout,
+                                      nvfp4_stream_t stream);
+
+/* MXFP4 dequantize ([P1] fp_dequantize fallback, e8m0 branch with 4-bit
+ * codes): out = T(e2m1(q) * 2^(s-127)).  codes [rows, K/8], scales as
+ * produced by mxfp4_quantize in `layout`, out [rows, K] of out_dt. */
+NVFP4_API nvfp4_status mxfp4_dequantize(const uint32_t* codes, const uint8_t* scales,
+                                        nvfp4_layout layout, int64_t rows, int64_t K, void* out,
+                                        nvfp4_dtype out_dt, nvfp4_stream_t stream);
+
 /* a4 -- LINEAR -> SWIZZLED re-layout of a [rows, cols] uint8 scale matrix
  * ([P5] swizzle_scales; [P1] pad_and_swizzle_scales), for scales produced
  * elsewhere.  swz: nvfp4_scale_bytes(rows, cols, SWIZZLED) bytes, all
@@ -162,6 +180,9 @@ NVFP4_API nvfp4_status nvfp4_swizzle_scales(const uint8_t* lin, int64_t rows, in
  *    alpha = (g_x / 2688) * (g_w / 2688) ([P2] compute_qqmm_pointers).
  *  mode MXFP8: a_codes [M, K/4], b_codes [N, K/4], e8m0 scales SWIZZLED
  *    (K/32 per row); g_x, g_w must be NULL.
+ *  mode MXFP4: a_codes [M, K/8], b_codes [N, K/8] (mxfp4_quantize), e8m0
+ *    scales SWIZZLED (K/32 per row); g_x, g_w must be NULL;
+ *    y = sum_b 2^(sx-127) 2^(sw-127) sum_k e2m1 e2m1.
  *  K % 32 == 0 (NVFP4: K % 64 recommended; a ragged last 64-block is zero
  *  padded by the kernel).  y: [M, N] of y_dt (fp32, fp16 or bf16), written. */
 NVFP4_API nvfp4_status qqmm(nvfp4_mode mode, int64_t M, int64_t N, int64_t K, const uint32_t* a_codes,

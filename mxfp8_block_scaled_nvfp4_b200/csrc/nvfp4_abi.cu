@@ -169,10 +169,11 @@ nvfp4_status nvfp4_amax(const void* x, nvfp4_dtype dt, int64_t n, float* g_out, 
   return check_launch("amax");
 }
 
-static nvfp4_status quantize_common(const char* tag, bool mx, const void* x, nvfp4_dtype dt,
+// kind: 0 NVFP4, 1 MXFP8, 2 MXFP4 (the two MX kinds use 32-element blocks)
+static nvfp4_status quantize_common(const char* tag, int kind, const void* x, nvfp4_dtype dt,
                                     int64_t rows, int64_t K, const float* g, uint32_t* codes,
                                     uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
-  const int group = mx ? 32 : 16;
+  const int group = kind ? 32 : 16;
   if (!valid_dt(dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] dtype must be float32, float16 or bfloat16", tag);
   if (layout != NVFP4_LAYOUT_LINEAR && layout != NVFP4_LAYOUT_SWIZZLED)
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] unknown scale layout", tag);
@@ -199,8 +200,11 @@ static nvfp4_status quantize_common(const char* tag, bool mx, const void* x, nvf
   const unsigned grid = ew_grid(d, ((uint64_t)n_half + kUnroll - 1) / kUnroll);
   dispatch_dt(dt, [&](auto tag_t) {
     using T = decltype(tag_t);
-    if (mx)
+    if (kind == 1)
       k_mxfp8_quantize<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, codes, so,
+                                                           (uint32_t)rows);
+    else if (kind == 2)
+      k_mxfp4_quantize<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, codes, so,
                                                            (uint32_t)rows);
     else
       k_nvfp4_quantize<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, g, codes, so,
@@ -211,7 +215,7 @@ static nvfp4_status quantize_common(const char* tag, bool mx, const void* x, nvf
 
 nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K, const float* g,
                             uint32_t* codes, uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
-  return quantize_common("quantize", false, x, dt, rows, K, g, codes, scales, layout, stream);
+  return quantize_common("quantize", 0, x, dt, rows, K, g, codes, scales, layout, stream);
 }
 
 nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, int64_t rows, int64_t cols, const float* g,
@@ -250,13 +254,18 @@ nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, int64_t ro
 
 nvfp4_status mxfp8_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K, uint32_t* codes,
                             uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
-  return quantize_common("mxfp8_quantize", true, x, dt, rows, K, nullptr, codes, scales, layout, stream);
+  return quantize_common("mxfp8_quantize", 1, x, dt, rows, K, nullptr, codes, scales, layout, stream);
 }
 
-static nvfp4_status dequantize_common(const char* tag, bool mx, const uint32_t* codes, const uint8_t* scales,
+nvfp4_status mxfp4_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K, uint32_t* codes,
+                            uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
+  return quantize_common("mxfp4_quantize", 2, x, dt, rows, K, nullptr, codes, scales, layout, stream);
+}
+
+static nvfp4_status dequantize_common(const char* tag, int kind, const uint32_t* codes, const uint8_t* scales,
                                       nvfp4_layout layout, int64_t rows, int64_t K, const float* g, void* out,
                                       nvfp4_dtype out_dt, nvfp4_stream_t stream) {
-  const int group = mx ? 32 : 16;
+  const int group = kind ? 32 : 16;
   if (!valid_dt(out_dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] output dtype must be float32, float16 or bfloat16", tag);
   if (layout != NVFP4_LAYOUT_LINEAR && layout != NVFP4_LAYOUT_SWIZZLED)
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] unknown scale layout", tag);
@@ -279,8 +288,10 @@ static nvfp4_status dequantize_common(const char* tag, bool mx, const uint32_t* 
   const unsigned grid = ew_grid(d, n_half);
   dispatch_dt(out_dt, [&](auto tag_t) {
     using T = decltype(tag_t);
-    if (mx)
+    if (kind == 1)
       k_mxfp8_dequantize<T><<<grid, kEwThreads, 0, stream>>>(codes, si, n_half, static_cast<T*>(out));
+    else if (kind == 2)
+      k_mxfp4_dequantize<T><<<grid, kEwThreads, 0, stream>>>(codes, si, n_half, static_cast<T*>(out));
     else
       k_nvfp4_dequantize<T><<<grid, kEwThreads, 0, stream>>>(codes, si, g, n_half, static_cast<T*>(out));
   });
@@ -289,12 +300,17 @@ static nvfp4_status dequantize_common(const char* tag, bool mx, const uint32_t* 
 
 nvfp4_status nvfp4_dequantize(const uint32_t* codes, const uint8_t* scales, nvfp4_layout layout, int64_t rows,
                               int64_t K, const float* g, void* out, nvfp4_dtype out_dt, nvfp4_stream_t stream) {
-  return dequantize_common("dequantize", false, codes, scales, layout, rows, K, g, out, out_dt, stream);
+  return dequantize_common("dequantize", 0, codes, scales, layout, rows, K, g, out, out_dt, stream);
 }
 
 nvfp4_status mxfp8_dequantize(const uint32_t* codes, const uint8_t* scales, nvfp4_layout layout, int64_t rows,
                               int64_t K, void* out, nvfp4_dtype out_dt, nvfp4_stream_t stream) {
-  return dequantize_common("mxfp8_dequantize", true, codes, scales, layout, rows, K, nullptr, out, out_dt, stream);
+  return dequantize_common("mxfp8_dequantize", 1, codes, scales, layout, rows, K, nullptr, out, out_dt, stream);
+}
+
+nvfp4_status mxfp4_dequantize(const uint32_t* codes, const uint8_t* scales, nvfp4_layout layout, int64_t rows,
+                              int64_t K, void* out, nvfp4_dtype out_dt, nvfp4_stream_t stream) {
+  return dequantize_common("mxfp4_dequantize", 2, codes, scales, layout, rows, K, nullptr, out, out_dt, stream);
 }
 
 nvfp4_status nvfp4_swizzle_scales(const uint8_t* lin, int64_t rows, int64_t cols, uint8_t* swz,
@@ -328,8 +344,8 @@ static nvfp4_status check_qqmm_global_scales(nvfp4_mode mode, const float* g_x, 
 nvfp4_status qqmm(nvfp4_mode mode, int64_t M, int64_t N, int64_t K, const uint32_t* a_codes,
                   const uint8_t* a_scales, const uint32_t* b_codes, const uint8_t* b_scales, const float* g_x,
                   const float* g_w, void* y, nvfp4_dtype y_dt, nvfp4_stream_t stream) {
-  if (mode != NVFP4_MODE_NVFP4 && mode != NVFP4_MODE_MXFP8)
-    return fail(NVFP4_ERR_INVALID_ARG, "[qqmm] Only 'nvfp4' and 'mxfp8' modes are supported.");
+  if (mode != NVFP4_MODE_NVFP4 && mode != NVFP4_MODE_MXFP8 && mode != NVFP4_MODE_MXFP4)
+    return fail(NVFP4_ERR_INVALID_ARG, "[qqmm] Only 'nvfp4', 'mxfp8' and 'mxfp4' modes are supported.");
   nvfp4_status st = check_qqmm_global_scales(mode, g_x, g_w);
   if (st != NVFP4_OK) return st;
   if (!valid_dt(y_dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[qqmm] output dtype must be float32, float16 or bfloat16");
@@ -346,7 +362,7 @@ nvfp4_status qqmm(nvfp4_mode mode, int64_t M, int64_t N, int64_t K, const uint32
   st = device_info("qqmm", &d);
   if (st != NVFP4_OK) return st;
   if (M * N == 0) return ok();
-  return qqmm_launch(mode == NVFP4_MODE_MXFP8, M, N, K, a_codes, a_scales, b_codes, b_scales, g_x, g_w, y,
+  return qqmm_launch((int)mode, M, N, K, a_codes, a_scales, b_codes, b_scales, g_x, g_w, y,
                      (int)y_dt, d.sm_count, stream, t_msg, sizeof(t_msg));
 }
 

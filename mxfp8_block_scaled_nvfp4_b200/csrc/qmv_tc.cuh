@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
           const uint32_t dcol = (g % (2u * steps_per_half)) * ncols;
 #pragma unroll
           for (uint32_t j = 0; j < 4; ++j)
-            mma_block_scaled<false>(tmem + dcol + j * ncols,
+            mma_block_scaled<kNV>(tmem + dcol + j * ncols,
                                     mk((uint32_t)a_base + ((s * STAGE_BYTES + 32u * j) >> 4), a_hi),
                                     mk((uint32_t)b_base + (((g + j) * 256u * MM) >> 4), b_hi), idesc, tmem + T_ONES,
                                     tmem + T_ONES, 0u);

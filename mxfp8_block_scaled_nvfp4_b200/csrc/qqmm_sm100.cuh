@@ -6,7 +6,9 @@
 // NVFP4: e2m1 codes, ue4m3 scales per 16 elements, alpha = (g_x / 2688) *
 // (g_w / 2688) (the device alpha of compute_qqmm_pointers, "mlx 0.30.7.2 ->
 // 0.30.7.6" diff, page 7, qqmm_utils.cu).  MXFP8: e4m3 codes, ue8m0 scales per
-// 32 elements, alpha = 1.  Folding the global scales into alpha is exact in
+// 32 elements, alpha = 1.  MXFP4: e2m1 codes, ue8m0 scales per 32 elements
+// (kind::mxf4nvf4 .block32: two scale bytes per K = 64 step, picked by the
+// scale-factor id), alpha = 1.  Folding the global scales into alpha is exact in
 // real arithmetic (sum (c sx dx)(c sw dw) = dx dw sum c sx c sw), and no
 // operand is rounded to a narrower type on this path, so it is equivalent to
 // decoding each block with its global scale.
@@ -166,10 +168,22 @@ __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-template <bool MX>
+// Operand kinds of the dense GEMM: NVFP4 (e2m1, ue4m3 per 16), MXFP8 (e4m3,
+// ue8m0 per 32), MXFP4 (e2m1, ue8m0 per 32).
+enum { kNV = 0, kMX8 = 1, kMX4 = 2 };
+
+template <int KIND>
 __device__ __forceinline__ void mma_block_scaled(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                                  uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
-  if constexpr (MX) {
+  if constexpr (KIND == kMX4) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+  } else if constexpr (KIND == kMX8) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
@@ -354,7 +368,7 @@ __device__ __forceinline__ void tile_coords(uint32_t t, uint32_t mt, uint32_t nt
   tn = r / gm;
 }
 
-template <bool MX>
+template <int KIND>
 __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUtensorMap tmap_a,
                                                      const __grid_constant__ CUtensorMap tmap_b,
                                                      const __grid_constant__ CUtensorMap tmap_y, Params p) {
@@ -391,7 +405,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_holder;
-  const uint32_t tiles_per_stage = MX ? 1u : 4u;
+  const uint32_t tiles_per_stage = KIND == kNV ? 4u : KIND == kMX8 ? 1u : 2u;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -465,25 +479,34 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
           const uint32_t g0 = kb * tiles_per_stage;
           if (g0 + tiles_per_stage <= p.sf_groups && p.k_bytes >= (kb + 1) * BKB) {
             // full stage: all scale tiles and all four k-steps present
-            if (MX) {
+            if constexpr (KIND == kMX8) {
               tmem_cp_sf(tsfa, mk(sfa_lo, sfa_hi));
               tmem_cp_sf(tsfb, mk(sfb_lo, sfb_hi));
               if (b_second) tmem_cp_sf(tsfb + 4, mk(sfb_lo + (4 * 512 >> 4), sfb_hi));
 #pragma unroll
               for (uint32_t j = 0; j < 4; ++j)
-                mma_block_scaled<true>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi),
+                mma_block_scaled<kMX8>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi),
                                        block_scaled_idesc(0u, 1u, j), tsfa, tsfb, (kb | j) != 0);
             } else {
+              // NVFP4: one scale tile per k-step; MXFP4: one per two k-steps,
+              // the k-step's two scale bytes selected by the scale-factor id
+              constexpr uint32_t TPS = KIND == kNV ? 4u : 2u;
 #pragma unroll
-              for (uint32_t u = 0; u < 4; ++u) {
+              for (uint32_t u = 0; u < TPS; ++u) {
                 tmem_cp_sf(tsfa + 4 * u, mk(sfa_lo + 32 * u, sfa_hi));
                 tmem_cp_sf(tsfb + 8 * u, mk(sfb_lo + 32 * u, sfb_hi));
                 if (b_second) tmem_cp_sf(tsfb + 8 * u + 4, mk(sfb_lo + (4 * 512 >> 4) + 32 * u, sfb_hi));
               }
 #pragma unroll
-              for (uint32_t j = 0; j < 4; ++j)
-                mma_block_scaled<false>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi), idesc_nv, tsfa + 4 * j,
+              for (uint32_t j = 0; j < 4; ++j) {
+                if constexpr (KIND == kNV)
+                  mma_block_scaled<kNV>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi), idesc_nv, tsfa + 4 * j,
                                         tsfb + 8 * j, (kb | j) != 0);
+                else
+                  mma_block_scaled<kMX4>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi),
+                                         block_scaled_idesc(1u, 1u, (j & 1u) * 2u), tsfa + 4 * (j >> 1),
+                                         tsfb + 8 * (j >> 1), (kb | j) != 0);
+              }
             }
           } else {
             // ragged last stage: only the scale tiles and k-steps that exist
@@ -496,12 +519,16 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
             }
             for (uint32_t j = 0; j < 4; ++j) {
               if (kb * BKB + j * 32u >= p.k_bytes) break;
-              if (MX)
-                mma_block_scaled<true>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi),
+              if constexpr (KIND == kMX8)
+                mma_block_scaled<kMX8>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi),
                                        block_scaled_idesc(0u, 1u, j), tsfa, tsfb, (kb | j) != 0);
+              else if constexpr (KIND == kMX4)
+                mma_block_scaled<kMX4>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi),
+                                       block_scaled_idesc(1u, 1u, (j & 1u) * 2u), tsfa + 4 * (j >> 1),
+                                       tsfb + 8 * (j >> 1), (kb | j) != 0);
               else
-                mma_block_scaled<false>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi), idesc_nv, tsfa + 4 * j,
-                                        tsfb + 8 * j, (kb | j) != 0);
+                mma_block_scaled<kNV>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi), idesc_nv, tsfa + 4 * j,
+                                      tsfb + 8 * j, (kb | j) != 0);
             }
           }
             mma_commit(smem_u32(&empty_bar[s]));
@@ -553,7 +580,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
     const int q = warp & 3;                // TMEM lane quarter this warp may read
     const int half = (warp - 2) >> 2;      // which 128 accumulator columns
     float alpha = 1.0f;
-    if (!MX && p.g_x != nullptr) alpha = (__ldg(p.g_x) / kGlobalEncode) * (__ldg(p.g_w) / kGlobalEncode);
+    if (KIND == kNV && p.g_x != nullptr) alpha = (__ldg(p.g_x) / kGlobalEncode) * (__ldg(p.g_w) / kGlobalEncode);
     uint32_t tile_i = 0;
     for (uint32_t t = blockIdx.x; t < tiles; t += gridDim.x, ++tile_i) {
       uint32_t tm, tn;
@@ -640,11 +667,12 @@ inline bool make_y_tmap(CUtensorMap* m, void* y, int y_dt, int64_t M, int64_t N)
 
 }  // namespace tc
 
-inline nvfp4_status qqmm_launch(bool mx, int64_t M, int64_t N, int64_t K, const uint32_t* a_codes,
+inline nvfp4_status qqmm_launch(int kind, int64_t M, int64_t N, int64_t K, const uint32_t* a_codes,
                                 const uint8_t* a_scales, const uint32_t* b_codes, const uint8_t* b_scales,
                                 const float* g_x, const float* g_w, void* y, int y_dt, int sm_count,
                                 cudaStream_t stream, char* msg, size_t msg_len) {
   using namespace tc;
+  const bool mx = kind == tc::kMX8;
   const uint64_t k_bytes = mx ? (uint64_t)K : (uint64_t)K / 2;
   CUtensorMap ta, tb;
   if (!make_tmap(&ta, a_codes, (uint64_t)M, k_bytes, BM) || !make_tmap(&tb, b_codes, (uint64_t)N, k_bytes, BN)) {
@@ -666,19 +694,19 @@ inline nvfp4_status qqmm_launch(bool mx, int64_t M, int64_t N, int64_t K, const 
   p.y_dt = y_dt;
   p.k_bytes = (uint32_t)k_bytes;
   p.kb_count = (uint32_t)((k_bytes + BKB - 1) / BKB);
-  const int64_t sf_cols = mx ? K / 32 : K / 16;
+  const int64_t sf_cols = kind == tc::kNV ? K / 16 : K / 32;
   p.sf_groups = (uint32_t)((sf_cols + 3) / 4);
   p.rows_b_pad = (uint32_t)((N + 127) / 128 * 128);
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   dim3 grid((unsigned)(tiles < sm_count ? tiles : sm_count));  // persistent: one CTA per SM
   cudaError_t e;
-  if (mx) {
-    e = cudaFuncSetAttribute(k_qqmm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-    if (e == cudaSuccess) k_qqmm<true><<<grid, THREADS, SMEM_ALLOC, stream>>>(ta, tb, ty, p);
-  } else {
-    e = cudaFuncSetAttribute(k_qqmm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-    if (e == cudaSuccess) k_qqmm<false><<<grid, THREADS, SMEM_ALLOC, stream>>>(ta, tb, ty, p);
-  }
+  auto go = [&](auto kern) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+    if (e == cudaSuccess) kern<<<grid, THREADS, SMEM_ALLOC, stream>>>(ta, tb, ty, p);
+  };
+  if (kind == kMX8) go(k_qqmm<kMX8>);
+  else if (kind == kMX4) go(k_qqmm<kMX4>);
+  else go(k_qqmm<kNV>);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     snprintf(msg, msg_len, "[qqmm] launch failed: %s", cudaGetErrorString(e));

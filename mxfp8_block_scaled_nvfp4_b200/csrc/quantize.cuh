@@ -275,6 +275,55 @@ __global__ void __launch_bounds__(kEwThreads) k_mxfp8_quantize(
   zero_scale_padding(so, rows);
 }
 
+// ---------------------------------------------------------------------------
+// MXFP4 quantize (fp_quantize_rowwise with bits 4 and the e8m0 scale, "mlx
+// 0.30.7.2 -> 0.30.7.6" diff, page 7; the scale rounded up as for MXFP8):
+// per 32-block: v = max|x| / 6;  s = ue8m0 rounded up (v);
+//   k = 1 / 2^(s-127);  q_i = e2m1_rne_satfinite(x_i * k), 8 codes per word
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kEwThreads) k_mxfp4_quantize(
+    const T* __restrict__ x, uint32_t n_half, uint32_t* __restrict__ codes, ScaleOut so,
+    uint32_t rows) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (uint32_t base = warp * 32u * kUnroll; base < n_half; base += nwarps * 32u * kUnroll) {
+    float v[kUnroll][8];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const uint32_t hb = base + u * 32u + lane;
+      if (hb < n_half) {
+        load8<T>(x + (size_t)hb * 8, v[u]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const uint32_t hb = base + u * 32u + lane;
+      float a = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[u][j]));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+      const float sv = a / kE2M1Max;
+      const uint32_t s = f32_to_ue8m0_rp(sv);
+      const float k = 1.0f / ue8m0_to_f32(s);
+      float q[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) q[j] = v[u][j] * k;
+      const uint32_t w = f32x8_to_e2m1x8(q);
+      if (hb < n_half) {
+        codes[hb] = w;
+        if ((lane & 3u) == 0) so.store(hb >> 2, s);
+      }
+    }
+  }
+  zero_scale_padding(so, rows);
+}
+
 // Scale byte of block `block` from a LINEAR or 128x4-tile buffer.
 struct ScaleIn {
   const uint8_t* p;
@@ -326,6 +375,23 @@ __global__ void __launch_bounds__(kEwThreads) k_mxfp8_dequantize(
       v[j] = a[j] * sc;
       v[4 + j] = b[j] * sc;
     }
+    store8<T>(out + (size_t)hb * 8, v);
+  }
+}
+
+// MXFP4 dequantize (fp_dequantize, e8m0 branch with 4-bit codes):
+//   w_hat = T(e2m1(q) * 2^(s-127)).
+template <typename T>
+__global__ void __launch_bounds__(kEwThreads) k_mxfp4_dequantize(
+    const uint32_t* __restrict__ codes, ScaleIn si, uint32_t n_half, T* __restrict__ out) {
+  const uint32_t tid = blockIdx.x * blockDim.x + threadIdx.x, nthr = gridDim.x * blockDim.x;
+  for (uint32_t hb = tid; hb < n_half; hb += nthr) {
+    const uint32_t w = __ldg(codes + hb);
+    const float sc = ue8m0_to_f32(si.load(hb >> 2));
+    float v[8];
+    e2m1x8_to_f32(w, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = v[j] * sc;
     store8<T>(out + (size_t)hb * 8, v);
   }
 }

@@ -22,7 +22,7 @@ LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_DEVICE_INDEX = range(6)
 DT = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
 LAYOUT = {"linear": 0, "swizzled": 1}
-MODE = {"nvfp4": 0, "mxfp8": 1}
+MODE = {"nvfp4": 0, "mxfp8": 1, "mxfp4": 2}
 
 # (name, restype, argtypes) of every symbol declared in include/nvfp4.h
 _P, _I64, _I, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -37,6 +37,8 @@ SIGNATURES = [
     ("nvfp4_dequantize", _I, [_P, _P, _I, _I64, _I64, _P, _P, _I, _P]),
     ("mxfp8_quantize", _I, [_P, _I, _I64, _I64, _P, _P, _I, _P]),
     ("mxfp8_dequantize", _I, [_P, _P, _I, _I64, _I64, _P, _I, _P]),
+    ("mxfp4_quantize", _I, [_P, _I, _I64, _I64, _P, _P, _I, _P]),
+    ("mxfp4_dequantize", _I, [_P, _P, _I, _I64, _I64, _P, _I, _P]),
     ("nvfp4_swizzle_scales", _I, [_P, _I64, _I64, _P, _P]),
     ("qqmm", _I, [_I, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
     ("qmv", _I, [_P, _I, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
@@ -168,6 +170,28 @@ def mxfp8_quantize(x: torch.Tensor, layout: str = "linear", codes=None, scales=N
     _check(lib().mxfp8_quantize(_ptr(x), DT[x.dtype], rows, K, _ptr(codes), _ptr(scales), LAYOUT[layout],
                                 _stream()))
     return codes, scales
+
+
+def mxfp4_quantize(x: torch.Tensor, layout: str = "linear", codes=None, scales=None):
+    """(codes int32 [rows, K/8], e8m0 scales uint8) of a 2-D x, 32-element blocks."""
+    _need_cuda(x)
+    rows, K = x.shape
+    if codes is None:
+        codes = torch.empty(rows, K // 8, dtype=torch.int32, device=x.device)
+    if scales is None:
+        scales = torch.empty(scale_shape(rows, K // 32, layout), dtype=torch.uint8, device=x.device)
+    _check(lib().mxfp4_quantize(_ptr(x), DT[x.dtype], rows, K, _ptr(codes), _ptr(scales), LAYOUT[layout],
+                                _stream()))
+    return codes, scales
+
+
+def mxfp4_dequantize(codes, scales, layout: str = "linear", dtype=torch.bfloat16) -> torch.Tensor:
+    _need_cuda(codes, scales)
+    rows, K = codes.shape[0], codes.shape[1] * 8
+    out = torch.empty(rows, K, dtype=dtype, device=codes.device)
+    _check(lib().mxfp4_dequantize(_ptr(codes), _ptr(scales), LAYOUT[layout], rows, K, _ptr(out), DT[dtype],
+                                  _stream()))
+    return out
 
 
 def mxfp8_dequantize(codes, scales, layout: str = "linear", dtype=torch.bfloat16) -> torch.Tensor:

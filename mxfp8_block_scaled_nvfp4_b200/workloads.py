@@ -36,6 +36,8 @@ WORKLOADS = {
     "moe": {"T": 4096, "E": 64, "topk": 8, "N": 1408, "K": 2048, "dtype": torch.bfloat16,
             "seeds": (5, 6, 7)},
     "mxfp8": {"M": 8192, "N": 8192, "K": 8192, "dtype": torch.bfloat16, "seeds": (8, 9)},
+    # the mxfp8 GEMM's operands quantized in the MXFP4 mode instead
+    "mxfp4": {"M": 8192, "N": 8192, "K": 8192, "dtype": torch.bfloat16, "seeds": (8, 9)},
     "quant1g": {"R": 32768, "K": 16384, "dtype": torch.bfloat16, "seeds": (10,)},
     "prefill_bwd": {"M": 4096, "N": 4096, "K": 4096, "dtype": torch.bfloat16, "seeds": (3, 4, 11)},
 }
@@ -87,7 +89,7 @@ def make(name: str, device="cpu", scale_down: int = 1) -> dict:
         x = torch.randn(w["M"], w["K"], generator=g, device=device, dtype=torch.float32)
         W = torch.randn(w["N"], w["K"], generator=g, device=device, dtype=torch.float32)
         return {"x": x, "w": W}
-    if name in ("gemv", "prefill", "mxfp8"):
+    if name in ("gemv", "prefill", "mxfp8", "mxfp4"):
         M, N, K = w["M"], w["N"], w["K"]
         if sd > 1:
             M, N = max(1, M // sd), max(1, N // sd)
