@@ -385,18 +385,20 @@ def qmv(x, x_dt, g_x, w_codes, w_scales, g_w):
 # --------------------------------------------------------------------------
 # a10: gather_qmm (MoE) with per-expert global scales
 # --------------------------------------------------------------------------
-def gather_qmm(x, w_codes, w_scales, g, idx, tokens=None, x_dt="bf16"):
+def gather_qmm(x, w_codes, w_scales, g, idx, tokens=None, x_dt="bf16", transpose=True):
     """y[t, j, :] = x[t] . w_hat_e^T with e = idx[t, j] ([P3] "[Metal] global
     scale for qmm": the per-expert global scale multiplies each block scale
-    inside dequantization, before the cast to T).  w is [E, N, K] (transposed
-    weights); g is [E] or None.  float64 sum, one rounding to T.
-    ``tokens`` optionally selects a subset of tokens.
+    inside dequantization, before the cast to T).  transpose=True: w is
+    [E, N, K] (transposed weights, quantized along K); transpose=False
+    (the other layout the pull's tests loop over): w is [E, K, N], quantized
+    along N, and y[t, j, :] = x[t] . w_hat_e.  g is [E] or None.  float64
+    sum, one rounding to T.  ``tokens`` optionally selects a subset of tokens.
     Returns dict(y_ref float64 [T', topk, N], abs_ref, y raw)."""
     x = _raw(x, x_dt)
     idx = np.asarray(idx)
     tok = np.arange(x.shape[0]) if tokens is None else np.asarray(tokens)
     E = w_codes.shape[0]
-    N = w_codes.shape[1]
+    N = w_codes.shape[1] if transpose else w_codes.shape[2] * 8
     topk = idx.shape[1]
     xf = to_f64(np.ascontiguousarray(x[tok]), x_dt)
     y_ref = np.zeros((len(tok), topk, N), dtype=np.float64)
@@ -405,6 +407,8 @@ def gather_qmm(x, w_codes, w_scales, g, idx, tokens=None, x_dt="bf16"):
     for e in used:
         ge = None if g is None else float(g[e])
         wh = to_f64(nvfp4_dequantize(w_codes[e], w_scales[e], ge, x_dt), x_dt)
+        if not transpose:
+            wh = wh.T  # [K, N] decoded along its rows (N): the matmul takes w_hat itself
         ti, ji = np.nonzero(idx[tok] == e)
         y_ref[ti, ji] = xf[ti] @ wh.T
         abs_ref[ti, ji] = np.abs(xf[ti]) @ np.abs(wh).T
