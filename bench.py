@@ -13,6 +13,7 @@ One step = one pass over every row of the hot path, each on its workload
   prefill_bwd f1    qqmm backward: amax + quantize of the gradient, column-wise
                     quantizes of W, x and the gradient, dx and dw GEMMs 4096^3
   moe       a10     gather_qmm: 64 experts [1408,2048], 4096 tokens, top-8 -> bf16
+  moe_kn    f2      gather_qmm with transpose=False: the moe row's weights stored [E, K, N]
   moe_decode f2     gather_qmm decode (gather_qmv): the same experts, 4 tokens, top-8
   mxfp8     a11-a12 mxfp8 quantize x2 + FP8 GEMM 8192^3 -> bf16
   mxfp4     f3      mxfp4 quantize x2 + FP4 GEMM 8192^3 (mxfp4 mode) -> bf16
@@ -388,6 +389,46 @@ class Moe(Row):
                              "hbm_frac": self.bytes / t / 1e6 / peaks["hbm_gbs"], "algorithmic_bytes": self.bytes}}
 
 
+class MoeKN(Moe):
+    """The MoE config with the expert weights stored [E, K, N] and quantized
+    along N (gather_qmm with transpose=False): same tokens, routing and
+    per-expert global scales as the moe row."""
+    name, launches = "moe_kn", 3
+
+    def setup(self):
+        d = self.wl.make("moe", device=self.dev)
+        self.x, w, self.idx = d["x"], d["w"], d["idx"]
+        E, N, K = w.shape
+        self.E, self.N, self.K = E, N, K
+        wt = w.transpose(1, 2).contiguous()  # [E, K, N]
+        del w
+        self.g = torch.stack([self.nv.amax(wt[e]) for e in range(E)]).view(E)
+        wc, ws = [], []
+        for e in range(E):
+            c, s = self.nv.nvfp4_quantize(wt[e], self.g[e:e + 1], "linear")
+            wc.append(c)
+            ws.append(s)
+        self.wc, self.ws = torch.stack(wc), torch.stack(ws)
+        del wt, wc, ws
+        T, topk = self.idx.shape
+        self.T, self.topk = T, topk
+        self.ws_buf = torch.empty(self.nv.gather_qmm_workspace_size(T, topk, E), dtype=torch.uint8, device=self.dev)
+        self.y = torch.empty(T, topk, N, dtype=torch.bfloat16, device=self.dev)
+        self.flop = 2 * T * topk * N * K
+        self.bytes = self.wc.numel() * 4 + self.ws.numel() + self.x.numel() * 2 + self.y.numel() * 2 + self.idx.numel() * 4
+        self.nv.gather_qmm(self.x[:16], self.wc, self.ws, self.g, self.idx[:16].contiguous(), transpose=False)
+
+    def calls(self):
+        return [("gather_qmm", lambda: self.nv.gather_qmm(self.x, self.wc, self.ws, self.g, self.idx,
+                                                          self.ws_buf, self.y, transpose=False))]
+
+    def report(self, ms, row_ms, peaks):
+        r = super().report(ms, row_ms, peaks)
+        r["metric"] = "gather_qmm (transpose=False) TFLOP/s"
+        r["roofline"]["kernel"] = "gather_qmm (kn)"
+        return r
+
+
 class MoeDecode(Row):
     """Decode-time MoE (the gather_qmv path): the MoE config's 64 experts
     [1408, 2048], 4 tokens routed top-8 (tokens 0-3 of the MoE routing)."""
@@ -501,7 +542,7 @@ class Mxfp4(Row):
                              "peak_note": "measured bf16 burst x 4 (nominal fp4:bf16 ratio)"}}
 
 
-ROWS = [Quant1G, Gemv, Dequant, Prefill, PrefillBwd, Moe, MoeDecode, Mxfp8, Mxfp4]
+ROWS = [Quant1G, Gemv, Dequant, Prefill, PrefillBwd, Moe, MoeKN, MoeDecode, Mxfp8, Mxfp4]
 
 
 # ---------------------------------------------------------------------------

@@ -219,6 +219,18 @@ NVFP4_API nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const 
                         int64_t E, int64_t N, int64_t K, void* y, void* workspace,
                         size_t workspace_bytes, nvfp4_stream_t stream);
 
+/* f2 -- gather_qmm with transpose=False ([P3] tests loop over both layouts):
+ * the weights stored [K, N] per expert and quantized along N.
+ *   y[t, j, :] = x[t, :] . w_hat_e,  e = idx[t, j],
+ *   w_hat_e[k, n] = bf16(e2m1(q[e,k,n]) * (f8(s[e,k,n/16]) * g[e] / 2688)).
+ * x [T, K] bf16; w_codes [E, K, N/8]; w_scales LINEAR [E, K, N/16]; g, idx,
+ * y, workspace and errors as gather_qmm.  K % 64 == 0, N % 32 == 0.  Every
+ * T runs the tensor-core kernel (no separate decode path for this layout). */
+NVFP4_API nvfp4_status gather_qmm_kn(const void* x, const uint32_t* w_codes, const uint8_t* w_scales,
+                        const float* g, const int32_t* idx, int64_t T, int64_t topk,
+                        int64_t E, int64_t N, int64_t K, void* y, void* workspace,
+                        size_t workspace_bytes, nvfp4_stream_t stream);
+
 NVFP4_API size_t gather_qmm_workspace_size(int64_t T, int64_t topk, int64_t E);
 
 /* gather_qmm without a workspace argument; the pages have no counterpart of

@@ -294,6 +294,12 @@ __device__ __forceinline__ void unit_coords(uint32_t u, uint32_t n_tiles_n, uint
   n0 = (u - tile * n_tiles_n) * (uint32_t)BN;
 }
 
+// KN = false: w is [E, N, K] (quantized along K, the transposed layout);
+// KN = true: w is [E, K, N] (quantized along N).  With KN the bf16 weight
+// stage is written N-major (the codes' own order) and the MMA reads B as an
+// MN-major operand: 128-byte-swizzled atoms of 8 k-rows x 64 n, LBO 1 KiB
+// between the four atoms along N, SBO 4 KiB between 8-row groups along K.
+template <bool KN>
 __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant__ CUtensorMap tmap_x,
                                                            const __grid_constant__ CUtensorMap tmap_w, Args a) {
   using namespace tc;
@@ -386,7 +392,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
     for (uint32_t u = blockIdx.x; u < units; u += gridDim.x) {
       uint32_t tile, n0;
       unit_coords(u, (uint32_t)a.n_tiles_n, tile, n0);
-      const int wrow = a.ws.tile_expert[tile] * a.N + (int)n0;
+      const int wrow = KN ? a.ws.tile_expert[tile] * a.K : a.ws.tile_expert[tile] * a.N + (int)n0;
       bool ok = true;
       for (uint32_t kb = 0; kb < kb_count; ++kb, ++it) {
         const uint32_t s = it % RS;
@@ -398,7 +404,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
         if (leader) {
           const uint32_t bar = smem_u32(&r_full[s]);
           mbar_expect_tx(bar, R_STAGE);
-          tma_load_2d(sbase + SMEM_R + s * R_STAGE, &tmap_w, (int)(kb * 32u), wrow, bar);
+          if (KN)  // 64 k-rows x 256 codes along n
+            tma_load_2d(sbase + SMEM_R + s * R_STAGE, &tmap_w, (int)(n0 / 2u), wrow + (int)(kb * 64u), bar);
+          else     // 256 n-rows x 64 codes along k
+            tma_load_2d(sbase + SMEM_R + s * R_STAGE, &tmap_w, (int)(kb * 32u), wrow, bar);
         }
         __syncwarp();
       }
@@ -414,8 +423,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
   } else if (warp == W_MMA) {
     // ------------------------------------------------------------ MMA issuer
     const bool leader = elect_one();
-    const uint32_t idesc = f16_idesc();
-    const uint64_t x_base = kmajor_sw128_desc(sbase + SMEM_X), w_base = kmajor_sw128_desc(sbase + SMEM_W);
+    const uint32_t idesc = f16_idesc() | (KN ? (1u << 16) : 0u);  // B MN-major for KN
+    const uint64_t x_base = kmajor_sw128_desc(sbase + SMEM_X);
+    const uint64_t w_base = KN ? smem_desc(sbase + SMEM_W, 1024u, 4096u, 2u /* 128B swizzle */) : kmajor_sw128_desc(sbase + SMEM_W);
+    constexpr uint32_t kWStep = KN ? (8192u >> 4) : 2u;  // descriptor advance per K = 16: two 8-row groups, or 32 B
     const uint32_t x_hi = (uint32_t)(x_base >> 32), w_hi = (uint32_t)(w_base >> 32);
     auto mk = [](uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; };
     uint32_t xit = 0, wit = 0, ui = 0;
@@ -443,13 +454,73 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
           for (uint32_t hh = 0; hh < 2; ++hh)
 #pragma unroll
             for (uint32_t j = 0; j < 4; ++j)
-              mma_bf16(tmem + hh * 256u, mk(xl + hh * ((MMA_M * 128) >> 4) + 2 * j, x_hi), mk(wl + 2 * j, w_hi), idesc,
-                       (kb | j) != 0);
+              mma_bf16(tmem + hh * 256u, mk(xl + hh * ((MMA_M * 128) >> 4) + 2 * j, x_hi), mk(wl + kWStep * j, w_hi),
+                       idesc, (kb | j) != 0);
           mma_commit(smem_u32(&x_empty[xs]));
           mma_commit(smem_u32(&w_empty[ws]));
           if (kb + 1 == kb_count) mma_commit(smem_u32(&acc_full));
         }
         __syncwarp();
+      }
+    }
+    if (!ok && lane == 0) abort_flag = 1;
+  } else if (KN && warp >= W_DEQ) {
+    // ------------------------------------------------------------ dequantize (w stored [K, N])
+    // thread (warp w, lane o) takes code word o (n = n0 + 8o .. +7) of k-rows
+    // w, w + 16, w + 32, w + 48 of each k-step: one 16-byte N-major store per
+    // word, conflict-free (the 8 lanes of a store phase hit 8 chunks of one
+    // 128-byte row)
+    const uint32_t o = lane, kr = (uint32_t)(warp - W_DEQ);
+    const uint32_t nb16 = (uint32_t)a.N / 16u;
+    uint32_t rit = 0, wit = 0;
+    bool ok = true;
+    for (uint32_t u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      uint32_t tile, n0;
+      unit_coords(u, (uint32_t)a.n_tiles_n, tile, n0);
+      const int e = a.ws.tile_expert[tile];
+      const bool valid = n0 + 8u * o < (uint32_t)a.N;  // N % 16 == 0: whole words valid or not
+      const float d = a.g ? __ldg(a.g + e) / kGlobalEncode : 1.0f;
+      // scale byte of (k-row k of the expert, this word's 16-block)
+      const uint8_t* scol = a.wsc + (size_t)e * a.K * nb16 + (n0 + 8u * o) / 16u;
+      auto load_sc = [&](uint32_t kb, uint32_t (&sc)[4]) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          sc[i] = (valid && kb < kb_count) ? __ldg(scol + (size_t)(kb * 64u + kr + 16u * i) * nb16) : 0u;
+      };
+      uint32_t sc[4];
+      load_sc(0, sc);
+      for (uint32_t kb = 0; kb < kb_count; ++kb, ++rit, ++wit) {
+        const uint32_t rs = rit % RS, ws = wit % WS;
+        uint32_t sc_next[4];
+        load_sc(kb + 1, sc_next);  // next k-step's scales in flight
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&r_full[rs]), (rit / RS) & 1u) &&
+                                         mbar_wait(smem_u32(&w_empty[ws]), ((wit / WS) & 1u) ^ 1u)) ||
+            *(volatile int*)&abort_flag) {
+          ok = false;
+          break;
+        }
+        uint32_t words[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          words[i] = *reinterpret_cast<const uint32_t*>(smem + SMEM_R + rs * R_STAGE + (kr + 16u * i) * 128u + 4u * o);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&r_empty[rs]));  // codes are in registers
+        const uint32_t dst = sbase + SMEM_W + ws * W_STAGE;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t k = kr + 16u * i;
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (valid) v = dequant8_bf16(words[i], e4m3_to_f32(sc[i]) * d);
+          const uint32_t off = (k >> 3) * 4096u + (o >> 3) * 1024u + (k & 7u) * 128u + (((o & 7u) ^ (k & 7u)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + off), "r"(v.x), "r"(v.y), "r"(v.z),
+                       "r"(v.w)
+                       : "memory");
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // st.shared visible to tcgen05.mma
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&w_full[ws]));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sc[i] = sc_next[i];
       }
     }
     if (!ok && lane == 0) abort_flag = 1;
@@ -691,7 +762,7 @@ __global__ void __launch_bounds__(QV_THREADS) k_gather_qmv(const __nv_bfloat16* 
 // x [T, K] bf16: box 64 x 1 rows (tile::gather4 takes four rows of it),
 // 128-byte swizzle.  Codes [E*N rows, K/2 bytes]: box 32 B x 256 rows.
 inline bool make_maps(CUtensorMap* mx, CUtensorMap* mw, const void* x, const uint32_t* wc, uint64_t T, uint64_t K,
-                      uint64_t EN) {
+                      uint64_t EN, bool kn = false, uint64_t E = 0, uint64_t N = 0) {
   auto fn = tc::encode_fn();
   if (!fn) return false;
   {
@@ -703,6 +774,15 @@ inline bool make_maps(CUtensorMap* mx, CUtensorMap* mw, const void* x, const uin
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return false;
+  }
+  if (kn) {  // codes [E * K rows, N/2 bytes], box 128 B (256 n) x 64 k-rows
+    cuuint64_t dims[2] = {N / 2, E * K};
+    cuuint64_t strides[1] = {N / 2};
+    cuuint32_t box[2] = {128, (cuuint32_t)BK};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint32_t*>(wc), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
   }
   {
     cuuint64_t dims[2] = {K / 2, EN};
@@ -724,7 +804,7 @@ inline size_t gather_workspace_bytes(int64_t T, int64_t topk, int64_t E) { retur
 inline nvfp4_status gather_qmm_launch(const void* x, const uint32_t* w_codes, const uint8_t* w_scales, const float* g,
                                       const int32_t* idx, int64_t T, int64_t topk, int64_t E, int64_t N, int64_t K,
                                       void* y, void* workspace, int sm_count, cudaStream_t stream, char* msg,
-                                      size_t msg_len) {
+                                      size_t msg_len, bool kn = false) {
   using namespace gq;
   if (E > MAX_E) {
     snprintf(msg, msg_len, "[gather_qmm] at most %d experts", MAX_E);
@@ -733,7 +813,7 @@ inline nvfp4_status gather_qmm_launch(const void* x, const uint32_t* w_codes, co
   const int64_t P = T * topk;
   Workspace ws = carve(workspace, P, E);
   CUtensorMap mx, mw;
-  if (!make_maps(&mx, &mw, x, w_codes, (uint64_t)T, (uint64_t)K, (uint64_t)(E * N))) {
+  if (!make_maps(&mx, &mw, x, w_codes, (uint64_t)T, (uint64_t)K, (uint64_t)(E * N), kn, (uint64_t)E, (uint64_t)N)) {
     snprintf(msg, msg_len, "[gather_qmm] cuTensorMapEncodeTiled failed");
     return NVFP4_ERR_CUDA;
   }
@@ -744,7 +824,7 @@ inline nvfp4_status gather_qmm_launch(const void* x, const uint32_t* w_codes, co
     err = cudaGetLastError();
   }
   const size_t qv_smem = (size_t)kQmvPairs * (size_t)K * sizeof(float);
-  if (err == cudaSuccess && T <= kQmvTokens && qv_smem <= 200u * 1024u) {
+  if (err == cudaSuccess && !kn && T <= kQmvTokens && qv_smem <= 200u * 1024u) {
     // decode: gather_qmv
     err = cudaFuncSetAttribute(k_gather_qmv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qv_smem);
     if (err == cudaSuccess) {
@@ -769,7 +849,8 @@ inline nvfp4_status gather_qmm_launch(const void* x, const uint32_t* w_codes, co
     msg[0] = '\0';
     return NVFP4_OK;
   }
-  if (err == cudaSuccess) err = cudaFuncSetAttribute(k_gather_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+  auto kern = kn ? k_gather_mma<true> : k_gather_mma<false>;
+  if (err == cudaSuccess) err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
   if (err == cudaSuccess) {
     Args a;
     a.wsc = w_scales;
@@ -782,7 +863,7 @@ inline nvfp4_status gather_qmm_launch(const void* x, const uint32_t* w_codes, co
     a.n_tiles_n = (int)((N + BN - 1) / BN);
     const int64_t max_units = max_tiles(P, E) * a.n_tiles_n;
     const unsigned grid = (unsigned)(max_units < sm_count ? max_units : sm_count);
-    k_gather_mma<<<grid, THREADS, SMEM_ALLOC, stream>>>(mx, mw, a);
+    kern<<<grid, THREADS, SMEM_ALLOC, stream>>>(mx, mw, a);
     err = cudaGetLastError();
   }
   if (err != cudaSuccess) {

@@ -458,6 +458,30 @@ nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const uint8_t* w
                            sizeof(t_msg));
 }
 
+nvfp4_status gather_qmm_kn(const void* x, const uint32_t* w_codes, const uint8_t* w_scales, const float* g,
+                        const int32_t* idx, int64_t T, int64_t topk, int64_t E, int64_t N, int64_t K, void* y,
+                        void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+  if (T < 0 || topk < 1 || E < 1 || N < 0 || K < 0 || T * topk > (1 << 30) || E > (1 << 20))
+    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm_kn] bad shape");
+  if (K % 64 != 0 || N % 32 != 0)
+    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm_kn] K must be a multiple of 64 and N of 32 (K=%lld N=%lld)",
+                (long long)K, (long long)N);
+  if (workspace_bytes < gather_workspace_bytes(T, topk, E))
+    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm_kn] workspace too small: %zu < %zu", workspace_bytes,
+                gather_workspace_bytes(T, topk, E));
+  if (T * N > 0 && (!x || !w_codes || !w_scales || !idx || !y || !workspace))
+    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm_kn] null pointer");
+  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y) || !aligned16(workspace) ||
+      !aligned16(idx) || !aligned16(g))
+    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm_kn] tensor pointers must be 16-byte aligned");
+  DeviceInfo d;
+  nvfp4_status st = device_info("gather_qmm_kn", &d);
+  if (st != NVFP4_OK) return st;
+  if (T * N == 0) return ok();
+  return gather_qmm_launch(x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, workspace, d.sm_count, stream, t_msg,
+                           sizeof(t_msg), true);
+}
+
 // Device address of g_noalloc_scratch on the current device, resolved on
 // the first call per device (with that device current) and cached.
 static nvfp4_status noalloc_scratch(void** out) {

@@ -43,6 +43,7 @@ SIGNATURES = [
     ("qqmm", _I, [_I, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
     ("qmv", _I, [_P, _I, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     ("gather_qmm", _I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    ("gather_qmm_kn", _I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     ("gather_qmm_workspace_size", _SZ, [_I64, _I64, _I64]),
     ("gather_qmm_noalloc", _I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P]),
 ]
@@ -259,18 +260,22 @@ def gather_qmm_workspace_size(T: int, topk: int, E: int) -> int:
     return int(lib().gather_qmm_workspace_size(T, topk, E))
 
 
-def gather_qmm(x, w_codes, w_scales, g, idx, workspace=None, out=None) -> torch.Tensor:
-    """y [T, topk, N] bf16; w_codes [E, N, K/8], w_scales LINEAR [E, N, K/16]."""
+def gather_qmm(x, w_codes, w_scales, g, idx, workspace=None, out=None, transpose: bool = True) -> torch.Tensor:
+    """y [T, topk, N] bf16.  transpose=True: w_codes [E, N, K/8], w_scales
+    LINEAR [E, N, K/16] (y = x . w_hat^T); transpose=False: w_codes
+    [E, K, N/8], w_scales LINEAR [E, K, N/16] (y = x . w_hat)."""
     _need_cuda(x, w_codes, w_scales, g, idx, workspace)
     T, K = x.shape
     topk = idx.shape[1]
-    E, N = w_codes.shape[0], w_codes.shape[1]
+    E = w_codes.shape[0]
+    N = w_codes.shape[1] if transpose else w_codes.shape[2] * 8
     if workspace is None:
         workspace = torch.empty(gather_qmm_workspace_size(T, topk, E), dtype=torch.uint8, device=x.device)
     if out is None:
         out = torch.empty(T, topk, N, dtype=torch.bfloat16, device=x.device)
-    _check(lib().gather_qmm(_ptr(x), _ptr(w_codes), _ptr(w_scales), _ptr(g), _ptr(idx), T, topk, E, N, K,
-                            _ptr(out), _ptr(workspace), workspace.numel(), _stream()))
+    fn = lib().gather_qmm if transpose else lib().gather_qmm_kn
+    _check(fn(_ptr(x), _ptr(w_codes), _ptr(w_scales), _ptr(g), _ptr(idx), T, topk, E, N, K,
+              _ptr(out), _ptr(workspace), workspace.numel(), _stream()))
     return out
 
 
