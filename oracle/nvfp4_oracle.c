@@ -490,6 +490,103 @@ void orc_mxfp4_decode_exact(const uint32_t* codes, const uint8_t* scales,
 }
 
 /* ------------------------------------------------------------------------ */
+/* 8c. Stochastic rounding of the codes (the pages reserve it: [P2]           */
+/*    fp_quantize_rowwise<..., USE_SR> with `rbits` "reserved for future     */
+/*    use"; the reading taken here is the plain one):                        */
+/*    the block scale s is computed exactly as in section 5; each scaled     */
+/*    value t = x * k (fp32) goes to one of the two e2m1 magnitudes lo <= |t| */
+/*    <= hi around it, up with probability (|t| - lo) / (hi - lo), decided by */
+/*    32 random bits r: up iff fp32(r) * 2^-32 < (|t| - lo) / (hi - lo)      */
+/*    (both sides of the comparison are exact fp32 values; the difference is  */
+/*    exact by Sterbenz, the division by a power of two).  |t| >= 6 gives 6,  */
+/*    values on the grid are kept, the sign is kept (as in section 5).        */
+/*    r for element i of the flat [rows, K] array: word i % 4 of              */
+/*    Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers:    */
+/*    as easy as 1, 2, 3", SC 2011) with counter (i / 4 low, i / 4 high, 0,   */
+/*    0) and key (seed low, seed high).                                      */
+/* ------------------------------------------------------------------------ */
+static void philox_round(uint32_t c[4], const uint32_t k[2]) {
+  const uint64_t p0 = (uint64_t)0xD2511F53u * c[0];
+  const uint64_t p1 = (uint64_t)0xCD9E8D57u * c[2];
+  const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+  const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+  const uint32_t n0 = hi1 ^ c[1] ^ k[0], n1 = lo1, n2 = hi0 ^ c[3] ^ k[1], n3 = lo0;
+  c[0] = n0; c[1] = n1; c[2] = n2; c[3] = n3;
+}
+
+void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
+  uint32_t c[4] = {ctr[0], ctr[1], ctr[2], ctr[3]};
+  uint32_t k[2] = {key[0], key[1]};
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) { k[0] += 0x9E3779B9u; k[1] += 0xBB67AE85u; }
+    philox_round(c, k);
+  }
+  for (int i = 0; i < 4; ++i) out[i] = c[i];
+}
+
+uint32_t orc_sr_bits(uint64_t seed, uint64_t i) {
+  const uint64_t q = i >> 2;
+  const uint32_t ctr[4] = {(uint32_t)q, (uint32_t)(q >> 32), 0u, 0u};
+  const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  uint32_t out[4];
+  orc_philox4x32_10(ctr, key, out);
+  return out[i & 3u];
+}
+
+int orc_e2m1_sr_satfinite(float t, uint32_t r) {
+  static const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  const int neg = signbit(t) ? 8 : 0;
+  const float a = fabsf(t);
+  int m;
+  if (a >= 6.0f) {
+    m = 7;
+  } else {
+    int lo = 0;
+    while (lo < 7 && mag[lo + 1] <= a) ++lo;  /* mag[lo] <= a < mag[lo + 1] */
+    if (a == mag[lo]) {
+      m = lo;
+    } else {
+      const float frac = (a - mag[lo]) / (mag[lo + 1] - mag[lo]);
+      const float u = (float)r * 0x1p-32f;
+      m = u < frac ? lo + 1 : lo;
+    }
+  }
+  return neg | m;
+}
+
+void orc_nvfp4_quantize_sr(const void* x, int dt, int64_t rows, int64_t K, const float* g, uint64_t seed,
+                           uint32_t* codes, uint8_t* scales) {
+  const float E = encode_factor(g);
+  const int64_t nb = K / 16;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t b = 0; b < nb; ++b) {
+      float xv[16];
+      float a = 0.0f;
+      for (int i = 0; i < 16; ++i) {
+        xv[i] = (float)orc_load(x, dt, r * K + b * 16 + i);
+        if (fabsf(xv[i]) > a) a = fabsf(xv[i]);
+      }
+      float t = a / 6.0f;
+      t = t * E;
+      int s = orc_e4m3_rne_satfinite(t);
+      scales[r * nb + b] = (uint8_t)s;
+      float fs = (float)orc_e4m3_value(s);
+      uint32_t w[2] = {0, 0};
+      if (fs != 0.0f) {
+        float k = E / fs;
+        for (int i = 0; i < 16; ++i) {
+          const uint64_t idx = (uint64_t)(r * K + b * 16 + i);
+          uint32_t q = (uint32_t)orc_e2m1_sr_satfinite(xv[i] * k, orc_sr_bits(seed, idx));
+          w[i / 8] |= q << (4 * (i % 8));
+        }
+      }
+      codes[(r * K + b * 16) / 8] = w[0];
+      codes[(r * K + b * 16) / 8 + 1] = w[1];
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
 /* 9. Scale layout for the block-scaled MMA ([P5] qqmm_utils.cu comment:     */
 /*    tmp = s.reshape(rb, 4, 32, cb, 4); tmp.transpose(0, 3, 2, 1, 4), and   */
 /*    its worked index table; [P1] pad_and_swizzle_scales: pad to 128-row x  */

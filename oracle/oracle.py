@@ -87,6 +87,10 @@ def _L():
                 "orc_mxfp8_dequantize": (None, [P, P, I64, I64, P, I]),
                 "orc_mxfp8_decode_exact": (None, [P, P, I64, I64, P]),
                 "orc_mxfp4_quantize": (None, [P, I, I64, I64, P, P]),
+                "orc_philox4x32_10": (None, [P, P, P]),
+                "orc_sr_bits": (ctypes.c_uint32, [ctypes.c_uint64, ctypes.c_uint64]),
+                "orc_e2m1_sr_satfinite": (I, [ctypes.c_float, ctypes.c_uint32]),
+                "orc_nvfp4_quantize_sr": (None, [P, I, I64, I64, P, ctypes.c_uint64, P, P]),
                 "orc_mxfp4_dequantize": (None, [P, P, I64, I64, P, I]),
                 "orc_mxfp4_decode_exact": (None, [P, P, I64, I64, P]),
                 "orc_swizzle_scales": (None, [P, I64, I64, P]),
@@ -282,6 +286,40 @@ def mxfp8_decode_exact(codes, scales) -> np.ndarray:
     out = np.empty((rows, K), dtype=np.float64)
     _L().orc_mxfp8_decode_exact(_p(codes), _p(scales), rows, K, _p(out))
     return out
+
+
+# --------------------------------------------------------------------------
+# NVFP4 quantize with stochastic rounding of the codes
+# --------------------------------------------------------------------------
+def philox4x32_10(ctr, key):
+    """Philox4x32-10 (Salmon et al., SC 2011): 4 counter words, 2 key words."""
+    c = np.ascontiguousarray(ctr, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    out = np.zeros(4, dtype=np.uint32)
+    _L().orc_philox4x32_10(_p(c), _p(k), _p(out))
+    return out
+
+
+def sr_bits(seed: int, i: int) -> int:
+    return int(_L().orc_sr_bits(seed, i))
+
+
+def e2m1_sr(t: float, r: int) -> int:
+    return int(_L().orc_e2m1_sr_satfinite(t, r))
+
+
+def nvfp4_quantize_sr(x: np.ndarray, dt: str, g: float | None = None, seed: int = 0):
+    """NVFP4 quantize whose codes are rounded stochastically (the scales as in
+    nvfp4_quantize; random bits from Philox4x32-10 keyed by ``seed``, counter
+    = flat element index / 4).  Returns (codes, scales LINEAR)."""
+    x = _raw(x, dt)
+    rows, K = x.shape
+    assert K % 16 == 0
+    codes = np.zeros((rows, K // 8), dtype=np.uint32)
+    scales = np.zeros((rows, K // 16), dtype=np.uint8)
+    gb, gp = _g(g)
+    _L().orc_nvfp4_quantize_sr(_p(x), DT[dt], rows, K, gp, seed, _p(codes), _p(scales))
+    return codes, scales
 
 
 # --------------------------------------------------------------------------
