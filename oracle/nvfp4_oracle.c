@@ -496,14 +496,16 @@ void orc_mxfp4_decode_exact(const uint32_t* codes, const uint8_t* scales,
 /*    the block scale s is computed exactly as in section 5; each scaled     */
 /*    value t = x * k (fp32) goes to one of the two e2m1 magnitudes lo <= |t| */
 /*    <= hi around it, up with probability (|t| - lo) / (hi - lo), decided by */
-/*    32 random bits r: up iff fp32(r) * 2^-32 < (|t| - lo) / (hi - lo)      */
-/*    (both sides of the comparison are exact fp32 values; the difference is  */
-/*    exact by Sterbenz, the division by a power of two).  |t| >= 6 gives 6,  */
-/*    values on the grid are kept, the sign is kept (as in section 5).        */
-/*    r for element i of the flat [rows, K] array: word i % 4 of              */
-/*    Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers:    */
-/*    as easy as 1, 2, 3", SC 2011) with counter (i / 4 low, i / 4 high, 0,   */
-/*    0) and key (seed low, seed high).                                      */
+/*    8 random bits b: up iff b * 2^-8 < (|t| - lo) / (hi - lo) (both sides   */
+/*    exact fp32 values; the difference is exact by Sterbenz, the division    */
+/*    by a power of two).  |t| >= 6 gives 6, values on the grid are kept,     */
+/*    the sign is kept (as in section 5).                                     */
+/*    Random bits: one 32-bit word per group of 4 consecutive elements, as    */
+/*    [P2] passes one `rbits` word to each 4-value conversion                 */
+/*    (scale_cvt_Tx4_to_fp4x4<T, USE_SR>); element i takes byte i % 4 of word */
+/*    i / 4, and word w is output w % 4 of Philox4x32-10 (Salmon, Moraes,     */
+/*    Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011) at  */
+/*    counter (w / 4 low, w / 4 high, 0, 0), key (seed low, seed high).       */
 /* ------------------------------------------------------------------------ */
 static void philox_round(uint32_t c[4], const uint32_t k[2]) {
   const uint64_t p0 = (uint64_t)0xD2511F53u * c[0];
@@ -525,12 +527,12 @@ void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t ou
 }
 
 uint32_t orc_sr_bits(uint64_t seed, uint64_t i) {
-  const uint64_t q = i >> 2;
+  const uint64_t w = i >> 2, q = w >> 2;
   const uint32_t ctr[4] = {(uint32_t)q, (uint32_t)(q >> 32), 0u, 0u};
   const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
   uint32_t out[4];
   orc_philox4x32_10(ctr, key, out);
-  return out[i & 3u];
+  return (out[w & 3u] >> (8u * (uint32_t)(i & 3u))) & 0xFFu;
 }
 
 int orc_e2m1_sr_satfinite(float t, uint32_t r) {
@@ -547,7 +549,7 @@ int orc_e2m1_sr_satfinite(float t, uint32_t r) {
       m = lo;
     } else {
       const float frac = (a - mag[lo]) / (mag[lo + 1] - mag[lo]);
-      const float u = (float)r * 0x1p-32f;
+      const float u = (float)r * 0x1p-8f;  /* r: 8 random bits */
       m = u < frac ? lo + 1 : lo;
     }
   }

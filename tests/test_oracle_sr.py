@@ -5,7 +5,9 @@ page 7, fp_quantize_rowwise<..., USE_SR> with rbits "reserved for future
 use"); the reading pinned here: scales as in the round-to-nearest quantizer,
 each scaled value rounded to one of its two e2m1 neighbours, up with
 probability equal to its relative position between them, decided by 32
-Philox4x32-10 bits per element."""
+random bits per element: byte i % 4 of one Philox4x32-10 word per group of
+4 elements (the pages pass one 32-bit rbits word to each 4-value conversion,
+scale_cvt_Tx4_to_fp4x4<T, USE_SR>)."""
 import os
 
 import numpy as np
@@ -38,17 +40,29 @@ def _val(code):
 
 @pytest.mark.parametrize("t,r,code", [
     (2.5, 0, 5),              # u = 0 < 1/2: up to 3
-    (2.5, 0xFFFFFFFF, 4),     # u = fp32(2^32 - 1) * 2^-32 = 1: down to 2
-    (5.0, 0x80000000, 6),     # u = 1/2, not < 1/2: down to 4
-    (5.0, 0x7FFFFF00, 7),     # u just below 1/2: up to 6
+    (2.5, 0xFF, 4),           # u = 255/256 >= 1/2: down to 2
+    (5.0, 0x80, 6),           # u = 1/2, not < 1/2: down to 4
+    (5.0, 0x7F, 7),           # u = 127/256 < 1/2: up to 6
+    (2.25, 0x3F, 5),          # frac 1/4: u = 63/256 < 1/4: up
+    (2.25, 0x40, 4),          # u = 1/4: down
     (-0.25, 0, 9),            # sign kept: -0.5
-    (-0.25, 0xFFFFFFFF, 8),   # -0 (code 8), as the round-to-nearest path keeps the sign
+    (-0.25, 0xFF, 8),         # -0 (code 8), as the round-to-nearest path keeps the sign
     (7.0, 0, 7),              # saturates at 6
-    (1.5, 12345, 3),          # on the grid: kept
+    (1.5, 123, 3),            # on the grid: kept
     (0.0, 0, 0),
 ])
 def test_sr_hand_cases(orc, t, r, code):
     assert orc.e2m1_sr(t, r) == code
+
+
+def test_sr_bits_are_bytes_of_philox_words(orc):
+    """Element i takes byte i % 4 of word i / 4; word w is output w % 4 of
+    Philox at counter w / 4 (16 elements per generator call)."""
+    seed = 0x0123456789ABCDEF
+    for i in [0, 1, 2, 3, 4, 7, 15, 16, 17, 1000003, 2**33 + 5]:
+        w = i // 4
+        out = orc.philox4x32_10([w // 4 & 0xFFFFFFFF, w // 4 >> 32, 0, 0], [seed & 0xFFFFFFFF, seed >> 32])
+        assert orc.sr_bits(seed, i) == (int(out[w % 4]) >> (8 * (i % 4))) & 0xFF
 
 
 def test_sr_only_neighbours_and_unbiased(orc):
