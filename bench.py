@@ -7,6 +7,7 @@ One step = one pass over every row of the hot path, each on its workload
 (seeded synthetic inputs, resident in HBM before timing):
 
   quant1g   a1-a4   amax + NVFP4 quantize (SWIZZLED scales) of bf16 [32768,16384]
+  quant1g_sr f4     the same quantize with stochastic rounding of the codes
   gemv      a1,a6-a7  amax(x) + qmv: x [1,4096] bf16, W [14336,4096] pre-quantized
   dequant   a5      NVFP4 dequantize of W [14336,4096] to bf16
   prefill   a1-a4,a8-a9  qqmm op: amax x2, quantize x2 (SWIZZLED), FP4 GEMM 4096^3 -> bf16
@@ -211,6 +212,23 @@ class Quant1G(Row):
                                        "frac": self.bytes_q / q / 1e6 / peaks["hbm_gbs"],
                                        "frac_of_8tbs": self.bytes_q / q / 1e6 / 8000.0,
                                        "algorithmic_bytes": self.bytes_q}}
+
+
+class Quant1GSR(Quant1G):
+    """The 1 GiB quantize with stochastic rounding of the codes (Philox4x32-10
+    bits per element, seed fixed): the same bytes as quant1g."""
+    name, launches = "quant1g_sr", 2
+
+    def calls(self):
+        return [("amax", lambda: self.nv.amax(self.x, self.g)),
+                ("quantize", lambda: self.nv.nvfp4_quantize_sr(self.x, self.g, 20261202, "swizzled", self.codes,
+                                                               self.scales))]
+
+    def report(self, ms, row_ms, peaks):
+        r = super().report(ms, row_ms, peaks)
+        r["metric"] = "nvfp4 quantize (stochastic rounding) GB/s"
+        r["roofline"]["kernel"] = "k_nvfp4_quantize<SR>"
+        return r
 
 
 class Gemv(Row):
@@ -542,7 +560,7 @@ class Mxfp4(Row):
                              "peak_note": "measured bf16 burst x 4 (nominal fp4:bf16 ratio)"}}
 
 
-ROWS = [Quant1G, Gemv, Dequant, Prefill, PrefillBwd, Moe, MoeKN, MoeDecode, Mxfp8, Mxfp4]
+ROWS = [Quant1G, Quant1GSR, Gemv, Dequant, Prefill, PrefillBwd, Moe, MoeKN, MoeDecode, Mxfp8, Mxfp4]
 
 
 # ---------------------------------------------------------------------------

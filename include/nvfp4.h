@@ -131,6 +131,21 @@ NVFP4_API nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, 
                                                  const float* g, uint32_t* codes, uint8_t* scales,
                                                  nvfp4_layout layout, nvfp4_stream_t stream);
 
+/* f4 -- NVFP4 quantize with stochastic rounding of the codes (the pages
+ * reserve it: [P2] fp_quantize_rowwise<..., USE_SR> with rbits "reserved for
+ * future use"; this library's reading).  Scales exactly as nvfp4_quantize;
+ * each scaled value t = x * E / f8(s) (fp32) goes to one of its two e2m1
+ * neighbours lo <= |t| <= hi: up iff b * 2^-8 < (|t| - lo) / (hi - lo)
+ * (|t| >= 6 gives 6, grid values are kept, the sign is kept), with b byte
+ * i % 4 of the 32-bit word w = i / 4 (one word per 4 values, as [P2] passes
+ * rbits to each 4-value conversion), word w being output w % 4 of
+ * Philox4x32-10 (Salmon et al., SC 2011) at counter (w / 4 as 64 bits, 0,
+ * 0) and key (seed), i = row * K + k.  Same arguments, layouts and errors
+ * as nvfp4_quantize, plus the 64-bit seed. */
+NVFP4_API nvfp4_status nvfp4_quantize_sr(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K,
+                                         const float* g, uint64_t seed, uint32_t* codes, uint8_t* scales,
+                                         nvfp4_layout layout, nvfp4_stream_t stream);
+
 /* a11 -- MXFP8 quantize ([P2] fp_quantize_rowwise with 8 bits and the e8m0
  * scale; group size 32, [P1] fp_quantize; the E8M0 scale is rounded up, [P3]
  * mlxcel note).  Per 32-block: s = ue8m0_round_up(amax / 448);

@@ -172,7 +172,8 @@ nvfp4_status nvfp4_amax(const void* x, nvfp4_dtype dt, int64_t n, float* g_out, 
 // kind: 0 NVFP4, 1 MXFP8, 2 MXFP4 (the two MX kinds use 32-element blocks)
 static nvfp4_status quantize_common(const char* tag, int kind, const void* x, nvfp4_dtype dt,
                                     int64_t rows, int64_t K, const float* g, uint32_t* codes,
-                                    uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
+                                    uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream,
+                                    bool sr = false, uint64_t seed = 0) {
   const int group = kind ? 32 : 16;
   if (!valid_dt(dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] dtype must be float32, float16 or bfloat16", tag);
   if (layout != NVFP4_LAYOUT_LINEAR && layout != NVFP4_LAYOUT_SWIZZLED)
@@ -207,7 +208,11 @@ static nvfp4_status quantize_common(const char* tag, int kind, const void* x, nv
       k_mxfp4_quantize<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, codes, so,
                                                            (uint32_t)rows);
     else
-      k_nvfp4_quantize<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, g, codes, so,
+      if (sr)
+        k_nvfp4_quantize<T, true><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, g, codes, so,
+                                                                   (uint32_t)rows, seed);
+      else
+        k_nvfp4_quantize<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, g, codes, so,
                                                            (uint32_t)rows);
   });
   return check_launch(tag);
@@ -216,6 +221,12 @@ static nvfp4_status quantize_common(const char* tag, int kind, const void* x, nv
 nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K, const float* g,
                             uint32_t* codes, uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
   return quantize_common("quantize", 0, x, dt, rows, K, g, codes, scales, layout, stream);
+}
+
+nvfp4_status nvfp4_quantize_sr(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K, const float* g,
+                               uint64_t seed, uint32_t* codes, uint8_t* scales, nvfp4_layout layout,
+                               nvfp4_stream_t stream) {
+  return quantize_common("quantize_sr", 0, x, dt, rows, K, g, codes, scales, layout, stream, true, seed);
 }
 
 nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, int64_t rows, int64_t cols, const float* g,

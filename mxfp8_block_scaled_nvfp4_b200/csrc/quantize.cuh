@@ -92,16 +92,55 @@ __device__ __forceinline__ void zero_scale_padding(const ScaleOut& so, uint32_t 
 }
 
 // ---------------------------------------------------------------------------
-// a2-a4: NVFP4 two-level quantize ("mlx 0.30.7.2 -> 0.30.7.6" diff, page 7,
-// fp_quantize.cu, fp_quantize_rowwise with global scale):
-//   E = 2688 / g (1 without g);  per 16-block: a = max|x|;
-//   s = e4m3_rne_satfinite((a / 6) * E);  k = E / f8(s);
-//   q_i = e2m1_rne_satfinite(x_i * k);  a block with f8(s) == 0 stores 0 codes.
+// f4: stochastic rounding of the NVFP4 codes.  The pages reserve it
+// ("mlx 0.30.7.2 -> 0.30.7.6" diff, page 7, fp_quantize_rowwise<..., USE_SR>
+// with rbits "reserved for future use"); this library's reading: the block
+// scale as in the round-to-nearest path, each scaled value t to one of its
+// two e2m1 neighbours lo <= |t| <= hi, up iff b * 2^-8 < (|t| - lo) / (hi -
+// lo) for 8 random bits b.  As the pages pass one 32-bit rbits word to each
+// 4-value conversion, element i of the flat [rows, K] array takes byte i % 4
+// of word i / 4, and word w is output w % 4 of Philox4x32-10 (Salmon,
+// Moraes, Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC
+// 2011) at counter (w / 4 as 64 bits, 0, 0), key (seed).
 // ---------------------------------------------------------------------------
-template <typename T>
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint64_t p0 = (uint64_t)0xD2511F53u * c.x, p1 = (uint64_t)0xCD9E8D57u * c.z;  // one wide multiply each
+    c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ k0, (uint32_t)p1, (uint32_t)(p0 >> 32) ^ c.w ^ k1, (uint32_t)p0);
+  }
+  return c;
+}
+
+// e2m1 code of t with stochastic rounding by the random byte r (sign kept,
+// saturating at 6), without branches: the grid has spacing 0.5 on [0, 2),
+// 1 on [2, 4) and 2 on [4, 6), so pos = (|t| - base) / spacing is exact in
+// fp32, floor(pos) indexes the lower neighbour and pos - floor(pos) is the
+// exact position between the two neighbours.
+__device__ __forceinline__ uint32_t e2m1_sr(float t, uint32_t r) {
+  const float a = fabsf(t);
+  const bool i0 = a < 2.0f, i1 = a < 4.0f;
+  const float base = i0 ? 0.0f : (i1 ? 2.0f : 4.0f);
+  const float inv_gap = i0 ? 2.0f : (i1 ? 1.0f : 0.5f);
+  const uint32_t code0 = i0 ? 0u : (i1 ? 4u : 6u);
+  const float pos = (a - base) * inv_gap;
+  const float fl = floorf(pos);
+  const float frac = pos - fl;
+  const float u = (float)r * 0x1p-8f;
+  uint32_t m = code0 + (uint32_t)fl + (u < frac ? 1u : 0u);
+  m = a >= 6.0f ? 7u : m;
+  return (signbit(t) ? 8u : 0u) | m;
+}
+
+// ---------------------------------------------------------------------------
+template <typename T, bool SR = false>
 __global__ void __launch_bounds__(kEwThreads) k_nvfp4_quantize(
     const T* __restrict__ x, uint32_t n_half, const float* __restrict__ g,
-    uint32_t* __restrict__ codes, ScaleOut so, uint32_t rows) {
+    uint32_t* __restrict__ codes, ScaleOut so, uint32_t rows, uint64_t seed = 0) {
   const float E = g ? kGlobalEncode / __ldg(g) : 1.0f;
   const uint32_t lane = threadIdx.x & 31u;
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -135,7 +174,18 @@ __global__ void __launch_bounds__(kEwThreads) k_nvfp4_quantize(
         float q[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) q[j] = v[u][j] * k;
-        w = f32x8_to_e2m1x8(q);
+        if constexpr (SR) {
+          // elements 8hb..8hb+7 use words 2hb and 2hb+1: outputs 2(hb%2) and
+          // 2(hb%2)+1 of the generator call at counter hb/2
+          const uint64_t c0 = (uint64_t)hb >> 1;
+          const uint4 r4 = philox4x32_10(make_uint4((uint32_t)c0, (uint32_t)(c0 >> 32), 0u, 0u), (uint32_t)seed,
+                                         (uint32_t)(seed >> 32));
+          const uint32_t wa = (hb & 1u) ? r4.z : r4.x, wb = (hb & 1u) ? r4.w : r4.y;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) w |= e2m1_sr(q[j], ((j < 4 ? wa : wb) >> (8 * (j & 3))) & 0xFFu) << (4 * j);
+        } else {
+          w = f32x8_to_e2m1x8(q);
+        }
       }
       if (hb < n_half) {
         codes[hb] = w;

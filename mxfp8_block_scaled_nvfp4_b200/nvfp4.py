@@ -35,6 +35,7 @@ SIGNATURES = [
     ("nvfp4_quantize", _I, [_P, _I, _I64, _I64, _P, _P, _P, _I, _P]),
     ("nvfp4_quantize_columnwise", _I, [_P, _I, _I64, _I64, _P, _P, _P, _I, _P]),
     ("nvfp4_dequantize", _I, [_P, _P, _I, _I64, _I64, _P, _P, _I, _P]),
+    ("nvfp4_quantize_sr", _I, [_P, _I, _I64, _I64, _P, ctypes.c_uint64, _P, _P, _I, _P]),
     ("mxfp8_quantize", _I, [_P, _I, _I64, _I64, _P, _P, _I, _P]),
     ("mxfp8_dequantize", _I, [_P, _P, _I, _I64, _I64, _P, _I, _P]),
     ("mxfp4_quantize", _I, [_P, _I, _I64, _I64, _P, _P, _I, _P]),
@@ -159,6 +160,21 @@ def nvfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, g: torch.Tensor 
     _check(lib().nvfp4_dequantize(_ptr(codes), _ptr(scales), LAYOUT[layout], rows, K, _ptr(g), _ptr(out),
                                   DT[dtype], _stream()))
     return out
+
+
+def nvfp4_quantize_sr(x: torch.Tensor, g: torch.Tensor | None = None, seed: int = 0, layout: str = "linear",
+                      codes: torch.Tensor | None = None, scales: torch.Tensor | None = None):
+    """nvfp4_quantize with stochastic rounding of the codes (Philox4x32-10
+    random bits keyed by ``seed``); scales as nvfp4_quantize."""
+    _need_cuda(x, g)
+    rows, K = x.shape
+    if codes is None:
+        codes = torch.empty(rows, K // 8, dtype=torch.int32, device=x.device)
+    if scales is None:
+        scales = torch.empty(scale_shape(rows, K // 16, layout), dtype=torch.uint8, device=x.device)
+    _check(lib().nvfp4_quantize_sr(_ptr(x), DT[x.dtype], rows, K, _ptr(g), seed, _ptr(codes), _ptr(scales),
+                                   LAYOUT[layout], _stream()))
+    return codes, scales
 
 
 def mxfp8_quantize(x: torch.Tensor, layout: str = "linear", codes=None, scales=None):
