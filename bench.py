@@ -59,7 +59,10 @@ L2_FLUSH_BYTES = 256 << 20
 NCU_TRAFFIC_BYTES = {
     "qqmm_sm100 (nvfp4)": 18958336 + 225536,    # profiles/qqmm_nvfp4_4096x4096x4096.md
     "k_qmv_tc": 33109760 + 0,                   # profiles/qmv_tc_gemv_14336x4096.md
-    "gather_qmm": 90273024 + 3263744,           # profiles/gather_qmm_moe_T4096_top8_E64_N1408_K2048.md
+    "gather_qmm": 126970112 + 56426240,         # profiles/gather_qmm_moe_T4096_top8_E64_N1408_K2048.md
+    "gather_qmm (kn)": 127318528 + 56494080,    # profiles/gather_qmm_kn_moe_T4096_top8_E64_N1408_K2048.md
+    "qqmm_sm100 (mxfp4)": 104143360 + 107496960,  # profiles/qqmm_mxfp4_8192x8192x8192.md
+    "k_nvfp4_quantize<SR>": 1120127232 + 319645184,  # profiles/quantize_sr_32768x16384.md
 }
 
 
