@@ -97,6 +97,43 @@ def test_gather_workspace_and_shape_checks(L):
     assert L.gather_qmm(A, A, A, A, A, 16, 2, 4, 64, 128, A, A, 0, None) == 1  # workspace
 
 
+def test_header_declares_the_next_rows():
+    syms = declared_symbols()
+    for sname in ["nvfp4_quantize_columnwise", "nvfp4_quantize_sr", "mxfp4_quantize", "mxfp4_dequantize",
+                  "mxfp8_dequantize", "gather_qmm_kn"]:
+        assert sname in syms
+
+
+def test_mxfp4_checks(L):
+    # 32-element groups
+    assert L.mxfp4_quantize(A, 2, 4, 48, A, A, 0, None) == 1
+    assert "group size 32" in msg(L)
+    assert L.mxfp4_dequantize(A, A, 0, 4, 48, A, 2, None) == 1
+    assert L.mxfp4_quantize(A, 7, 4, 64, A, A, 0, None) == 2  # dtype
+    # qqmm in mxfp4 mode takes no global scale; an unknown mode is rejected
+    assert L.qqmm(2, 128, 128, 256, A, A, A, A, A, A, A, 2, None) == 1
+    assert "only supported for 'nvfp4'" in msg(L)
+    assert L.qqmm(3, 128, 128, 256, A, A, A, A, None, None, A, 2, None) == 1
+    assert "'mxfp4'" in msg(L)
+
+
+def test_quantize_sr_checks(L):
+    assert L.nvfp4_quantize_sr(A, 2, 4, 24, None, 7, A, A, 0, None) == 1
+    assert "divisible by the quantization group size 16" in msg(L)
+    assert L.nvfp4_quantize_sr(A, 2, 4, 32, None, 7, A, A, 5, None) == 1  # layout
+    assert L.nvfp4_quantize_sr(A + 8, 2, 4, 32, None, 7, A, A, 0, None) == 1
+    assert "aligned" in msg(L)
+
+
+def test_gather_kn_checks(L):
+    ws = L.gather_qmm_workspace_size(64, 2, 4)
+    assert L.gather_qmm_kn(A, A, A, A, A, 64, 2, 4, 48, 128, A, A, ws, None) == 1  # N % 32
+    assert "N of 32" in msg(L)
+    assert L.gather_qmm_kn(A, A, A, A, A, 64, 2, 4, 64, 96, A, A, ws, None) == 1  # K % 64
+    assert L.gather_qmm_kn(A, A, A, A, A, 64, 2, 4, 64, 128, A, A, 0, None) == 1  # workspace
+    assert "workspace" in msg(L)
+
+
 def test_scale_bytes(L):
     assert L.nvfp4_scale_bytes(67, 16, 0) == 67 * 16
     assert L.nvfp4_scale_bytes(67, 16, 1) == 128 * 16
