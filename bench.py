@@ -299,9 +299,9 @@ class Gemv(Row):
     name, launches = "gemv", 2
     b2b_label = "qmv"
 
-    def b2b(self):  # six copies of the 33 MB weight (198 MB)
+    def b2b(self):  # six copies of the 33 MB weight (198 MB), two passes
         cps = [(self.wc.clone(), self.ws.clone()) for _ in range(6)]
-        return [lambda c=c: self.nv.qmv(self.x, c[0], c[1], self.g_x, self.g_w, self.y) for c in cps]
+        return _rot([lambda c=c: self.nv.qmv(self.x, c[0], c[1], self.g_x, self.g_w, self.y) for c in cps], 12)
 
     def setup(self):
         d = self.wl.make("gemv", device=self.dev)
@@ -362,10 +362,10 @@ class Prefill(Row):
     name, launches = "prefill", 5
     b2b_label = "gemm"
 
-    def b2b(self):  # eight copies of the quantized operands (8 x 18.9 MB)
+    def b2b(self):  # eight copies of the quantized operands (8 x 18.9 MB), two passes
         cps = [(self.xc.clone(), self.xs.clone(), self.wc.clone(), self.ws.clone()) for _ in range(8)]
-        return [lambda c=c: self.nv.qqmm(c[0], c[1], c[2], c[3], self.K, "nvfp4", self.g_x, self.g_w, out=self.y)
-                for c in cps]
+        return _rot([lambda c=c: self.nv.qqmm(c[0], c[1], c[2], c[3], self.K, "nvfp4", self.g_x, self.g_w,
+                                              out=self.y) for c in cps], 16)
 
     def setup(self):
         d = self.wl.make("prefill", device=self.dev)
@@ -413,9 +413,10 @@ class PrefillBwd(Row):
     name, launches = "prefill_bwd", 7
     b2b_label = "gemm_dx"
 
-    def b2b(self):  # eight copies of dx's quantized operands
+    def b2b(self):  # eight copies of dx's quantized operands, two passes
         cps = [tuple(t.clone() for t in (*self.cq, *self.wtq)) for _ in range(8)]
-        return [lambda c=c: self.nv.qqmm(*c, self.N, "nvfp4", self.g_c, self.g_w, out=self.dx) for c in cps]
+        return _rot([lambda c=c: self.nv.qqmm(*c, self.N, "nvfp4", self.g_c, self.g_w, out=self.dx)
+                     for c in cps], 16)
 
     def setup(self):
         d = self.wl.make("prefill_bwd", device=self.dev)
