@@ -64,3 +64,20 @@ def test_kn_layout_equals_transposed_layout_on_exact_weights(orc):
             e = idx[t, j]
             np.testing.assert_allclose(r_kn["y_ref"][t, j], xf[t] @ (W[e].astype(np.float64) * g[e] / 2688.0),
                                        rtol=0, atol=1e-9)
+
+
+def test_mutation_kn_without_transposing_fails(orc):
+    """Mistake: take the [K, N] decode as if it were [N, K] (no transpose of
+    the decoded weight).  With K != N the product is not even defined; with
+    K == N it gives x . w_hat^T, which the exact-weights pin rejects."""
+    rng = np.random.default_rng(9)
+    K = N = 48
+    W = _grid_weight(rng, K, N)
+    c, s = orc.nvfp4_quantize(W, "f32")
+    x = bf16(rng.standard_normal((3, K)))
+    idx = np.zeros((3, 1), dtype=np.int32)
+    right = orc.gather_qmm(x, c[None], s[None], None, idx, transpose=False)["y_ref"]
+    wrong = orc.gather_qmm(x, c[None], s[None], None, idx, transpose=True)["y_ref"]  # w_hat used as [N, K]
+    assert not np.array_equal(right, wrong)
+    xf = bf16_value(x)
+    np.testing.assert_allclose(right[:, 0], xf @ W.astype(np.float64), rtol=0, atol=1e-9)

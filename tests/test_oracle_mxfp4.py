@@ -102,3 +102,45 @@ def test_mxfp4_dequantize_rounds_once_to_bf16(orc):
     exact = orc.mxfp4_decode_exact(codes, scales)
     # e2m1 (2 significant bits) times a power of two is a bf16 value: no rounding
     np.testing.assert_array_equal(orc.to_f64(orc.mxfp4_dequantize(codes, scales, "bf16"), "bf16"), exact)
+
+
+# ---------------------------------------------------------------------------
+# Mutation checks: plant a mistake in a copy of an MXFP4 step, see a pin fail
+# ---------------------------------------------------------------------------
+def _golden_scale_with(mistake):
+    """Scale byte of each hand-derived block computed with a planted mistake."""
+    out = []
+    for name, x4, s, _ in _golden_blocks():
+        a = np.float32(max(abs(v) for v in x4))
+        if mistake == "round_nearest":     # e8m0 of max/6 to the nearest power, not up
+            v = a / np.float32(6.0)
+            e = int(np.round(np.log2(float(v)))) if v > 0 else -127
+        elif mistake == "divisor_448":     # the MXFP8 divisor
+            v = a / np.float32(448.0)
+            e = int(np.ceil(np.log2(float(v)))) if v > 0 else -127
+        else:
+            v = a / np.float32(6.0)
+            e = int(np.ceil(np.log2(float(v)))) if v > 0 else -127
+        out.append((name, e + 127, s))
+    return out
+
+
+def test_mutation_mxfp4_round_nearest_scale_fails_golden():
+    assert any(got != want for _, got, want in _golden_scale_with("round_nearest"))
+    assert all(got == want for _, got, want in _golden_scale_with(None))  # the unmutated step agrees
+
+
+def test_mutation_mxfp4_mxfp8_divisor_fails_golden():
+    assert any(got != want for _, got, want in _golden_scale_with("divisor_448"))
+
+
+def test_mutation_mxfp4_ties_away_fails_golden(orc):
+    """Mistake: round ties away from zero instead of to the even code; the
+    max6 block's 2.5 would become 3 (code 5) where the pin expects code 4."""
+    name, x4, s, c4 = _golden_blocks()[0]
+    k = 2.0 ** (127 - s)
+    t = abs(x4[1]) * k
+    lo = max(m for m in E2M1 if m <= t)
+    hi = min(m for m in E2M1 if m >= t)
+    away = hi if (t - lo) >= (hi - t) else lo
+    assert E2M1.index(away) != c4[1]

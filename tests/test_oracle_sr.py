@@ -113,3 +113,29 @@ def test_sr_grid_values_unchanged(orc):
     c_rn, _ = orc.nvfp4_quantize(x, "f32", None)
     for seed in (0, 1, 2**40 + 3):
         assert np.array_equal(orc.nvfp4_quantize_sr(x, "f32", None, seed=seed)[0], c_rn)
+
+
+# ---------------------------------------------------------------------------
+# Mutation checks: plant a mistake in a copy of an SR step, see a pin fail
+# ---------------------------------------------------------------------------
+def test_mutation_sr_comparison_reversed_is_biased(orc):
+    """Mistake: round up when u >= frac (the complementary event).  The mean
+    of many draws then sits at the mirror position, which the unbiasedness
+    pin rejects."""
+    t, lo, hi = 2.25, 2.0, 3.0
+    frac = (t - lo) / (hi - lo)
+    ups = sum(1 for i in range(20000) if ((orc.sr_bits(7, i) / 256.0) >= frac))
+    mean = lo + (hi - lo) * ups / 20000
+    sigma = (hi - lo) * np.sqrt(frac * (1 - frac) / 20000)
+    assert abs(mean - t) > 5 * sigma
+
+
+def test_mutation_sr_wrong_byte_fails_extraction_pin(orc):
+    """Mistake: every element of a group of 4 takes byte 0 of the word."""
+    seed = 0x0123456789ABCDEF
+    diffs = 0
+    for i in range(1, 64, 4):
+        w = i // 4
+        out = orc.philox4x32_10([w // 4 & 0xFFFFFFFF, w // 4 >> 32, 0, 0], [seed & 0xFFFFFFFF, seed >> 32])
+        diffs += orc.sr_bits(seed, i) != (int(out[w % 4]) & 0xFF)
+    assert diffs > 0
