@@ -28,14 +28,18 @@
 //   warp 1   TMEM allocator and MMA issuer: one elected lane of the
 //            converged warp moves the stage's
 //            scale tiles into tensor memory (tcgen05.cp 32x128b.warpx4) and
-//            issues the block-scaled MMAs (M=128, N=256, K=64 NVFP4 / 32
-//            MXFP8 per instruction) into a 128 x 256 fp32 accumulator in TMEM;
+//            issues the block-scaled MMAs (M=128, N=256, K=64 NVFP4 and
+//            MXFP4 / 32 MXFP8 per instruction) into a 128 x 256 fp32
+//            accumulator in TMEM;
 //            tcgen05.commit frees the stage when its MMAs are done.
 //   warps 2-9 epilogue: two warps per TMEM lane quarter (warp w reads lanes
 //            32*(w%4)...), 128 accumulator columns each; they drain the
 //            accumulator into registers, release it to the MMA warp at once
 //            (so the next tile's MMAs start), then apply alpha, convert and
-//            store while the tensor core works on the next tile.
+//            store while the tensor core works on the next tile: 32 rows x
+//            32 bytes at a time staged in the warp's shared-memory box and
+//            written by a TMA tensor store (direct stores when the output's
+//            row pitch is not a multiple of 16 bytes).
 // Every mbarrier wait is bounded; on timeout the kernel sets the device
 // error word (NVFP4_ERR_TIMEOUT through nvfp4_check_device_errors), drains,
 // frees its TMEM and exits.  No cluster multicast is used.
