@@ -798,6 +798,42 @@ def cpu_baseline_prefill(sample_rows=16):
                       f"element steps single-threaded C, contraction numpy float64 ({threads} BLAS threads)"}
 
 
+def cpu_baseline_rows(quant_rows=256, gemv_rows=2048):
+    """The oracle as it stands on two more rows of the hot path, on this
+    host's cores, each on a bounded slice of its config: the NVFP4 quantize
+    on ``quant_rows`` of the 1 GiB config's 32768 rows, and the qmv decode
+    GEMV (quantize-dequantize of x, exact weight decode, float64 sum) on
+    ``gemv_rows`` of the weight's 14336 rows; GB/s of the slice.  Element
+    steps are single-threaded C."""
+    from mxfp8_block_scaled_nvfp4_b200 import workloads
+    from oracle import oracle as orc
+    orc.build()
+    out = {}
+    xq = workloads.normal((quant_rows, 16384), 1.0, 10, torch.bfloat16, "cpu")
+    xr = xq.contiguous().view(torch.int16).numpy().view(np.uint16)
+    t0 = time.perf_counter()
+    g = orc.amax(xr, "bf16")
+    orc.nvfp4_quantize(xr, "bf16", g)
+    dt = time.perf_counter() - t0
+    nbytes = quant_rows * 16384 * (2 + 0.5 + 1 / 16)
+    out["quant1g"] = {"value": nbytes / dt / 1e9, "unit": "GB/s", "seconds": dt,
+                      "sample": f"amax + NVFP4 quantize of {quant_rows} of 32768 rows of the 1 GiB config"}
+    d = workloads.make("gemv", device="cpu")
+    x = d["x"].contiguous().view(torch.int16).numpy().view(np.uint16)
+    w = d["w"][:gemv_rows].contiguous().view(torch.int16).numpy().view(np.uint16)
+    gw = orc.amax(w, "bf16")
+    wc, ws = orc.nvfp4_quantize(w, "bf16", gw)
+    t0 = time.perf_counter()
+    gx = orc.amax(x, "bf16")
+    orc.qmv(x, "bf16", gx, wc, ws, gw)
+    dt = time.perf_counter() - t0
+    nbytes = wc.nbytes + ws.nbytes + x.nbytes + 2 * w.shape[0]
+    out["gemv"] = {"value": nbytes / dt / 1e9, "unit": "GB/s", "seconds": dt,
+                   "sample": f"qmv of the decode config on {gemv_rows} of 14336 weight rows "
+                             "(weight pre-quantized, as on the GPU)"}
+    return out
+
+
 def run_ours(args):
     world, rank, local = dist_setup(args.gpus)
     from mxfp8_block_scaled_nvfp4_b200 import build, nvfp4 as nv, workloads as wl
@@ -904,6 +940,7 @@ def run_ours(args):
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             cpu = cpu_baseline_prefill()
+            cpu["rows"] = cpu_baseline_rows()
             if head_row != "prefill":
                 cpu["note"] = "headline row is not prefill; baseline of the prefill op shown"
         roof = dict(head["roofline"])
