@@ -1,6 +1,6 @@
 /*
- * nvfp4.h -- C ABI of libnvfp4.so: NVFP4 / MXFP8 block-scaled quantize,
- * dequantize and quantized matmuls on NVIDIA B200 (sm_100a).
+ * nvfp4.h -- C ABI of libnvfp4.so: NVFP4 / MXFP8 / MXFP4 block-scaled
+ * quantize, dequantize and quantized matmuls on NVIDIA B200 (sm_100a).
  *
  * Sources, cited by page title and section:
  *  [P1] "mlx 0.30.7.2 -> 0.30.7.6" diff, page 8: ops.cpp validate_global_scale,
@@ -21,9 +21,9 @@
  *    device memory and never synchronizes; each call only enqueues kernels on
  *    `stream` (NULL = legacy default stream) and returns.
  *  - Layout: row-major, contiguous.  Every tensor pointer must be 16-byte
- *    aligned.  Codes of NVFP4 are uint32 words holding 8 e2m1 codes, element
- *    8w+i of a row in bits 4i..4i+3 of word w; codes of MXFP8 hold 4 e4m3
- *    bytes, element 4w+i in byte i.
+ *    aligned.  Codes of NVFP4 and MXFP4 are uint32 words holding 8 e2m1
+ *    codes, element 8w+i of a row in bits 4i..4i+3 of word w; codes of MXFP8
+ *    hold 4 e4m3 bytes, element 4w+i in byte i.
  *  - Scale layouts: NVFP4_LAYOUT_LINEAR is [rows, K/group] uint8.
  *    NVFP4_LAYOUT_SWIZZLED is the 128x4-tile layout the block-scaled MMA
  *    reads ([P5]; [P1] pad_and_swizzle_scales): a [ceil128(rows),
