@@ -185,6 +185,8 @@ class Row:
     # launches), captured as one graph with events only around the R launches,
     # so the mean is the kernel's own launch duration with cold operands.
     b2b_label = None
+    b2b_kernels = 1  # our kernels per back-to-back call
+    b2b_n = 0
 
     def b2b(self):
         return None
@@ -457,8 +459,9 @@ class PrefillBwd(Row):
 
 
 class Moe(Row):
-    name, launches = "moe", 3
+    name, launches = "moe", 2  # k_route + k_gather_mma
     b2b_label = "gather_qmm"
+    b2b_kernels = 2  # routing + the tensor-core kernel
     b2b_transpose = True
 
     def b2b(self):  # two copies of the 108 MB expert weights, alternating
@@ -505,7 +508,7 @@ class MoeKN(Moe):
     """The MoE config with the expert weights stored [E, K, N] and quantized
     along N (gather_qmm with transpose=False): same tokens, routing and
     per-expert global scales as the moe row."""
-    name, launches = "moe_kn", 3
+    name, launches = "moe_kn", 2
     b2b_transpose = False
 
     def setup(self):
@@ -547,6 +550,7 @@ class MoeDecode(Row):
     [1408, 2048], 4 tokens routed top-8 (tokens 0-3 of the MoE routing)."""
     name, launches = "moe_decode", 2
     b2b_label = "gather_qmm"
+    b2b_kernels = 2  # routing + the decode kernel
 
     def b2b(self):  # four copies of the experts' weights (the call reads the routed ones)
         cps = [(self.wc.clone(), self.ws.clone()) for _ in range(4)]
@@ -964,7 +968,7 @@ def run_ours(args):
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": sum(r.launches for r in rows) * args.steps,
+            "gpu_launches": sum(r.launches + r.b2b_n * r.b2b_kernels for r in rows) * args.steps,
             "clocks": clocks,
             "rows": reports,
         }
