@@ -41,6 +41,12 @@
  *    index out of range in gather_qmm; a bounded wait that gave up in the
  *    tensor-core GEMM) set a device error word instead of trapping; read it
  *    with nvfp4_check_device_errors().
+ *  - Empty outputs: a call whose output has no element (rows, N, M or T is
+ *    0, or K is 0 for the quantizers) returns NVFP4_OK after its argument
+ *    checks without querying or touching the device; its pointers may then
+ *    be NULL.  nvfp4_amax is the exception: it writes *g_out = 0 for n = 0.
+ *    The GEMMs (qqmm, gather_qmm, gather_qmm_kn) reject K = 0 with a
+ *    non-empty output (NVFP4_ERR_INVALID_ARG); qmv needs K >= 32.
  */
 #ifndef NVFP4_H_
 #define NVFP4_H_

@@ -188,10 +188,10 @@ static nvfp4_status quantize_common(const char* tag, int kind, const void* x, nv
   if (rows * K > 0 && (!x || !codes || !scales)) return fail(NVFP4_ERR_INVALID_ARG, "[%s] null pointer", tag);
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(g) & 3u))
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] tensor pointers must be 16-byte aligned", tag);
+  if (rows * K == 0) return ok();  // nothing to write: no device work, no device query
   DeviceInfo d;
   nvfp4_status st = device_info(tag, &d);
   if (st != NVFP4_OK) return st;
-  if (rows * K == 0) return ok();
   ScaleOut so;
   so.p = scales;
   so.blocks_per_row = (uint32_t)(K / group);
@@ -245,10 +245,10 @@ nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, int64_t ro
   if (rows * cols > 0 && (!x || !codes || !scales)) return fail(NVFP4_ERR_INVALID_ARG, "[%s] null pointer", tag);
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(g) & 3u))
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] tensor pointers must be 16-byte aligned", tag);
+  if (rows * cols == 0) return ok();
   DeviceInfo d;
   nvfp4_status st = device_info(tag, &d);
   if (st != NVFP4_OK) return st;
-  if (rows * cols == 0) return ok();
   ScaleOut so;
   so.p = scales;
   so.blocks_per_row = (uint32_t)(rows / 16);
@@ -286,10 +286,10 @@ static nvfp4_status dequantize_common(const char* tag, int kind, const uint32_t*
   if (rows * K > 0 && (!codes || !scales || !out)) return fail(NVFP4_ERR_INVALID_ARG, "[%s] null pointer", tag);
   if (!aligned16(codes) || !aligned16(scales) || !aligned16(out) || (reinterpret_cast<uintptr_t>(g) & 3u))
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] tensor pointers must be 16-byte aligned", tag);
+  if (rows * K == 0) return ok();  // nothing to write: no device work, no device query
   DeviceInfo d;
   nvfp4_status st = device_info(tag, &d);
   if (st != NVFP4_OK) return st;
-  if (rows * K == 0) return ok();
   ScaleIn si;
   si.p = scales;
   si.blocks_per_row = (uint32_t)(K / group);
@@ -331,10 +331,10 @@ nvfp4_status nvfp4_swizzle_scales(const uint8_t* lin, int64_t rows, int64_t cols
   if (rows * cols > 0 && (!lin || !swz)) return fail(NVFP4_ERR_INVALID_ARG, "[swizzle_scales] null pointer");
   if (!aligned16(lin) || !aligned16(swz))
     return fail(NVFP4_ERR_INVALID_ARG, "[swizzle_scales] Starting addresses must be 16-byte aligned");
+  if (rows * cols == 0) return ok();
   DeviceInfo d;
   nvfp4_status st = device_info("swizzle_scales", &d);
   if (st != NVFP4_OK) return st;
-  if (rows * cols == 0) return ok();
   const uint32_t Rp = (uint32_t)((rows + 127) / 128 * 128), Cp = (uint32_t)((cols + 3) / 4 * 4);
   const unsigned grid = ew_grid(d, (uint64_t)Rp * Cp);
   k_swizzle_scales<<<grid, kEwThreads, 0, stream>>>(lin, (uint32_t)rows, (uint32_t)cols, Rp, Cp, swz);
@@ -364,15 +364,16 @@ nvfp4_status qqmm(nvfp4_mode mode, int64_t M, int64_t N, int64_t K, const uint32
     return fail(NVFP4_ERR_INVALID_ARG, "[qqmm] bad shape");
   if (K % 32 != 0)
     return fail(NVFP4_ERR_INVALID_ARG, "[qqmm] K must be a multiple of 32, got %lld", (long long)K);
+  if (K == 0 && M * N > 0) return fail(NVFP4_ERR_INVALID_ARG, "[qqmm] K must be positive when M*N > 0");
   if (M * N > 0 && (!a_codes || !a_scales || !b_codes || !b_scales || !y))
     return fail(NVFP4_ERR_INVALID_ARG, "[qqmm] null pointer");
   if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) || !aligned16(y) ||
       (reinterpret_cast<uintptr_t>(g_x) & 3u) || (reinterpret_cast<uintptr_t>(g_w) & 3u))
     return fail(NVFP4_ERR_INVALID_ARG, "[qqmm] tensor pointers must be 16-byte aligned");
+  if (M * N == 0) return ok();
   DeviceInfo d;
   st = device_info("qqmm", &d);
   if (st != NVFP4_OK) return st;
-  if (M * N == 0) return ok();
   return qqmm_launch((int)mode, M, N, K, a_codes, a_scales, b_codes, b_scales, g_x, g_w, y,
                      (int)y_dt, d.sm_count, stream, t_msg, sizeof(t_msg));
 }
@@ -392,10 +393,10 @@ nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32
   if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y) ||
       (reinterpret_cast<uintptr_t>(g_x) & 3u) || (reinterpret_cast<uintptr_t>(g_w) & 3u))
     return fail(NVFP4_ERR_INVALID_ARG, "[qmv] tensor pointers must be 16-byte aligned");
+  if (N == 0) return ok();
   DeviceInfo d;
   nvfp4_status st = device_info("qmv", &d);
   if (st != NVFP4_OK) return st;
-  if (N == 0) return ok();
   cudaError_t e = cudaSuccess;
   const uint32_t stages = qtc::pick_stages(M, K);
   if (stages > 0) {
@@ -445,26 +446,40 @@ size_t gather_qmm_workspace_size(int64_t T, int64_t topk, int64_t E) {
   return gather_workspace_bytes(T, topk, E);
 }
 
+// Host checks shared by the gather entries: shapes (K % 64, N % n_mult, K > 0
+// when there is output), pointers and, where the caller passes one
+// (check_ws), the workspace size.
+static nvfp4_status check_gather(const char* tag, int n_mult, const void* x, const uint32_t* w_codes,
+                                 const uint8_t* w_scales, const float* g, const int32_t* idx, int64_t T,
+                                 int64_t topk, int64_t E, int64_t N, int64_t K, const void* y, bool check_ws,
+                                 const void* workspace, size_t workspace_bytes) {
+  if (T < 0 || topk < 1 || E < 1 || N < 0 || K < 0 || T * topk > (1 << 30) || E > (1 << 20))
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] bad shape", tag);
+  if (K % 64 != 0 || N % n_mult != 0)
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] K must be a multiple of 64 and N of %d (K=%lld N=%lld)", tag, n_mult,
+                (long long)K, (long long)N);
+  if (K == 0 && T * N > 0) return fail(NVFP4_ERR_INVALID_ARG, "[%s] K must be positive when T*N > 0", tag);
+  if (check_ws && workspace_bytes < gather_workspace_bytes(T, topk, E))
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] workspace too small: %zu < %zu", tag, workspace_bytes,
+                gather_workspace_bytes(T, topk, E));
+  if (T * N > 0 && (!x || !w_codes || !w_scales || !idx || !y || (check_ws && !workspace)))
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] null pointer", tag);
+  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y) || !aligned16(workspace) ||
+      !aligned16(idx) || !aligned16(g))
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] tensor pointers must be 16-byte aligned", tag);
+  return NVFP4_OK;
+}
+
 nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const uint8_t* w_scales, const float* g,
                         const int32_t* idx, int64_t T, int64_t topk, int64_t E, int64_t N, int64_t K, void* y,
                         void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
-  if (T < 0 || topk < 1 || E < 1 || N < 0 || K < 0 || T * topk > (1 << 30) || E > (1 << 20))
-    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm] bad shape");
-  if (K % 64 != 0 || N % 16 != 0)
-    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm] K must be a multiple of 64 and N of 16 (K=%lld N=%lld)",
-                (long long)K, (long long)N);
-  if (workspace_bytes < gather_workspace_bytes(T, topk, E))
-    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm] workspace too small: %zu < %zu", workspace_bytes,
-                gather_workspace_bytes(T, topk, E));
-  if (T * N > 0 && (!x || !w_codes || !w_scales || !idx || !y || !workspace))
-    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm] null pointer");
-  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y) || !aligned16(workspace) ||
-      !aligned16(idx) || !aligned16(g))
-    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm] tensor pointers must be 16-byte aligned");
-  DeviceInfo d;
-  nvfp4_status st = device_info("gather_qmm", &d);
+  nvfp4_status st = check_gather("gather_qmm", 16, x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, true,
+                                 workspace, workspace_bytes);
   if (st != NVFP4_OK) return st;
   if (T * N == 0) return ok();
+  DeviceInfo d;
+  st = device_info("gather_qmm", &d);
+  if (st != NVFP4_OK) return st;
   return gather_qmm_launch(x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, workspace, d.sm_count, stream, t_msg,
                            sizeof(t_msg));
 }
@@ -472,23 +487,13 @@ nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const uint8_t* w
 nvfp4_status gather_qmm_kn(const void* x, const uint32_t* w_codes, const uint8_t* w_scales, const float* g,
                         const int32_t* idx, int64_t T, int64_t topk, int64_t E, int64_t N, int64_t K, void* y,
                         void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
-  if (T < 0 || topk < 1 || E < 1 || N < 0 || K < 0 || T * topk > (1 << 30) || E > (1 << 20))
-    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm_kn] bad shape");
-  if (K % 64 != 0 || N % 32 != 0)
-    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm_kn] K must be a multiple of 64 and N of 32 (K=%lld N=%lld)",
-                (long long)K, (long long)N);
-  if (workspace_bytes < gather_workspace_bytes(T, topk, E))
-    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm_kn] workspace too small: %zu < %zu", workspace_bytes,
-                gather_workspace_bytes(T, topk, E));
-  if (T * N > 0 && (!x || !w_codes || !w_scales || !idx || !y || !workspace))
-    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm_kn] null pointer");
-  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y) || !aligned16(workspace) ||
-      !aligned16(idx) || !aligned16(g))
-    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm_kn] tensor pointers must be 16-byte aligned");
-  DeviceInfo d;
-  nvfp4_status st = device_info("gather_qmm_kn", &d);
+  nvfp4_status st = check_gather("gather_qmm_kn", 32, x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, true,
+                                 workspace, workspace_bytes);
   if (st != NVFP4_OK) return st;
   if (T * N == 0) return ok();
+  DeviceInfo d;
+  st = device_info("gather_qmm_kn", &d);
+  if (st != NVFP4_OK) return st;
   return gather_qmm_launch(x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, workspace, d.sm_count, stream, t_msg,
                            sizeof(t_msg), true);
 }
@@ -526,8 +531,12 @@ nvfp4_status gather_qmm_noalloc(const void* x, const uint32_t* w_codes, const ui
                 "[gather_qmm_noalloc] T=%lld, topk=%lld, E=%lld needs %zu bytes of scratch; the static scratch "
                 "holds %zu bytes (use gather_qmm with a caller-provided workspace)",
                 (long long)T, (long long)topk, (long long)E, need, kNoAllocScratchBytes);
+  nvfp4_status st = check_gather("gather_qmm_noalloc", 16, x, w_codes, w_scales, g, idx, T, topk, E, N, K, y,
+                                 false, nullptr, 0);
+  if (st != NVFP4_OK) return st;
+  if (T * N == 0) return ok();
   void* scratch = nullptr;
-  nvfp4_status st = noalloc_scratch(&scratch);
+  st = noalloc_scratch(&scratch);
   if (st != NVFP4_OK) return st;
   // The routing kernel rewrites every scratch entry the grouped kernel reads
   // (tile count, tile list, permutation), so nothing needs clearing between

@@ -145,3 +145,49 @@ def test_binding_refuses_cpu_tensors():
     from mxfp8_block_scaled_nvfp4_b200 import nvfp4
     with pytest.raises(ValueError):
         nvfp4.amax(torch.ones(16))
+
+
+def test_empty_outputs_return_ok_without_a_device(L):
+    """A call with nothing to write returns NVFP4_OK after its argument checks,
+    with NULL pointers and no device present; the same call with work needs
+    the device (here: none, so it fails)."""
+    N0 = None
+    assert L.nvfp4_quantize(N0, 2, 0, 64, N0, N0, N0, 0, N0) == 0
+    assert L.nvfp4_quantize(N0, 2, 7, 0, N0, N0, N0, 1, N0) == 0
+    assert L.nvfp4_quantize_sr(N0, 2, 0, 64, N0, 5, N0, N0, 1, N0) == 0
+    assert L.nvfp4_quantize_columnwise(N0, 2, 32, 0, N0, N0, N0, 1, N0) == 0
+    assert L.nvfp4_quantize_columnwise(N0, 2, 0, 5, N0, N0, N0, 0, N0) == 0
+    assert L.mxfp8_quantize(N0, 2, 0, 64, N0, N0, 1, N0) == 0
+    assert L.mxfp4_quantize(N0, 2, 3, 0, N0, N0, 0, N0) == 0
+    assert L.nvfp4_dequantize(N0, N0, 1, 0, 64, N0, N0, 2, N0) == 0
+    assert L.mxfp8_dequantize(N0, N0, 0, 5, 0, N0, 0, N0) == 0
+    assert L.mxfp4_dequantize(N0, N0, 1, 0, 32, N0, 1, N0) == 0
+    assert L.nvfp4_swizzle_scales(N0, 0, 4, N0, N0) == 0
+    for mode in (0, 1, 2):
+        assert L.qqmm(mode, 0, 128, 256, N0, N0, N0, N0, N0, N0, N0, 2, N0) == 0
+        assert L.qqmm(mode, 64, 0, 0, N0, N0, N0, N0, N0, N0, N0, 0, N0) == 0
+    assert L.qmv(N0, 2, N0, N0, N0, N0, 1, 0, 256, N0, N0) == 0
+    ws = L.gather_qmm_workspace_size(0, 2, 4)
+    assert L.gather_qmm(N0, N0, N0, N0, N0, 0, 2, 4, 64, 128, N0, N0, ws, N0) == 0
+    assert L.gather_qmm(N0, N0, N0, N0, N0, 16, 2, 4, 0, 128, N0, N0, L.gather_qmm_workspace_size(16, 2, 4), N0) == 0
+    assert L.gather_qmm_kn(N0, N0, N0, N0, N0, 0, 2, 4, 64, 128, N0, N0, ws, N0) == 0
+    assert L.gather_qmm_noalloc(N0, N0, N0, N0, N0, 0, 2, 4, 64, 128, N0, N0) == 0
+    # argument checks still run for empty outputs
+    assert L.nvfp4_quantize(N0, 2, 0, 24, N0, N0, N0, 0, N0) == 1
+    assert L.qqmm(0, 0, 128, 48, N0, N0, N0, N0, N0, N0, N0, 2, N0) == 1
+    assert L.gather_qmm_noalloc(N0, N0, N0, N0, N0, 0, 2, 4, -16, 128, N0, N0) == 1
+    # the same shapes with work to do reach the device query (no device here)
+    assert L.nvfp4_quantize(A, 2, 4, 64, N0, A, A, 0, N0) not in (0, 1, 2)
+    assert L.qqmm(0, 128, 128, 256, A, A, A, A, N0, N0, A, 2, N0) not in (0, 1, 2)
+
+
+def test_gemms_reject_K_zero_with_an_output(L):
+    for mode in (0, 1, 2):
+        assert L.qqmm(mode, 128, 128, 0, A, A, A, A, None, None, A, 2, None) == 1
+        assert "K must be positive" in msg(L)
+    ws = L.gather_qmm_workspace_size(16, 2, 4)
+    assert L.gather_qmm(A, A, A, A, A, 16, 2, 4, 64, 0, A, A, ws, None) == 1
+    assert "K must be positive" in msg(L)
+    assert L.gather_qmm_kn(A, A, A, A, A, 16, 2, 4, 64, 0, A, A, ws, None) == 1
+    assert L.gather_qmm_noalloc(A, A, A, A, A, 16, 2, 4, 64, 0, A, None) == 1
+    assert L.qmv(A, 2, None, A, A, None, 1, 64, 0, A, None) == 1
