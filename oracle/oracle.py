@@ -391,6 +391,27 @@ def qqmm(a_codes, a_scales, b_codes, b_scales, mode="nvfp4", g_x=None, g_w=None,
     return {"y_ref": y_ref, "abs_ref": abs_ref, "y": round_to(y_ref, out_dt)}
 
 
+def qqmm_vjp(x, w, cotan, dt: str, g_x: float, g_w: float):
+    """Backward pass of y = qqmm(x, w) in NVFP4 mode ([P1] primitives.cpp
+    QQMatmul::vjp), each product a fresh quantize of both operands followed by
+    the dense quantized matmul above:
+      dx [M, K] = cotan_hat . ((w^T)_hat)^T, cotan quantized along N with
+                  g_c = amax(cotan), w^T [K, N] quantized along N with g_w;
+      dw [N, K] = (cotan^T)_hat . ((x^T)_hat)^T, cotan^T [N, M] and x^T [K, M]
+                  quantized along M, with g_c and g_x.
+    x [M, K], w [N, K], cotan [M, N] are raw arrays of dt.  Returns
+    (dx, dw), each qqmm's dict with the output in dt."""
+    x, w, cotan = np.asarray(x), np.asarray(w), np.asarray(cotan)
+    g_c = amax(cotan, dt)
+    c_codes, c_scales = nvfp4_quantize(cotan, dt, g_c)
+    wt_codes, wt_scales = nvfp4_quantize(np.ascontiguousarray(w.T), dt, g_w)
+    dx = qqmm(c_codes, c_scales, wt_codes, wt_scales, "nvfp4", g_c, g_w, dt)
+    ct_codes, ct_scales = nvfp4_quantize(np.ascontiguousarray(cotan.T), dt, g_c)
+    xt_codes, xt_scales = nvfp4_quantize(np.ascontiguousarray(x.T), dt, g_x)
+    dw = qqmm(ct_codes, ct_scales, xt_codes, xt_scales, "nvfp4", g_c, g_x, dt)
+    return dx, dw
+
+
 # --------------------------------------------------------------------------
 # a6-a7: qmv (small-M route of qqmm with pre-quantized w)
 # --------------------------------------------------------------------------

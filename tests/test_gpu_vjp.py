@@ -67,15 +67,7 @@ def test_qqmm_vjp_parity(nv, orc, M, N, K, dt):
     g_x, g_w = nv.amax(xg), nv.amax(wg)
     dx, dw = nv.qqmm_vjp(xg, wg, cg, g_x, g_w)
     nv.check_device_errors()
-    gc = orc.amax(raw(cotan), dt)
-    gx, gw = g_x.item(), g_w.item()
-    # dx: cotan quantized along N, w^T along N
-    occ, ocs = orc.nvfp4_quantize(raw(cotan), dt, gc)
-    owt, ows = orc.nvfp4_quantize(raw(w.t().contiguous()), dt, gw)
-    r = orc.qqmm(occ, ocs, owt, ows, "nvfp4", gc, gw, dt)
-    check_gemm_output(raw(dx), r, dt, orc)
-    # dw: cotan^T along M, x^T along M
-    oct_, octs = orc.nvfp4_quantize(raw(cotan.t().contiguous()), dt, gc)
-    oxt, oxts = orc.nvfp4_quantize(raw(x.t().contiguous()), dt, gx)
-    r = orc.qqmm(oct_, octs, oxt, oxts, "nvfp4", gc, gx, dt)
-    check_gemm_output(raw(dw), r, dt, orc)
+    # dx: cotan and w^T quantized along N; dw: cotan^T and x^T along M
+    r_dx, r_dw = orc.qqmm_vjp(raw(x), raw(w), raw(cotan), dt, g_x.item(), g_w.item())
+    check_gemm_output(raw(dx), r_dx, dt, orc)
+    check_gemm_output(raw(dw), r_dw, dt, orc)
