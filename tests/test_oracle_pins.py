@@ -257,6 +257,53 @@ def test_mxfp8_zero_block(orc):
     assert np.all(s == 0) and np.all(q == 0)
 
 
+# (e4m3 code byte, e8m0 scale byte, value) from the two formats' definitions:
+# e4m3 (-1)^s 2^(e-7) (1 + m/8), subnormal (e = 0) 2^-6 m/8; e8m0 2^(b-127).
+MXFP8_DECODE_CASES = [
+    (0x38, 127, 1.0),                 # e=7 m=0
+    (0x7E, 127, 448.0),               # e=15 m=6: 2^8 * 1.75, the largest e4m3
+    (0x01, 127, 0.001953125),         # subnormal m=1: 2^-6 / 8 = 2^-9
+    (0xB8, 130, -8.0),                # sign, 1.0 * 2^3
+    (0x7A, 121, 5.0),                 # 320 * 2^-6: the round-up case decoded
+    (0x00, 200, 0.0),
+    (0x80, 127, -0.0),                # signed zero keeps its sign
+    (0x3C, 254, 1.5 * 2.0 ** 127),    # e=7 m=4, the largest e8m0 scale
+    (0x38, 0, 2.0 ** -127),           # the smallest e8m0 scale
+]
+
+
+@pytest.mark.parametrize("out_dt", ["f32", "bf16"])
+def test_mxfp8_dequantize_hand_decoded_bytes(orc, out_dt):
+    """One row per case: element 0 holds the case's code, the other 31 hold
+    0x38 (1.0), all under the case's scale; the product is exact in f32 and
+    bf16 for every case, so the dequantize returns it exactly."""
+    rows = len(MXFP8_DECODE_CASES)
+    code_bytes = np.full((rows, 32), 0x38, dtype=np.uint32)
+    scales = np.zeros((rows, 1), dtype=np.uint8)
+    want = np.zeros((rows, 32))
+    for r, (c, sb, v) in enumerate(MXFP8_DECODE_CASES):
+        code_bytes[r, 0] = c
+        scales[r, 0] = sb
+        want[r, 0] = v
+        want[r, 1:] = 2.0 ** (sb - 127)
+    words = code_bytes.reshape(rows, 8, 4)
+    codes = np.bitwise_or.reduce(words << (8 * np.arange(4, dtype=np.uint32)), axis=2).astype(np.uint32)
+    got = orc.to_f64(orc.mxfp8_dequantize(codes, scales, out_dt), out_dt)
+    np.testing.assert_array_equal(got, want)
+    assert np.signbit(got[6, 0]) and not np.signbit(got[5, 0])
+    np.testing.assert_array_equal(orc.mxfp8_decode_exact(codes, scales), want)
+
+
+def test_mxfp8_dequantize_of_quantize_round_up_case(orc):
+    """The round-up case's block maximum (4.8046875) comes back as 5.0: code
+    320 under scale 2^-6."""
+    G = golden("mxfp8_round_up.txt")
+    x = np.zeros((1, 32), dtype=np.float32)
+    x[0, 0] = float(G["block_max"])
+    q, s = orc.mxfp8_quantize(x, "f32")
+    assert orc.to_f64(orc.mxfp8_dequantize(q, s, "f32"), "f32")[0, 0] == 5.0
+
+
 # ---------------------------------------------------------------------------
 # Scale layout: the page's index table ("mlx 0.30.7" diff page 71)
 # ---------------------------------------------------------------------------
