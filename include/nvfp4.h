@@ -232,7 +232,8 @@ NVFP4_API nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, co
  * x [T, K] bf16; w_codes [E, N, K/8]; w_scales LINEAR [E, N, K/16];
  * g [E] fp32 or NULL; idx [T, topk] int32 in [0, E) (checked on the device:
  * out-of-range entries set NVFP4_ERR_DEVICE_INDEX and produce zero rows);
- * y [T, topk, N] bf16.  K % 64 == 0, N % 16 == 0.
+ * y [T, topk, N] bf16.  K % 64 == 0, N % 16 == 0; T*topk, N and K at most
+ * 2^30; 1 <= E <= 1024 (more experts: NVFP4_ERR_UNSUPPORTED).
  * workspace: device scratch of gather_qmm_workspace_size(T, topk, E) bytes,
  * 16-byte aligned, contents undefined on entry and exit. */
 NVFP4_API nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const uint8_t* w_scales,
@@ -252,6 +253,9 @@ NVFP4_API nvfp4_status gather_qmm_kn(const void* x, const uint32_t* w_codes, con
                         int64_t E, int64_t N, int64_t K, void* y, void* workspace,
                         size_t workspace_bytes, nvfp4_stream_t stream);
 
+/* Bytes of workspace gather_qmm and gather_qmm_kn need for (T, topk, E);
+ * 0 for a triple they reject (T < 0, topk < 1, E outside [1, 1024],
+ * T*topk > 2^30).  Host only. */
 NVFP4_API size_t gather_qmm_workspace_size(int64_t T, int64_t topk, int64_t E);
 
 /* gather_qmm without a workspace argument; the pages have no counterpart of

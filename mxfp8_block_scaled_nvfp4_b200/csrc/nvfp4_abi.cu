@@ -53,6 +53,9 @@ nvfp4_status check_launch(const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// a * b > limit for a, b >= 0, without forming the (possibly overflowing) product.
+bool product_exceeds(int64_t a, int64_t b, int64_t limit) { return b != 0 && a > limit / b; }
+
 struct DeviceInfo {
   int sm_count = 0;
   int cc_major = 0;
@@ -178,7 +181,7 @@ static nvfp4_status quantize_common(const char* tag, int kind, const void* x, nv
   if (!valid_dt(dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] dtype must be float32, float16 or bfloat16", tag);
   if (layout != NVFP4_LAYOUT_LINEAR && layout != NVFP4_LAYOUT_SWIZZLED)
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] unknown scale layout", tag);
-  if (rows < 0 || K < 0 || rows * K > kMaxElems)
+  if (rows < 0 || K < 0 || product_exceeds(rows, K, kMaxElems))
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] bad shape [%lld, %lld]", tag, (long long)rows, (long long)K);
   if (K % group != 0)
     return fail(NVFP4_ERR_INVALID_ARG,
@@ -235,7 +238,7 @@ nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, int64_t ro
   if (!valid_dt(dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] dtype must be float32, float16 or bfloat16", tag);
   if (layout != NVFP4_LAYOUT_LINEAR && layout != NVFP4_LAYOUT_SWIZZLED)
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] unknown scale layout", tag);
-  if (rows < 0 || cols < 0 || rows * cols > kMaxElems || rows > (1 << 30) || cols > (1 << 30))
+  if (rows < 0 || cols < 0 || rows > (1 << 30) || cols > (1 << 30) || rows * cols > kMaxElems)
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] bad shape [%lld, %lld]", tag, (long long)rows, (long long)cols);
   if (rows % 16 != 0)
     return fail(NVFP4_ERR_INVALID_ARG,
@@ -280,7 +283,7 @@ static nvfp4_status dequantize_common(const char* tag, int kind, const uint32_t*
   if (!valid_dt(out_dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] output dtype must be float32, float16 or bfloat16", tag);
   if (layout != NVFP4_LAYOUT_LINEAR && layout != NVFP4_LAYOUT_SWIZZLED)
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] unknown scale layout", tag);
-  if (rows < 0 || K < 0 || rows * K > kMaxElems || K % group != 0)
+  if (rows < 0 || K < 0 || product_exceeds(rows, K, kMaxElems) || K % group != 0)
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] bad shape [%lld, %lld] for group size %d", tag, (long long)rows,
                 (long long)K, group);
   if (rows * K > 0 && (!codes || !scales || !out)) return fail(NVFP4_ERR_INVALID_ARG, "[%s] null pointer", tag);
@@ -326,7 +329,7 @@ nvfp4_status mxfp4_dequantize(const uint32_t* codes, const uint8_t* scales, nvfp
 
 nvfp4_status nvfp4_swizzle_scales(const uint8_t* lin, int64_t rows, int64_t cols, uint8_t* swz,
                                   nvfp4_stream_t stream) {
-  if (rows < 0 || cols < 0 || rows * cols > ((int64_t)1 << 31))
+  if (rows < 0 || cols < 0 || product_exceeds(rows, cols, (int64_t)1 << 31))
     return fail(NVFP4_ERR_INVALID_ARG, "[swizzle_scales] bad shape");
   if (rows * cols > 0 && (!lin || !swz)) return fail(NVFP4_ERR_INVALID_ARG, "[swizzle_scales] null pointer");
   if (!aligned16(lin) || !aligned16(swz))
@@ -443,6 +446,7 @@ nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32
 }
 
 size_t gather_qmm_workspace_size(int64_t T, int64_t topk, int64_t E) {
+  if (T < 0 || topk < 1 || E < 1 || E > gq::MAX_E || product_exceeds(T, topk, 1 << 30)) return 0;
   return gather_workspace_bytes(T, topk, E);
 }
 
@@ -453,8 +457,10 @@ static nvfp4_status check_gather(const char* tag, int n_mult, const void* x, con
                                  const uint8_t* w_scales, const float* g, const int32_t* idx, int64_t T,
                                  int64_t topk, int64_t E, int64_t N, int64_t K, const void* y, bool check_ws,
                                  const void* workspace, size_t workspace_bytes) {
-  if (T < 0 || topk < 1 || E < 1 || N < 0 || K < 0 || T * topk > (1 << 30) || E > (1 << 20))
+  if (T < 0 || topk < 1 || E < 1 || N < 0 || K < 0 || product_exceeds(T, topk, 1 << 30) || N > (1 << 30) ||
+      K > (1 << 30))
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] bad shape", tag);
+  if (E > gq::MAX_E) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] at most %d experts, got %lld", tag, gq::MAX_E, (long long)E);
   if (K % 64 != 0 || N % n_mult != 0)
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] K must be a multiple of 64 and N of %d (K=%lld N=%lld)", tag, n_mult,
                 (long long)K, (long long)N);
@@ -523,18 +529,16 @@ static nvfp4_status noalloc_scratch(void** out) {
 nvfp4_status gather_qmm_noalloc(const void* x, const uint32_t* w_codes, const uint8_t* w_scales, const float* g,
                                 const int32_t* idx, int64_t T, int64_t topk, int64_t E, int64_t N, int64_t K,
                                 void* y, nvfp4_stream_t stream) {
-  if (T < 0 || topk < 1 || E < 1 || T * topk > (1 << 30) || E > (1 << 20))
-    return fail(NVFP4_ERR_INVALID_ARG, "[gather_qmm_noalloc] bad shape");
+  nvfp4_status st = check_gather("gather_qmm_noalloc", 16, x, w_codes, w_scales, g, idx, T, topk, E, N, K, y,
+                                 false, nullptr, 0);
+  if (st != NVFP4_OK) return st;
+  if (T * N == 0) return ok();
   const size_t need = gather_workspace_bytes(T, topk, E);
   if (need > kNoAllocScratchBytes)
     return fail(NVFP4_ERR_UNSUPPORTED,
                 "[gather_qmm_noalloc] T=%lld, topk=%lld, E=%lld needs %zu bytes of scratch; the static scratch "
                 "holds %zu bytes (use gather_qmm with a caller-provided workspace)",
                 (long long)T, (long long)topk, (long long)E, need, kNoAllocScratchBytes);
-  nvfp4_status st = check_gather("gather_qmm_noalloc", 16, x, w_codes, w_scales, g, idx, T, topk, E, N, K, y,
-                                 false, nullptr, 0);
-  if (st != NVFP4_OK) return st;
-  if (T * N == 0) return ok();
   void* scratch = nullptr;
   st = noalloc_scratch(&scratch);
   if (st != NVFP4_OK) return st;

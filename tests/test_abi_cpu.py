@@ -191,3 +191,37 @@ def test_gemms_reject_K_zero_with_an_output(L):
     assert L.gather_qmm_kn(A, A, A, A, A, 16, 2, 4, 64, 0, A, A, ws, None) == 1
     assert L.gather_qmm_noalloc(A, A, A, A, A, 16, 2, 4, 64, 0, A, None) == 1
     assert L.qmv(A, 2, None, A, A, None, 1, 64, 0, A, None) == 1
+
+
+def test_size_limits_without_overflow(L):
+    """Sizes whose products overflow int64 are rejected, not wrapped: the
+    checks bound each factor before multiplying."""
+    big = 1 << 40
+    assert L.nvfp4_quantize(A, 2, big, big, None, A, A, 0, None) == 1
+    assert L.nvfp4_quantize(A, 2, (1 << 33) + 1, 1 << 31, None, A, A, 0, None) == 1  # product wraps to 2^31
+    assert L.nvfp4_dequantize(A, A, 0, (1 << 33) + 1, 1 << 31, None, A, 2, None) == 1
+    assert L.mxfp8_quantize(A, 2, 1 << 62, 64, A, A, 0, None) == 1
+    assert L.nvfp4_quantize_columnwise(A, 2, 1 << 31, 1 << 40, None, A, A, 0, None) == 1
+    assert L.nvfp4_swizzle_scales(A, 1 << 40, 1 << 40, A, None) == 1
+    assert L.qqmm(0, (1 << 30) + 1, 128, 256, A, A, A, A, None, None, A, 2, None) == 1
+    ws = L.gather_qmm_workspace_size(16, 2, 4)
+    assert L.gather_qmm(A, A, A, A, A, 1 << 62, 4, 4, 64, 128, A, A, ws, None) == 1  # T*topk wraps to 0
+    assert L.gather_qmm(A, A, A, A, A, 16, 2, 4, 1 << 40, 128, A, A, ws, None) == 1
+    assert L.gather_qmm_noalloc(A, A, A, A, A, 1 << 62, 4, 4, 64, 128, A, None) == 1
+    # the largest accepted sizes pass the argument checks and reach the device query
+    assert L.nvfp4_quantize(A, 2, 1 << 20, 1 << 14, None, A, A, 0, None) not in (0, 1, 2)
+    assert L.nvfp4_quantize(A, 2, (1 << 20) + 1, 1 << 14, None, A, A, 0, None) == 1
+
+
+def test_gather_expert_limit_and_workspace_size(L):
+    ws = L.gather_qmm_workspace_size(16, 2, 1025)
+    assert ws == 0
+    big = L.gather_qmm_workspace_size(16, 2, 1024)
+    assert L.gather_qmm(A, A, A, A, A, 16, 2, 1025, 64, 128, A, A, big, None) == 2
+    assert "at most 1024 experts" in msg(L)
+    assert L.gather_qmm_noalloc(A, A, A, A, A, 16, 2, 1025, 64, 128, A, None) == 2
+    for bad in [(-1, 2, 4), (16, 0, 4), (16, 2, 0), (1 << 62, 4, 4)]:
+        assert L.gather_qmm_workspace_size(*bad) == 0
+    # monotone in T and covers at least the permutation (4 bytes per routed row)
+    sizes = [L.gather_qmm_workspace_size(t, 8, 64) for t in (1, 64, 4096)]
+    assert sizes == sorted(sizes) and sizes[-1] >= 4 * 4096 * 8
