@@ -98,6 +98,33 @@ def _need_cuda(*ts):
                 raise ValueError("tensors must be contiguous")
 
 
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+def _need_bytes(t, nbytes: int, what: str):
+    """The library takes raw pointers and cannot see a buffer's size: refuse
+    one smaller than the bytes the call reads or writes through it."""
+    if t is not None and _nbytes(t) < nbytes:
+        raise ValueError(f"{what} holds {_nbytes(t)} bytes; the call needs {nbytes}")
+
+
+def _need_dtype(t, dtype, what: str):
+    if t is not None and t.dtype != dtype:
+        raise ValueError(f"{what} must be {dtype}, got {t.dtype}")
+
+
+def _need_g(g, n: int = 1, what: str = "global scale"):
+    """Global scales are fp32 device scalars (n of them for per-expert g)."""
+    _need_dtype(g, torch.float32, what)
+    _need_bytes(g, 4 * n, what)
+
+
+def _scale_nbytes(rows: int, cols: int, layout: str) -> int:
+    r, c = scale_shape(rows, cols, layout)
+    return r * c
+
+
 def check_device_errors():
     _check(lib().nvfp4_check_device_errors(_stream()))
 
@@ -115,7 +142,8 @@ def scale_shape(rows: int, cols: int, layout: str):
 # ---------------------------------------------------------------------------
 def amax(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
     """fp32 [1] tensor holding max |x| (the global scale g)."""
-    _need_cuda(x)
+    _need_g(out, 1, "out")
+    _need_cuda(x, out)
     out = torch.empty(1, dtype=torch.float32, device=x.device) if out is None else out
     _check(lib().nvfp4_amax(_ptr(x), DT[x.dtype], x.numel(), _ptr(out), _stream()))
     return out
@@ -124,8 +152,11 @@ def amax(x: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
 def nvfp4_quantize(x: torch.Tensor, g: torch.Tensor | None = None, layout: str = "linear",
                    codes: torch.Tensor | None = None, scales: torch.Tensor | None = None):
     """(codes uint32 [rows, K/8] viewed as int32, scales uint8) of a 2-D x."""
-    _need_cuda(x, g)
     rows, K = x.shape
+    _need_g(g)
+    _need_bytes(codes, rows * (K // 8) * 4, "codes")
+    _need_bytes(scales, _scale_nbytes(rows, K // 16, layout), "scales")
+    _need_cuda(x, g, codes, scales)
     if codes is None:
         codes = torch.empty(rows, K // 8, dtype=torch.int32, device=x.device)
     if scales is None:
@@ -139,8 +170,11 @@ def nvfp4_quantize_columnwise(x: torch.Tensor, g: torch.Tensor | None = None, la
                               codes: torch.Tensor | None = None, scales: torch.Tensor | None = None):
     """(codes [cols, rows/8], scales) of x^T quantized along the rows of a 2-D x
     (equal to nvfp4_quantize(x.T.contiguous(), g, layout))."""
-    _need_cuda(x, g)
     rows, cols = x.shape
+    _need_g(g)
+    _need_bytes(codes, cols * (rows // 8) * 4, "codes")
+    _need_bytes(scales, _scale_nbytes(cols, rows // 16, layout), "scales")
+    _need_cuda(x, g, codes, scales)
     if codes is None:
         codes = torch.empty(cols, rows // 8, dtype=torch.int32, device=x.device)
     if scales is None:
@@ -152,8 +186,11 @@ def nvfp4_quantize_columnwise(x: torch.Tensor, g: torch.Tensor | None = None, la
 
 def nvfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, g: torch.Tensor | None = None,
                      layout: str = "linear", dtype=torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
-    _need_cuda(codes, scales, g)
     rows, K = codes.shape[0], codes.shape[1] * 8
+    _need_g(g)
+    _need_bytes(scales, _scale_nbytes(rows, K // 16, layout), "scales")
+    _need_bytes(out, rows * K * (out.element_size() if out is not None else 0), "out")
+    _need_cuda(codes, scales, g, out)
     if out is None:
         out = torch.empty(rows, K, dtype=dtype, device=codes.device)
     dtype = out.dtype
@@ -166,8 +203,11 @@ def nvfp4_quantize_sr(x: torch.Tensor, g: torch.Tensor | None = None, seed: int 
                       codes: torch.Tensor | None = None, scales: torch.Tensor | None = None):
     """nvfp4_quantize with stochastic rounding of the codes (Philox4x32-10
     random bits keyed by ``seed``); scales as nvfp4_quantize."""
-    _need_cuda(x, g)
     rows, K = x.shape
+    _need_g(g)
+    _need_bytes(codes, rows * (K // 8) * 4, "codes")
+    _need_bytes(scales, _scale_nbytes(rows, K // 16, layout), "scales")
+    _need_cuda(x, g, codes, scales)
     if codes is None:
         codes = torch.empty(rows, K // 8, dtype=torch.int32, device=x.device)
     if scales is None:
@@ -178,8 +218,10 @@ def nvfp4_quantize_sr(x: torch.Tensor, g: torch.Tensor | None = None, seed: int 
 
 
 def mxfp8_quantize(x: torch.Tensor, layout: str = "linear", codes=None, scales=None):
-    _need_cuda(x)
     rows, K = x.shape
+    _need_bytes(codes, rows * (K // 4) * 4, "codes")
+    _need_bytes(scales, _scale_nbytes(rows, K // 32, layout), "scales")
+    _need_cuda(x, codes, scales)
     if codes is None:
         codes = torch.empty(rows, K // 4, dtype=torch.int32, device=x.device)
     if scales is None:
@@ -191,8 +233,10 @@ def mxfp8_quantize(x: torch.Tensor, layout: str = "linear", codes=None, scales=N
 
 def mxfp4_quantize(x: torch.Tensor, layout: str = "linear", codes=None, scales=None):
     """(codes int32 [rows, K/8], e8m0 scales uint8) of a 2-D x, 32-element blocks."""
-    _need_cuda(x)
     rows, K = x.shape
+    _need_bytes(codes, rows * (K // 8) * 4, "codes")
+    _need_bytes(scales, _scale_nbytes(rows, K // 32, layout), "scales")
+    _need_cuda(x, codes, scales)
     if codes is None:
         codes = torch.empty(rows, K // 8, dtype=torch.int32, device=x.device)
     if scales is None:
@@ -203,8 +247,9 @@ def mxfp4_quantize(x: torch.Tensor, layout: str = "linear", codes=None, scales=N
 
 
 def mxfp4_dequantize(codes, scales, layout: str = "linear", dtype=torch.bfloat16) -> torch.Tensor:
-    _need_cuda(codes, scales)
     rows, K = codes.shape[0], codes.shape[1] * 8
+    _need_bytes(scales, _scale_nbytes(rows, K // 32, layout), "scales")
+    _need_cuda(codes, scales)
     out = torch.empty(rows, K, dtype=dtype, device=codes.device)
     _check(lib().mxfp4_dequantize(_ptr(codes), _ptr(scales), LAYOUT[layout], rows, K, _ptr(out), DT[dtype],
                                   _stream()))
@@ -212,8 +257,9 @@ def mxfp4_dequantize(codes, scales, layout: str = "linear", dtype=torch.bfloat16
 
 
 def mxfp8_dequantize(codes, scales, layout: str = "linear", dtype=torch.bfloat16) -> torch.Tensor:
-    _need_cuda(codes, scales)
     rows, K = codes.shape[0], codes.shape[1] * 4
+    _need_bytes(scales, _scale_nbytes(rows, K // 32, layout), "scales")
+    _need_cuda(codes, scales)
     out = torch.empty(rows, K, dtype=dtype, device=codes.device)
     _check(lib().mxfp8_dequantize(_ptr(codes), _ptr(scales), LAYOUT[layout], rows, K, _ptr(out), DT[dtype],
                                   _stream()))
@@ -231,8 +277,18 @@ def swizzle_scales(lin: torch.Tensor) -> torch.Tensor:
 def qqmm(a_codes, a_scales, b_codes, b_scales, K: int, mode: str = "nvfp4", g_x=None, g_w=None,
          out_dtype=torch.bfloat16, out: torch.Tensor | None = None) -> torch.Tensor:
     """y [M, N] = x_hat . w_hat^T from quantized operands with SWIZZLED scales."""
-    _need_cuda(a_codes, a_scales, b_codes, b_scales, g_x, g_w)
     M, N = a_codes.shape[0], b_codes.shape[0]
+    if mode in MODE:
+        row_bytes = K if mode == "mxfp8" else K // 2
+        group = 16 if mode == "nvfp4" else 32
+        _need_bytes(a_codes, M * row_bytes, "a_codes")
+        _need_bytes(b_codes, N * row_bytes, "b_codes")
+        _need_bytes(a_scales, _scale_nbytes(M, K // group, "swizzled"), "a_scales")
+        _need_bytes(b_scales, _scale_nbytes(N, K // group, "swizzled"), "b_scales")
+    _need_g(g_x, 1, "g_x")
+    _need_g(g_w, 1, "g_w")
+    _need_bytes(out, M * N * (out.element_size() if out is not None else 0), "out")
+    _need_cuda(a_codes, a_scales, b_codes, b_scales, g_x, g_w, out)
     if out is None:
         out = torch.empty(M, N, dtype=out_dtype, device=a_codes.device)
     _check(lib().qqmm(MODE[mode], M, N, K, _ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales),
@@ -262,9 +318,15 @@ def qqmm_vjp(x: torch.Tensor, w: torch.Tensor, cotan: torch.Tensor, g_x: torch.T
 
 def qmv(x: torch.Tensor, w_codes, w_scales, g_x=None, g_w=None, out=None) -> torch.Tensor:
     """y [M, N] (x's dtype) = x_hat . w_hat^T, M <= 8, w pre-quantized (LINEAR scales)."""
-    _need_cuda(x, w_codes, w_scales, g_x, g_w)
     M, K = x.shape
     N = w_codes.shape[0]
+    _need_bytes(w_codes, N * (K // 8) * 4, "w_codes")
+    _need_bytes(w_scales, N * (K // 16), "w_scales")
+    _need_g(g_x, 1, "g_x")
+    _need_g(g_w, 1, "g_w")
+    _need_dtype(out, x.dtype, "out")
+    _need_bytes(out, M * N * x.element_size(), "out")
+    _need_cuda(x, w_codes, w_scales, g_x, g_w, out)
     if out is None:
         out = torch.empty(M, N, dtype=x.dtype, device=x.device)
     _check(lib().qmv(_ptr(x), DT[x.dtype], _ptr(g_x), _ptr(w_codes), _ptr(w_scales), _ptr(g_w), M, N, K,
@@ -276,22 +338,39 @@ def gather_qmm_workspace_size(T: int, topk: int, E: int) -> int:
     return int(lib().gather_qmm_workspace_size(T, topk, E))
 
 
+def _need_gather(x, w_codes, w_scales, g, idx, out, T, topk, E, N, K, transpose):
+    """Types and sizes the gather entries read and write through raw pointers."""
+    _need_dtype(x, torch.bfloat16, "x")
+    _need_dtype(idx, torch.int32, "idx")
+    _need_bytes(idx, T * topk * 4, "idx")
+    if transpose:
+        _need_bytes(w_codes, E * N * (K // 8) * 4, "w_codes")
+        _need_bytes(w_scales, E * N * (K // 16), "w_scales")
+    else:
+        _need_bytes(w_codes, E * K * (N // 8) * 4, "w_codes")
+        _need_bytes(w_scales, E * K * (N // 16), "w_scales")
+    _need_g(g, E, "g")
+    _need_dtype(out, torch.bfloat16, "out")
+    _need_bytes(out, T * topk * N * 2, "out")
+
+
 def gather_qmm(x, w_codes, w_scales, g, idx, workspace=None, out=None, transpose: bool = True) -> torch.Tensor:
     """y [T, topk, N] bf16.  transpose=True: w_codes [E, N, K/8], w_scales
     LINEAR [E, N, K/16] (y = x . w_hat^T); transpose=False: w_codes
     [E, K, N/8], w_scales LINEAR [E, K, N/16] (y = x . w_hat)."""
-    _need_cuda(x, w_codes, w_scales, g, idx, workspace)
     T, K = x.shape
     topk = idx.shape[1]
     E = w_codes.shape[0]
     N = w_codes.shape[1] if transpose else w_codes.shape[2] * 8
+    _need_gather(x, w_codes, w_scales, g, idx, out, T, topk, E, N, K, transpose)
+    _need_cuda(x, w_codes, w_scales, g, idx, workspace, out)
     if workspace is None:
         workspace = torch.empty(gather_qmm_workspace_size(T, topk, E), dtype=torch.uint8, device=x.device)
     if out is None:
         out = torch.empty(T, topk, N, dtype=torch.bfloat16, device=x.device)
     fn = lib().gather_qmm if transpose else lib().gather_qmm_kn
     _check(fn(_ptr(x), _ptr(w_codes), _ptr(w_scales), _ptr(g), _ptr(idx), T, topk, E, N, K,
-              _ptr(out), _ptr(workspace), workspace.numel(), _stream()))
+              _ptr(out), _ptr(workspace), _nbytes(workspace), _stream()))
     return out
 
 
@@ -300,10 +379,11 @@ def gather_qmm_noalloc(x, w_codes, w_scales, g, idx, out=None) -> torch.Tensor:
     workspace (for callers that cannot allocate device memory); see
     include/nvfp4.h for its size limit and the rule that overlapping calls
     must be serialized."""
-    _need_cuda(x, w_codes, w_scales, g, idx)
     T, K = x.shape
     topk = idx.shape[1]
     E, N = w_codes.shape[0], w_codes.shape[1]
+    _need_gather(x, w_codes, w_scales, g, idx, out, T, topk, E, N, K, True)
+    _need_cuda(x, w_codes, w_scales, g, idx, out)
     if out is None:
         out = torch.empty(T, topk, N, dtype=torch.bfloat16, device=x.device)
     _check(lib().gather_qmm_noalloc(_ptr(x), _ptr(w_codes), _ptr(w_scales), _ptr(g), _ptr(idx), T, topk, E, N, K,
