@@ -233,7 +233,8 @@ NVFP4_API nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, co
  * g [E] fp32 or NULL; idx [T, topk] int32 in [0, E) (checked on the device:
  * out-of-range entries set NVFP4_ERR_DEVICE_INDEX and produce zero rows);
  * y [T, topk, N] bf16.  K % 64 == 0, N % 16 == 0; T*topk, N and K at most
- * 2^30; 1 <= E <= 1024 (more experts: NVFP4_ERR_UNSUPPORTED).
+ * 2^30; 1 <= E <= 1024 and E*N < 2^31 (E*K for gather_qmm_kn), the
+ * weight rows a 32-bit TMA coordinate reaches (beyond: NVFP4_ERR_UNSUPPORTED).
  * workspace: device scratch of gather_qmm_workspace_size(T, topk, E) bytes,
  * 16-byte aligned, contents undefined on entry and exit. */
 NVFP4_API nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const uint8_t* w_scales,

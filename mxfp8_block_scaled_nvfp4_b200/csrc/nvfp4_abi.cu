@@ -453,18 +453,25 @@ size_t gather_qmm_workspace_size(int64_t T, int64_t topk, int64_t E) {
 // Host checks shared by the gather entries: shapes (K % 64, N % n_mult, K > 0
 // when there is output), pointers and, where the caller passes one
 // (check_ws), the workspace size.
-static nvfp4_status check_gather(const char* tag, int n_mult, const void* x, const uint32_t* w_codes,
+static nvfp4_status check_gather(const char* tag, bool kn, const void* x, const uint32_t* w_codes,
                                  const uint8_t* w_scales, const float* g, const int32_t* idx, int64_t T,
                                  int64_t topk, int64_t E, int64_t N, int64_t K, const void* y, bool check_ws,
                                  const void* workspace, size_t workspace_bytes) {
   if (T < 0 || topk < 1 || E < 1 || N < 0 || K < 0 || product_exceeds(T, topk, 1 << 30) || N > (1 << 30) ||
       K > (1 << 30))
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] bad shape", tag);
-  if (E > gq::MAX_E) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] at most %d experts, got %lld", tag, gq::MAX_E, (long long)E);
+  const int n_mult = kn ? 32 : 16;
   if (K % 64 != 0 || N % n_mult != 0)
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] K must be a multiple of 64 and N of %d (K=%lld N=%lld)", tag, n_mult,
                 (long long)K, (long long)N);
   if (K == 0 && T * N > 0) return fail(NVFP4_ERR_INVALID_ARG, "[%s] K must be positive when T*N > 0", tag);
+  if (E > gq::MAX_E) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] at most %d experts, got %lld", tag, gq::MAX_E, (long long)E);
+  // The weight tensor map has E*N rows ([E, N, K]) or E*K rows ([E, K, N]);
+  // TMA row coordinates are 32-bit signed.
+  const int64_t w_rows = E * (kn ? K : N);
+  if (w_rows > INT32_MAX)
+    return fail(NVFP4_ERR_UNSUPPORTED, "[%s] the weights span %lld rows; at most %d", tag, (long long)w_rows,
+                INT32_MAX);
   if (check_ws && workspace_bytes < gather_workspace_bytes(T, topk, E))
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] workspace too small: %zu < %zu", tag, workspace_bytes,
                 gather_workspace_bytes(T, topk, E));
@@ -479,7 +486,7 @@ static nvfp4_status check_gather(const char* tag, int n_mult, const void* x, con
 nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const uint8_t* w_scales, const float* g,
                         const int32_t* idx, int64_t T, int64_t topk, int64_t E, int64_t N, int64_t K, void* y,
                         void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
-  nvfp4_status st = check_gather("gather_qmm", 16, x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, true,
+  nvfp4_status st = check_gather("gather_qmm", false, x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, true,
                                  workspace, workspace_bytes);
   if (st != NVFP4_OK) return st;
   if (T * N == 0) return ok();
@@ -493,7 +500,7 @@ nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const uint8_t* w
 nvfp4_status gather_qmm_kn(const void* x, const uint32_t* w_codes, const uint8_t* w_scales, const float* g,
                         const int32_t* idx, int64_t T, int64_t topk, int64_t E, int64_t N, int64_t K, void* y,
                         void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
-  nvfp4_status st = check_gather("gather_qmm_kn", 32, x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, true,
+  nvfp4_status st = check_gather("gather_qmm_kn", true, x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, true,
                                  workspace, workspace_bytes);
   if (st != NVFP4_OK) return st;
   if (T * N == 0) return ok();
@@ -529,7 +536,7 @@ static nvfp4_status noalloc_scratch(void** out) {
 nvfp4_status gather_qmm_noalloc(const void* x, const uint32_t* w_codes, const uint8_t* w_scales, const float* g,
                                 const int32_t* idx, int64_t T, int64_t topk, int64_t E, int64_t N, int64_t K,
                                 void* y, nvfp4_stream_t stream) {
-  nvfp4_status st = check_gather("gather_qmm_noalloc", 16, x, w_codes, w_scales, g, idx, T, topk, E, N, K, y,
+  nvfp4_status st = check_gather("gather_qmm_noalloc", false, x, w_codes, w_scales, g, idx, T, topk, E, N, K, y,
                                  false, nullptr, 0);
   if (st != NVFP4_OK) return st;
   if (T * N == 0) return ok();

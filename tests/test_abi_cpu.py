@@ -225,3 +225,14 @@ def test_gather_expert_limit_and_workspace_size(L):
     # monotone in T and covers at least the permutation (4 bytes per routed row)
     sizes = [L.gather_qmm_workspace_size(t, 8, 64) for t in (1, 64, 4096)]
     assert sizes == sorted(sizes) and sizes[-1] >= 4 * 4096 * 8
+
+
+def test_gather_weight_rows_fit_32_bit_coordinates(L):
+    """The weight tensor map's rows (E*N, or E*K for [E, K, N]) are addressed
+    by 32-bit signed TMA coordinates: more are refused, not wrapped."""
+    ws = L.gather_qmm_workspace_size(16, 2, 1024)
+    assert L.gather_qmm(A, A, A, A, A, 16, 2, 1024, 1 << 21, 128, A, A, ws, None) == 2  # E*N = 2^31
+    assert "rows" in msg(L)
+    assert L.gather_qmm_kn(A, A, A, A, A, 16, 2, 1024, 64, 1 << 21, A, A, ws, None) == 2  # E*K = 2^31
+    # just under the limit passes the checks (and reaches the device query)
+    assert L.gather_qmm(A, A, A, A, A, 16, 2, 1024, (1 << 21) - 16, 128, A, A, ws, None) not in (0, 1, 2)
