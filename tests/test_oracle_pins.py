@@ -429,3 +429,60 @@ def test_mutation_amax_over_16_not_scaled_by_E_fails_case_B(orc):
     t = a / np.float32(6.0)  # missing * 2688/g
     bytes_ = np.vectorize(lambda v: orc.e4m3_encode(float(v)))(t)
     assert not np.all(bytes_ == 0x38)
+
+
+# ---------------------------------------------------------------------------
+# MX modes of qqmm on exactly representable operands
+# ---------------------------------------------------------------------------
+def _mx_exact_operand(rng, rows, K, mags, top, ks):
+    """rows x K values: per 32-block a power of two 2^k (k from ks), each
+    element a random signed magnitude from ``mags`` times 2^k, and one
+    element +-top*2^k setting the block maximum.  With top = the format's
+    largest magnitude (448 for e4m3, 6 for e2m1) the e8m0 scale of the block
+    is 2^k exactly and every element's code represents it exactly."""
+    v = np.empty((rows, K))
+    kblk = rng.choice(ks, size=(rows, K // 32))
+    for r in range(rows):
+        for b in range(K // 32):
+            blk = rng.choice(mags, 32) * np.where(rng.random(32) < 0.5, -1.0, 1.0)
+            blk[rng.integers(0, 32)] = top * (1.0 if rng.random() < 0.5 else -1.0)
+            v[r, 32 * b:32 * b + 32] = blk * 2.0 ** kblk[r, b]
+    return v.astype(np.float32), kblk
+
+
+def _e4m3_magnitudes():
+    """Every finite e4m3 magnitude from the format's definition: subnormals
+    m/8 2^-6, normals (1 + m/8) 2^(e-7) for e = 1..15 except the NaN code."""
+    vals = [m / 8 * 2.0 ** -6 for m in range(8)]
+    vals += [(1 + m / 8) * 2.0 ** (e - 7) for e in range(1, 16) for m in range(8) if not (e == 15 and m == 7)]
+    return np.array(vals)
+
+
+@pytest.mark.parametrize("mode", ["mxfp8", "mxfp4"])
+def test_mx_qqmm_exact_on_representable_operands(orc, mode):
+    rng = np.random.default_rng(41)
+    M, N, K = 5, 7, 96
+    if mode == "mxfp8":
+        mags, top, quant = _e4m3_magnitudes(), 448.0, orc.mxfp8_quantize
+    else:
+        mags, top, quant = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]), 6.0, orc.mxfp4_quantize
+    x, kx = _mx_exact_operand(rng, M, K, mags, top, [-3, 0, 2])
+    w, kw = _mx_exact_operand(rng, N, K, mags, top, [-1, 1, 4])
+    xq, xs = quant(x, "f32")
+    wq, ws = quant(w, "f32")
+    assert np.array_equal(xs, 127 + kx) and np.array_equal(ws, 127 + kw)
+    r = orc.qqmm(xq, xs, wq, ws, mode, out_dt="f32")
+    assert r["y_ref"].shape == (M, N)
+    np.testing.assert_array_equal(r["y_ref"], x.astype(np.float64) @ w.astype(np.float64).T)
+
+
+def test_mutation_mx_qqmm_without_block_scales_fails_exact_pin(orc):
+    """Mistake: contract the codes' values without the per-block 2^(s-127)
+    (here: decode with every scale byte forced to 127)."""
+    rng = np.random.default_rng(42)
+    x, _ = _mx_exact_operand(rng, 4, 64, _e4m3_magnitudes(), 448.0, [-3, 0, 2])
+    w, _ = _mx_exact_operand(rng, 6, 64, _e4m3_magnitudes(), 448.0, [-1, 1, 4])
+    xq, xs = orc.mxfp8_quantize(x, "f32")
+    wq, ws = orc.mxfp8_quantize(w, "f32")
+    wrong = orc.qqmm(xq, np.full_like(xs, 127), wq, np.full_like(ws, 127), "mxfp8", out_dt="f32")["y_ref"]
+    assert not np.array_equal(wrong, x.astype(np.float64) @ w.astype(np.float64).T)
