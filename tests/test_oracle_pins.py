@@ -486,3 +486,24 @@ def test_mutation_mx_qqmm_without_block_scales_fails_exact_pin(orc):
     wq, ws = orc.mxfp8_quantize(w, "f32")
     wrong = orc.qqmm(xq, np.full_like(xs, 127), wq, np.full_like(ws, 127), "mxfp8", out_dt="f32")["y_ref"]
     assert not np.array_equal(wrong, x.astype(np.float64) @ w.astype(np.float64).T)
+
+
+def test_qmv_quantizes_x_first(orc):
+    """qmv contracts x_hat, not x.  One 16-block x = [6, 2.9, 1.2, 0.7, 0 ...]
+    (bf16), a zero second block, g_x = amax = 6: E = 2688/6 = 448, block scale
+    e4m3(6/6 * 448) = 448, encode factor 1, codes e2m1 of [6, 2.90625,
+    1.203125, 0.69921875] = [6, 3, 1, 0.5] (0.699 is below the 0.75
+    midpoint), decode factor 448 * 6/2688 = 1: x_hat = [6, 3, 1, 0.5].  With
+    every weight 1 (code 0x2, scale 1.0, no global scale) y = 10.5, where the
+    raw x would give bf16(10.80859375) = 10.8125."""
+    K = 32
+    xv = np.zeros((1, K))
+    xv[0, :4] = [6.0, 2.9, 1.2, 0.7]
+    x = bf16(xv)
+    g_x = orc.amax(x, "bf16")
+    assert g_x == 6.0
+    codes = pack_codes(np.full((2, K), 0x2))
+    scales = np.full((2, K // 16), 0x38, dtype=np.uint8)
+    r = orc.qmv(x, "bf16", g_x, codes, scales, None)
+    assert np.all(bf16_value(r["y"]) == 10.5)
+    assert float(bf16_value(x).sum()) == 10.80859375
