@@ -236,3 +236,25 @@ def test_gather_weight_rows_fit_32_bit_coordinates(L):
     assert L.gather_qmm_kn(A, A, A, A, A, 16, 2, 1024, 64, 1 << 21, A, A, ws, None) == 2  # E*K = 2^31
     # just under the limit passes the checks (and reaches the device query)
     assert L.gather_qmm(A, A, A, A, A, 16, 2, 1024, (1 << 21) - 16, 128, A, A, ws, None) not in (0, 1, 2)
+
+
+def test_plain_c_caller(L):
+    """The header compiles as strict C99 and a C program links the library
+    and sees the host-side contract (no CUDA or torch headers involved)."""
+    import shutil
+    import subprocess
+    from mxfp8_block_scaled_nvfp4_b200 import nvfp4
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    out_dir = os.path.join(ROOT, "tests", "_build")
+    os.makedirs(out_dir, exist_ok=True)
+    exe = os.path.join(out_dir, "c_abi_example")
+    lib_dir = os.path.dirname(nvfp4.LIB_PATH)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_example.c"), "-o", exe, "-L", lib_dir,
+                    "-l:" + os.path.basename(nvfp4.LIB_PATH), "-Wl,-rpath," + lib_dir], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.strip().endswith("ok")
+    assert "or neither" in r.stdout
