@@ -34,6 +34,8 @@
  *    fp32 (as the device alpha of [P2] GemmScalars); NULL means none (encode
  *    and decode factors 1).  They are meaningful for NVFP4 only ([P1]
  *    validate_global_scale) and must be finite and > 0.
+ *  - Inputs are finite: the codes, scales and outputs of a block holding a
+ *    NaN or an infinity are unspecified (the pages do not define them).
  *  - Errors: every call returns an nvfp4_status and never throws.  Argument
  *    checks happen on the host before anything is enqueued; on failure
  *    nothing is enqueued and nvfp4_last_error_message() explains.
