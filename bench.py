@@ -37,8 +37,9 @@ events only around the R launches; the roofline's ``achieved`` is work per
 launch over that mean, ``achieved_isolated`` the flushed single call.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs the same step on
-its own GPU (independent problems, no data-path collective): weak scaling;
-the reported time is the max over ranks.
+its own GPU over its own draw of each workload (seed offset = rank; rank 0
+has the workload itself): independent problems, no data-path collective,
+weak scaling; the reported time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -236,11 +237,6 @@ class Row:
         return {k: v / n for k, v in per.items()}, row / n
 
 
-def _gen(wl, name, dev, off):
-    d = wl.make(name, device=dev)
-    return d
-
-
 def _rot(fns, n):
     """n calls cycling through the callables fns (one per operand copy)."""
     return [fns[i % len(fns)] for i in range(n)]
@@ -254,7 +250,7 @@ class Quant1G(Row):
         return [lambda: self.nv.nvfp4_quantize(self.x, self.g, "swizzled", self.codes, self.scales)] * 2
 
     def setup(self):
-        self.x = self.wl.make("quant1g", device=self.dev)["x"]
+        self.x = self.wl.make("quant1g", device=self.dev, seed_offset=self.off)["x"]
         R, K = self.x.shape
         self.g = torch.empty(1, dtype=torch.float32, device=self.dev)
         self.codes = torch.empty(R, K // 8, dtype=torch.int32, device=self.dev)
@@ -306,7 +302,7 @@ class Gemv(Row):
         return _rot([lambda c=c: self.nv.qmv(self.x, c[0], c[1], self.g_x, self.g_w, self.y) for c in cps], 12)
 
     def setup(self):
-        d = self.wl.make("gemv", device=self.dev)
+        d = self.wl.make("gemv", device=self.dev, seed_offset=self.off)
         self.x, w = d["x"], d["w"]
         self.g_x = torch.empty(1, dtype=torch.float32, device=self.dev)
         self.g_w = self.nv.amax(w)
@@ -339,7 +335,7 @@ class Dequant(Row):
                      for c in cps], 6)
 
     def setup(self):
-        w = self.wl.make("gemv", device=self.dev)["w"]
+        w = self.wl.make("gemv", device=self.dev, seed_offset=self.off)["w"]
         g = self.nv.amax(w)
         self.g = g
         self.wc, self.ws = self.nv.nvfp4_quantize(w, g, "linear")
@@ -370,7 +366,7 @@ class Prefill(Row):
                                               out=self.y) for c in cps], 16)
 
     def setup(self):
-        d = self.wl.make("prefill", device=self.dev)
+        d = self.wl.make("prefill", device=self.dev, seed_offset=self.off)
         self.x, self.w = d["x"], d["w"]
         self.M, self.K = self.x.shape
         self.N = self.w.shape[0]
@@ -421,7 +417,7 @@ class PrefillBwd(Row):
                      for c in cps], 16)
 
     def setup(self):
-        d = self.wl.make("prefill_bwd", device=self.dev)
+        d = self.wl.make("prefill_bwd", device=self.dev, seed_offset=self.off)
         self.x, self.w, self.c = d["x"], d["w"], d["cotan"]
         M, K = self.x.shape
         N = self.w.shape[0]
@@ -470,7 +466,7 @@ class Moe(Row):
                                                     transpose=self.b2b_transpose) for c in cps], 4)
 
     def setup(self):
-        d = self.wl.make("moe", device=self.dev)
+        d = self.wl.make("moe", device=self.dev, seed_offset=self.off)
         self.x, w, self.idx = d["x"], d["w"], d["idx"]
         E, N, K = w.shape
         self.E, self.N, self.K = E, N, K
@@ -512,7 +508,7 @@ class MoeKN(Moe):
     b2b_transpose = False
 
     def setup(self):
-        d = self.wl.make("moe", device=self.dev)
+        d = self.wl.make("moe", device=self.dev, seed_offset=self.off)
         self.x, w, self.idx = d["x"], d["w"], d["idx"]
         E, N, K = w.shape
         self.E, self.N, self.K = E, N, K
@@ -558,7 +554,7 @@ class MoeDecode(Row):
                      for c in cps], 8)
 
     def setup(self):
-        d = self.wl.make("moe", device=self.dev)
+        d = self.wl.make("moe", device=self.dev, seed_offset=self.off)
         x, w, idx = d["x"], d["w"], d["idx"]
         E, N, K = w.shape
         self.E, self.N, self.K = E, N, K
@@ -602,7 +598,7 @@ class Mxfp8(Row):
         return [lambda: self.nv.qqmm(self.xc, self.xs, self.wc, self.ws, self.K, "mxfp8", out=self.y)] * 2
 
     def setup(self):
-        d = self.wl.make("mxfp8", device=self.dev)
+        d = self.wl.make("mxfp8", device=self.dev, seed_offset=self.off)
         self.x, self.w = d["x"], d["w"]
         self.M, self.K = self.x.shape
         self.N = self.w.shape[0]
@@ -643,7 +639,7 @@ class Mxfp4(Row):
         return _rot([lambda c=c: self.nv.qqmm(*c, self.K, "mxfp4", out=self.y) for c in cps], 4)
 
     def setup(self):
-        d = self.wl.make("mxfp4", device=self.dev)
+        d = self.wl.make("mxfp4", device=self.dev, seed_offset=self.off)
         self.x, self.w = d["x"], d["w"]
         self.M, self.K = self.x.shape
         self.N = self.w.shape[0]

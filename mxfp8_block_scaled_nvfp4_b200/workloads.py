@@ -79,13 +79,17 @@ def routing(T: int, E: int, topk: int, seed: int, device="cpu") -> torch.Tensor:
     return torch.argsort(keys, dim=1)[:, :topk].to(torch.int32).contiguous()
 
 
-def make(name: str, device="cpu", scale_down: int = 1) -> dict:
+def make(name: str, device="cpu", scale_down: int = 1, seed_offset: int = 0) -> dict:
     """Inputs of a named workload.  ``scale_down`` > 1 divides the large
-    dimensions (for CPU-sized variants with the same distributions)."""
+    dimensions (for CPU-sized variants with the same distributions).
+    ``seed_offset`` k > 0 draws another instance of the same workload (every
+    seed s becomes s + 1000 k): one per rank when each rank solves its own
+    problem; k = 0 is the workload itself."""
     w = WORKLOADS[name]
     sd = max(1, int(scale_down))
+    seeds = tuple(s + 1000 * int(seed_offset) for s in w["seeds"])
     if name == "tiny":
-        g = _gen(w["seeds"][0], device)
+        g = _gen(seeds[0], device)
         x = torch.randn(w["M"], w["K"], generator=g, device=device, dtype=torch.float32)
         W = torch.randn(w["N"], w["K"], generator=g, device=device, dtype=torch.float32)
         return {"x": x, "w": W}
@@ -93,7 +97,7 @@ def make(name: str, device="cpu", scale_down: int = 1) -> dict:
         M, N, K = w["M"], w["N"], w["K"]
         if sd > 1:
             M, N = max(1, M // sd), max(1, N // sd)
-        s0, s1 = w["seeds"]
+        s0, s1 = seeds
         std_w = 0.02 if name in ("gemv", "prefill") else 1.0
         x = normal((M, K), 1.0, s0, w["dtype"], device)
         if name == "prefill":
@@ -105,19 +109,19 @@ def make(name: str, device="cpu", scale_down: int = 1) -> dict:
         T, E, topk, N, K = w["T"], w["E"], w["topk"], w["N"], w["K"]
         if sd > 1:
             T, N = max(1, T // sd), max(8, N // sd)
-        s_w, s_x, s_i = w["seeds"]
+        s_w, s_x, s_i = seeds
         W = normal((E, N, K), 0.02, s_w, w["dtype"], device)
         x = normal((T, K), 1.0, s_x, w["dtype"], device)
         idx = routing(T, E, topk, s_i, device)
         return {"x": x, "w": W, "idx": idx}
     if name == "prefill_bwd":
-        d = make("prefill", device=device, scale_down=sd)
+        d = make("prefill", device=device, scale_down=sd, seed_offset=seed_offset)
         M, N = d["x"].shape[0], d["w"].shape[0]
-        d["cotan"] = normal((M, N), 1.0, w["seeds"][2], w["dtype"], device)
+        d["cotan"] = normal((M, N), 1.0, seeds[2], w["dtype"], device)
         return d
     if name == "quant1g":
         R, K = w["R"], w["K"]
         if sd > 1:
             R = max(1, R // sd)
-        return {"x": normal((R, K), 1.0, w["seeds"][0], w["dtype"], device)}
+        return {"x": normal((R, K), 1.0, seeds[0], w["dtype"], device)}
     raise KeyError(name)

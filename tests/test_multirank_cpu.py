@@ -41,3 +41,19 @@ def test_two_gloo_ranks_max_and_whole_job():
                        start_method="spawn")
     assert out[:world].tolist() == [2.5, 2.5]
     assert out[world:].tolist() == pytest.approx([8.0, 8.0])
+
+
+def test_each_rank_draws_its_own_instance():
+    """bench.py builds every row with seed_offset = rank: rank 0 gets the
+    workload itself, other ranks another draw of the same shapes and
+    distributions (weak scaling: no two ranks solve the same problem)."""
+    from mxfp8_block_scaled_nvfp4_b200 import workloads
+    for name in ["tiny", "gemv", "prefill", "moe", "quant1g", "prefill_bwd"]:
+        sd = 1 if name in ("tiny", "gemv") else 32
+        r0 = workloads.make(name, scale_down=sd)
+        r0b = workloads.make(name, scale_down=sd, seed_offset=0)
+        r1 = workloads.make(name, scale_down=sd, seed_offset=1)
+        for k in r0:
+            assert torch.equal(r0[k], r0b[k])
+            assert r1[k].shape == r0[k].shape and r1[k].dtype == r0[k].dtype
+            assert not torch.equal(r0[k], r1[k]), (name, k)
