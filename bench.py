@@ -680,6 +680,9 @@ def dist_setup(n_gpus):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if n_gpus != world:
+        raise SystemExit(f"--gpus {n_gpus} but {world} process(es): launch N > 1 with torchrun "
+                         f"--nproc-per-node N (one process per GPU)")
     if world > 1:
         import datetime
         torch.cuda.set_device(local)

@@ -304,8 +304,7 @@ def qqmm_vjp(x: torch.Tensor, w: torch.Tensor, cotan: torch.Tensor, g_x: torch.T
     x [M, K], w [N, K], cotan [M, N] bf16/fp16/fp32; M, N multiples of 32.
     Every step is one ABI call (amax, quantize, column-wise quantize, qqmm)."""
     _need_cuda(x, w, cotan, g_x, g_w)
-    M, K = x.shape
-    N = w.shape[0]
+    M, N = x.shape[0], w.shape[0]
     g_c = amax(cotan)
     c_codes, c_scales = nvfp4_quantize(cotan, g_c, "swizzled")                # [M, N/8]
     wt_codes, wt_scales = nvfp4_quantize_columnwise(w, g_w, "swizzled")      # w^T [K, N/8]
