@@ -965,7 +965,8 @@ def run_ours(args):
                           "recorded inside the graph before and after every call; each row's roofline kernel "
                           "also launched back to back over operand copies larger than L2, events around the "
                           "launches (roofline achieved; achieved_isolated is the flushed single call)",
-                "parallelism": f"{world} independent replicas" if world > 1 else "1 GPU"},
+                "parallelism": f"{world} ranks, each its own draw of every workload (no collective)" if world > 1
+                               else "1 GPU"},
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
