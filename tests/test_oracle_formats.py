@@ -137,7 +137,8 @@ def test_e2m1_ties_and_signs(orc):
 def test_e8m0_ceil_defining_inequalities(orc):
     rng = np.random.default_rng(0)
     exps = rng.uniform(-140, 130, size=4000)
-    vals = np.float32(np.exp2(exps))
+    with np.errstate(over="ignore"):  # draws above 2^128 become inf and are skipped below
+        vals = np.float32(np.exp2(exps))
     vals = np.concatenate([vals, np.float32(np.exp2(np.arange(-126, 128)))])
     for v in vals:
         v = float(v)
