@@ -90,12 +90,22 @@ def _stream():
 
 
 def _need_cuda(*ts):
+    """Every tensor is a contiguous CUDA tensor on the current device: the
+    library launches on the current device and the current stream, so a
+    tensor of another GPU would be read through a pointer that GPU's kernels
+    cannot use."""
+    dev = None
     for t in ts:
         if t is not None:
             if not t.is_cuda:
                 raise ValueError("tensors must be CUDA tensors (no CPU fallback)")
             if not t.is_contiguous():
                 raise ValueError("tensors must be contiguous")
+            if dev is None:
+                dev = torch.cuda.current_device()
+            if t.device.index != dev:
+                raise ValueError(f"tensor on {t.device}, but the current device is cuda:{dev}; "
+                                 "call under torch.cuda.device(tensor.device)")
 
 
 def _nbytes(t) -> int:

@@ -241,6 +241,23 @@ static float encode_factor(const float* g) {
   return g ? (448.0f * 6.0f) / *g : 1.0f;
 }
 
+/* Scale byte of one block from its amax a: t = a / 6 first, then t * E,
+ * each rounded to fp32 ([P2] fp_quantize_rowwise computes the block maximum
+ * over 6 and multiplies by the encode factor). */
+static int nvfp4_scale_byte(float a, float E) {
+  float t = a / 6.0f;
+  t = t * E;
+  return orc_e4m3_rne_satfinite(t);
+}
+
+/* Value handed to the e2m1 encoder: the factor k = E / f8(s) first, then
+ * x * k, each rounded to fp32 ([P2] fp_quantize_rowwise divides the encode
+ * factor by the block scale once and multiplies every element by it). */
+static float nvfp4_scaled_value(float x, float E, float fs) {
+  float k = E / fs;
+  return x * k;
+}
+
 void orc_nvfp4_quantize(const void* x, int dt, int64_t rows, int64_t K,
                         const float* g, uint32_t* codes, uint8_t* scales) {
   const float E = encode_factor(g);
@@ -253,16 +270,13 @@ void orc_nvfp4_quantize(const void* x, int dt, int64_t rows, int64_t K,
         xv[i] = (float)orc_load(x, dt, r * K + b * 16 + i);
         if (fabsf(xv[i]) > a) a = fabsf(xv[i]);
       }
-      float t = a / 6.0f;
-      t = t * E;
-      int s = orc_e4m3_rne_satfinite(t);
+      int s = nvfp4_scale_byte(a, E);
       scales[r * nb + b] = (uint8_t)s;
       float fs = (float)orc_e4m3_value(s);
       uint32_t w[2] = {0, 0};
       if (fs != 0.0f) {
-        float k = E / fs;
         for (int i = 0; i < 16; ++i) {
-          uint32_t q = (uint32_t)orc_e2m1_rne_satfinite(xv[i] * k);
+          uint32_t q = (uint32_t)orc_e2m1_rne_satfinite(nvfp4_scaled_value(xv[i], E, fs));
           w[i / 8] |= q << (4 * (i % 8));
         }
       }
@@ -568,17 +582,14 @@ void orc_nvfp4_quantize_sr(const void* x, int dt, int64_t rows, int64_t K, const
         xv[i] = (float)orc_load(x, dt, r * K + b * 16 + i);
         if (fabsf(xv[i]) > a) a = fabsf(xv[i]);
       }
-      float t = a / 6.0f;
-      t = t * E;
-      int s = orc_e4m3_rne_satfinite(t);
+      int s = nvfp4_scale_byte(a, E);
       scales[r * nb + b] = (uint8_t)s;
       float fs = (float)orc_e4m3_value(s);
       uint32_t w[2] = {0, 0};
       if (fs != 0.0f) {
-        float k = E / fs;
         for (int i = 0; i < 16; ++i) {
           const uint64_t idx = (uint64_t)(r * K + b * 16 + i);
-          uint32_t q = (uint32_t)orc_e2m1_sr_satfinite(xv[i] * k, orc_sr_bits(seed, idx));
+          uint32_t q = (uint32_t)orc_e2m1_sr_satfinite(nvfp4_scaled_value(xv[i], E, fs), orc_sr_bits(seed, idx));
           w[i / 8] |= q << (4 * (i % 8));
         }
       }

@@ -53,56 +53,67 @@ def build(force: bool = False) -> str:
     os.makedirs(_BUILD, exist_ok=True)
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
-        subprocess.check_call([
-            "gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-ffp-contract=off",
-            "-fno-fast-math", "-fexcess-precision=standard", "-o", tmp, _SRC, "-lm",
-        ])
+        compile_source(_SRC, tmp)
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
+
+
+def compile_source(src: str, out: str) -> None:
+    """gcc with the oracle's flags: C11, no FMA contraction, no fast-math,
+    float expressions evaluated in their own type.  The mutation tests build
+    edited copies of nvfp4_oracle.c with it."""
+    subprocess.check_call([
+        "gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-ffp-contract=off",
+        "-fno-fast-math", "-fexcess-precision=standard", "-o", out, src, "-lm",
+    ])
 
 
 def _L():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
-            P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
-            sig = {
-                "orc_e2m1_value": (ctypes.c_double, [I]),
-                "orc_e4m3_value": (ctypes.c_double, [I]),
-                "orc_e8m0_value": (ctypes.c_double, [I]),
-                "orc_e2m1_rne_satfinite": (I, [ctypes.c_float]),
-                "orc_e4m3_rne_satfinite": (I, [ctypes.c_float]),
-                "orc_e8m0_ceil": (I, [ctypes.c_float]),
-                "orc_round_to_format": (ctypes.c_double, [ctypes.c_double, I, I, ctypes.c_double]),
-                "orc_round_to_type": (ctypes.c_double, [ctypes.c_double, I]),
-                "orc_amax": (ctypes.c_float, [P, I, I64]),
-                "orc_nvfp4_quantize": (None, [P, I, I64, I64, P, P, P]),
-                "orc_nvfp4_block_scale": (ctypes.c_float, [ctypes.c_uint8, P]),
-                "orc_nvfp4_dequantize": (None, [P, P, I64, I64, P, P, I]),
-                "orc_nvfp4_decode_exact": (None, [P, P, I64, I64, P, P]),
-                "orc_nvfp4_decode_blockscale": (None, [P, P, I64, I64, P, P]),
-                "orc_nvfp4_quantize_dequantize": (None, [P, I, I64, I64, P, P]),
-                "orc_mxfp8_quantize": (None, [P, I, I64, I64, P, P]),
-                "orc_mxfp8_dequantize": (None, [P, P, I64, I64, P, I]),
-                "orc_mxfp8_decode_exact": (None, [P, P, I64, I64, P]),
-                "orc_mxfp4_quantize": (None, [P, I, I64, I64, P, P]),
-                "orc_philox4x32_10": (None, [P, P, P]),
-                "orc_sr_bits": (ctypes.c_uint32, [ctypes.c_uint64, ctypes.c_uint64]),
-                "orc_e2m1_sr_satfinite": (I, [ctypes.c_float, ctypes.c_uint32]),
-                "orc_nvfp4_quantize_sr": (None, [P, I, I64, I64, P, ctypes.c_uint64, P, P]),
-                "orc_mxfp4_dequantize": (None, [P, P, I64, I64, P, I]),
-                "orc_mxfp4_decode_exact": (None, [P, P, I64, I64, P]),
-                "orc_swizzle_scales": (None, [P, I64, I64, P]),
-                "orc_load_array": (None, [P, I, I64, P]),
-                "orc_store_array": (None, [P, I64, I, P]),
-            }
-            for name, (res, args) in sig.items():
-                f = getattr(lib, name)
-                f.restype = res
-                f.argtypes = args
-            _lib = lib
+            _lib = bind(ctypes.CDLL(build()))
         return _lib
+
+
+def bind(lib):
+    """Declare the C signatures on a loaded copy of the oracle library."""
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    sig = {
+        "orc_e2m1_value": (ctypes.c_double, [I]),
+        "orc_e4m3_value": (ctypes.c_double, [I]),
+        "orc_e8m0_value": (ctypes.c_double, [I]),
+        "orc_e2m1_rne_satfinite": (I, [ctypes.c_float]),
+        "orc_e4m3_rne_satfinite": (I, [ctypes.c_float]),
+        "orc_e8m0_ceil": (I, [ctypes.c_float]),
+        "orc_round_to_format": (ctypes.c_double, [ctypes.c_double, I, I, ctypes.c_double]),
+        "orc_round_to_type": (ctypes.c_double, [ctypes.c_double, I]),
+        "orc_amax": (ctypes.c_float, [P, I, I64]),
+        "orc_nvfp4_quantize": (None, [P, I, I64, I64, P, P, P]),
+        "orc_nvfp4_block_scale": (ctypes.c_float, [ctypes.c_uint8, P]),
+        "orc_nvfp4_dequantize": (None, [P, P, I64, I64, P, P, I]),
+        "orc_nvfp4_decode_exact": (None, [P, P, I64, I64, P, P]),
+        "orc_nvfp4_decode_blockscale": (None, [P, P, I64, I64, P, P]),
+        "orc_nvfp4_quantize_dequantize": (None, [P, I, I64, I64, P, P]),
+        "orc_mxfp8_quantize": (None, [P, I, I64, I64, P, P]),
+        "orc_mxfp8_dequantize": (None, [P, P, I64, I64, P, I]),
+        "orc_mxfp8_decode_exact": (None, [P, P, I64, I64, P]),
+        "orc_mxfp4_quantize": (None, [P, I, I64, I64, P, P]),
+        "orc_philox4x32_10": (None, [P, P, P]),
+        "orc_sr_bits": (ctypes.c_uint32, [ctypes.c_uint64, ctypes.c_uint64]),
+        "orc_e2m1_sr_satfinite": (I, [ctypes.c_float, ctypes.c_uint32]),
+        "orc_nvfp4_quantize_sr": (None, [P, I, I64, I64, P, ctypes.c_uint64, P, P]),
+        "orc_mxfp4_dequantize": (None, [P, P, I64, I64, P, I]),
+        "orc_mxfp4_decode_exact": (None, [P, P, I64, I64, P]),
+        "orc_swizzle_scales": (None, [P, I64, I64, P]),
+        "orc_load_array": (None, [P, I, I64, P]),
+        "orc_store_array": (None, [P, I64, I, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
 
 
 def _p(a: np.ndarray):

@@ -98,3 +98,25 @@ def test_gather_operands():
     wkn, skn = e(E, K, N // 8, dtype=i32), e(E, K, N // 16)
     reaches_cuda_check(nv.gather_qmm, x, wkn, skn, None, idx, transpose=False)
     refused(nv.gather_qmm, x, wkn, skn[:, :-1].contiguous(), None, idx, transpose=False, match="w_scales")
+
+
+class _OnDevice:
+    """Stand-in for a contiguous CUDA tensor on a given device (no GPU here)."""
+    is_cuda = True
+
+    def __init__(self, index):
+        self.device = torch.device("cuda", index)
+
+    def is_contiguous(self):
+        return True
+
+
+def test_tensors_on_another_device_are_refused(monkeypatch):
+    # the library launches on the current device: a tensor of another GPU
+    # would be read there through a pointer that device cannot use
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    nv._need_cuda(_OnDevice(0), None, _OnDevice(0))
+    refused(nv._need_cuda, _OnDevice(0), _OnDevice(1), match="current device is cuda:0")
+    refused(nv._need_cuda, _OnDevice(1), match="torch.cuda.device")
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 1)
+    nv._need_cuda(_OnDevice(1), _OnDevice(1))

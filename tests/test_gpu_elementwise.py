@@ -49,6 +49,27 @@ def test_nvfp4_quantize_parity(nv, orc, dt, shape, use_g, layout):
     assert np.array_equal(raw(scales), want_s)
 
 
+@pytest.mark.parametrize("tag", ["r1", "r2"])
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_nvfp4_quantize_operation_order_blocks(nv, tag, dt):
+    """The hand-derived blocks on which the fp32 order of the scale step (r1)
+    or the code step (r2) changes the result: the kernel gives the bytes and
+    codes of "mlx 0.30.7.2 -> 0.30.7.6" page 7 fp_quantize_rowwise's order
+    (tests/golden/quantize_operation_order.txt), with round-to-nearest and,
+    for the scale byte, with stochastic rounding."""
+    from test_oracle_operation_order import _block, _unpack
+    g, x, scale, codes = _block(tag)
+    xg = torch.from_numpy(x).to(TORCH_DT[dt]).cuda()
+    gg = torch.tensor([g], dtype=torch.float32, device="cuda")
+    q, s = nv.nvfp4_quantize(xg, gg, "linear")
+    torch.cuda.synchronize()
+    assert int(raw(s).reshape(-1)[0]) == scale
+    assert _unpack(raw(q)) == codes
+    _, s_sr = nv.nvfp4_quantize_sr(xg, gg, 7, "linear")
+    torch.cuda.synchronize()
+    assert int(raw(s_sr).reshape(-1)[0]) == scale
+
+
 @pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
 @pytest.mark.parametrize("out_dt", ["f32", "f16", "bf16"])
 @pytest.mark.parametrize("layout", ["linear", "swizzled"])
