@@ -107,6 +107,23 @@ NVFP4_API size_t nvfp4_scale_bytes(int64_t rows, int64_t cols, nvfp4_layout layo
 NVFP4_API nvfp4_status nvfp4_amax(const void* x, nvfp4_dtype dt, int64_t n, float* g_out,
                         nvfp4_stream_t stream);
 
+/* a1 for several tensors in one launch: the raw-operand qqmm takes the amax
+ * of both operands before quantizing them ([P1] qqmm; [P2]
+ * compute_qqmm_pointers reads tensor_amax_x and tensor_amax_w).  items[i]
+ * holds x (n elements of dt, 16-byte aligned) and g_out (device fp32,
+ * overwritten with max |x|, 0 for n = 0); 1 <= count <= 4; the outputs must
+ * be distinct (one memset clears them when they are consecutive floats).
+ * The items array is read on the host during the call.  Same checks and
+ * errors as nvfp4_amax, per item. */
+typedef struct {
+  const void* x;
+  int64_t n;
+  float* g_out;
+} nvfp4_amax_item;
+
+NVFP4_API nvfp4_status nvfp4_amax_multi(const nvfp4_amax_item* items, int count, nvfp4_dtype dt,
+                                        nvfp4_stream_t stream);
+
 /* a2-a4 -- NVFP4 two-level quantize ([P2] fp_quantize_rowwise with global
  * scale).  Per row, per 16-element block along K:
  *   E = 2688 / g (1 if g == NULL);  s = e4m3_rne_satfinite((amax/6) * E);
@@ -125,6 +142,26 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dt, int64_t row
 NVFP4_API nvfp4_status nvfp4_dequantize(const uint32_t* codes, const uint8_t* scales,
                               nvfp4_layout layout, int64_t rows, int64_t K, const float* g,
                               void* out, nvfp4_dtype out_dt, nvfp4_stream_t stream);
+
+/* nvfp4_quantize of several tensors in one launch (the raw-operand qqmm
+ * quantizes x and w, [P1] qqmm).  items[i] holds the arguments of one
+ * nvfp4_quantize call (x [rows, K] of dt, g, codes, scales, layout); every
+ * item gets exactly the codes and scales nvfp4_quantize would write.
+ * 1 <= count <= 4; items must not write overlapping buffers.  The items
+ * array is read on the host during the call.  Each item is checked as
+ * nvfp4_quantize checks its arguments; items with no element are skipped. */
+typedef struct {
+  const void* x;
+  int64_t rows;
+  int64_t K;
+  const float* g;
+  uint32_t* codes;
+  uint8_t* scales;
+  nvfp4_layout layout;
+} nvfp4_quantize_item;
+
+NVFP4_API nvfp4_status nvfp4_quantize_multi(const nvfp4_quantize_item* items, int count, nvfp4_dtype dt,
+                                            nvfp4_stream_t stream);
 
 /* f1 -- column-wise NVFP4 quantize ([P2] fp_quantize_columnwise: an M-major
  * matrix quantized along its last dimension): x [rows, cols] row-major is
@@ -277,8 +314,11 @@ NVFP4_API size_t gather_qmm_workspace_size(int64_t T, int64_t topk, int64_t E);
  * cudaMalloc, no cudaFree, no allocating library routine.
  *
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture.  All calls on a device share the
+ * (cudaGetSymbolAddress, with that device current) and caches it with the
+ * identity of the device's context; make that first call before any stream
+ * capture.  A later context on the device (after cudaDeviceReset, which
+ * unloads the array) makes the next call look the address up again, so
+ * that call too belongs outside a capture.  All calls on a device share the
  * one array, which keeps the previous call's contents (each call rewrites
  * every entry it reads, so nothing has to be cleared); two calls whose
  * kernels overlap on the GPU -- on different streams, or from different

@@ -49,21 +49,20 @@ template <> struct Elem<__nv_bfloat16> {
   static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
 };
 
-// Load 8 consecutive elements (16 B for 2-byte types, 32 B for fp32) as fp32.
+// 8 consecutive elements held in one 16-byte word (2-byte types) or two
+// (fp32), as fp32.
 template <typename T>
-__device__ __forceinline__ void load8(const T* p, float (&v)[8]);
+__device__ __forceinline__ void unpack8(uint4 a, uint4 b, float (&v)[8]);
 
 template <>
-__device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
-  float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+__device__ __forceinline__ void unpack8<float>(uint4 a, uint4 b, float (&v)[8]) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(w[i]);
 }
 
 template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
-  uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+__device__ __forceinline__ void unpack8<__nv_bfloat16>(uint4 u, uint4, float (&v)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -73,8 +72,7 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, flo
 }
 
 template <>
-__device__ __forceinline__ void load8<__half>(const __half* p, float (&v)[8]) {
-  uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+__device__ __forceinline__ void unpack8<__half>(uint4 u, uint4, float (&v)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -82,6 +80,21 @@ __device__ __forceinline__ void load8<__half>(const __half* p, float (&v)[8]) {
         : "=f"(v[2 * i]), "=f"(v[2 * i + 1])
         : "r"(w[i]));
   }
+}
+
+// Load 8 consecutive elements (16 B for 2-byte types, 32 B for fp32) of
+// global memory as fp32 (read-only path).
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&v)[8]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+  unpack8<T>(__ldg(q), sizeof(T) == 4 ? __ldg(q + 1) : make_uint4(0, 0, 0, 0), v);
+}
+
+// The same from shared memory (generic loads).
+template <typename T>
+__device__ __forceinline__ void load8_shared(const T* p, float (&v)[8]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+  unpack8<T>(q[0], sizeof(T) == 4 ? q[1] : make_uint4(0, 0, 0, 0), v);
 }
 
 // Store 8 fp32 values rounded to T (RNE).

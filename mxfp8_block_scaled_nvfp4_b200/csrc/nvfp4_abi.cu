@@ -152,31 +152,68 @@ size_t nvfp4_scale_bytes(int64_t rows, int64_t cols, nvfp4_layout layout) {
   return (size_t)(((rows + 127) / 128 * 128) * ((cols + 3) / 4 * 4));
 }
 
-nvfp4_status nvfp4_amax(const void* x, nvfp4_dtype dt, int64_t n, float* g_out, nvfp4_stream_t stream) {
-  if (!valid_dt(dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[amax] dtype must be float32, float16 or bfloat16");
-  if (n < 0 || n > kMaxElems) return fail(NVFP4_ERR_INVALID_ARG, "[amax] bad size %lld", (long long)n);
-  if (!g_out || (n > 0 && !x)) return fail(NVFP4_ERR_INVALID_ARG, "[amax] null pointer");
-  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(g_out) & 3u))
-    return fail(NVFP4_ERR_INVALID_ARG, "[amax] x must be 16-byte aligned, g_out 4-byte aligned");
+static nvfp4_status amax_launch(const char* tag, const nvfp4_amax_item* items, int count, nvfp4_dtype dt,
+                                nvfp4_stream_t stream) {
+  if (!valid_dt(dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] dtype must be float32, float16 or bfloat16", tag);
+  if (!items || count < 1 || count > kAmaxSegs)
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] between 1 and %d tensors, got %d", tag, kAmaxSegs, count);
+  for (int i = 0; i < count; ++i) {
+    const nvfp4_amax_item& it = items[i];
+    if (it.n < 0 || it.n > kMaxElems) return fail(NVFP4_ERR_INVALID_ARG, "[%s] bad size %lld", tag, (long long)it.n);
+    if (!it.g_out || (it.n > 0 && !it.x)) return fail(NVFP4_ERR_INVALID_ARG, "[%s] null pointer", tag);
+    if (!aligned16(it.x) || (reinterpret_cast<uintptr_t>(it.g_out) & 3u))
+      return fail(NVFP4_ERR_INVALID_ARG, "[%s] x must be 16-byte aligned, g_out 4-byte aligned", tag);
+    for (int j = 0; j < i; ++j)
+      if (items[j].g_out == it.g_out) return fail(NVFP4_ERR_INVALID_ARG, "[%s] two tensors share one output", tag);
+  }
   DeviceInfo d;
-  nvfp4_status st = device_info("amax", &d);
+  nvfp4_status st = device_info(tag, &d);
   if (st != NVFP4_OK) return st;
-  cudaError_t e = cudaMemsetAsync(g_out, 0, sizeof(float), stream);
-  if (e != cudaSuccess) return fail(NVFP4_ERR_CUDA, "[amax] memset: %s", cudaGetErrorString(e));
-  if (n == 0) return ok();
-  const unsigned grid = ew_grid(d, (uint64_t)(n / 8 + 1));
-  dispatch_dt(dt, [&](auto tag) {
-    using T = decltype(tag);
-    k_amax<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n, g_out);
+  // outputs start at 0 (max |x| >= 0); one memset when they are consecutive floats
+  bool consecutive = true;
+  for (int i = 1; i < count; ++i) consecutive = consecutive && items[i].g_out == items[0].g_out + i;
+  cudaError_t e = cudaSuccess;
+  if (consecutive) {
+    e = cudaMemsetAsync(items[0].g_out, 0, sizeof(float) * (size_t)count, stream);
+  } else {
+    for (int i = 0; i < count && e == cudaSuccess; ++i) e = cudaMemsetAsync(items[i].g_out, 0, sizeof(float), stream);
+  }
+  if (e != cudaSuccess) return fail(NVFP4_ERR_CUDA, "[%s] memset: %s", tag, cudaGetErrorString(e));
+  AmaxSegs a;
+  memset(&a, 0, sizeof(a));
+  uint64_t vecs = 0;
+  for (int i = 0; i < count; ++i) {
+    if (items[i].n == 0) continue;  // its output stays 0
+    a.x[a.count] = items[i].x;
+    a.n[a.count] = items[i].n;
+    a.out[a.count] = items[i].g_out;
+    ++a.count;
+    vecs += (uint64_t)(items[i].n / 8 + 1);
+  }
+  if (a.count == 0) return ok();
+  const unsigned grid = ew_grid(d, (vecs + 3) / 4);
+  dispatch_dt(dt, [&](auto tag_t) {
+    using T = decltype(tag_t);
+    k_amax<T><<<grid, kEwThreads, 0, stream>>>(a);
   });
-  return check_launch("amax");
+  return check_launch(tag);
 }
 
-// kind: 0 NVFP4, 1 MXFP8, 2 MXFP4 (the two MX kinds use 32-element blocks)
-static nvfp4_status quantize_common(const char* tag, int kind, const void* x, nvfp4_dtype dt,
-                                    int64_t rows, int64_t K, const float* g, uint32_t* codes,
-                                    uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream,
-                                    bool sr = false, uint64_t seed = 0) {
+nvfp4_status nvfp4_amax(const void* x, nvfp4_dtype dt, int64_t n, float* g_out, nvfp4_stream_t stream) {
+  const nvfp4_amax_item it{x, n, g_out};
+  return amax_launch("amax", &it, 1, dt, stream);
+}
+
+nvfp4_status nvfp4_amax_multi(const nvfp4_amax_item* items, int count, nvfp4_dtype dt, nvfp4_stream_t stream) {
+  return amax_launch("amax_multi", items, count, dt, stream);
+}
+
+// Argument checks of one row-wise quantize; *empty is set when the output
+// has no element.  kind: 0 NVFP4, 1 MXFP8, 2 MXFP4 (the two MX kinds use
+// 32-element blocks).
+static nvfp4_status check_quantize(const char* tag, int kind, const void* x, nvfp4_dtype dt, int64_t rows,
+                                   int64_t K, const float* g, const uint32_t* codes, const uint8_t* scales,
+                                   nvfp4_layout layout, bool* empty) {
   const int group = kind ? 32 : 16;
   if (!valid_dt(dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] dtype must be float32, float16 or bfloat16", tag);
   if (layout != NVFP4_LAYOUT_LINEAR && layout != NVFP4_LAYOUT_SWIZZLED)
@@ -191,15 +228,66 @@ static nvfp4_status quantize_common(const char* tag, int kind, const void* x, nv
   if (rows * K > 0 && (!x || !codes || !scales)) return fail(NVFP4_ERR_INVALID_ARG, "[%s] null pointer", tag);
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(g) & 3u))
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] tensor pointers must be 16-byte aligned", tag);
-  if (rows * K == 0) return ok();  // nothing to write: no device work, no device query
-  DeviceInfo d;
-  nvfp4_status st = device_info(tag, &d);
-  if (st != NVFP4_OK) return st;
+  *empty = rows * K == 0;
+  return NVFP4_OK;
+}
+
+static ScaleOut scale_out(uint8_t* scales, int64_t K, int group, nvfp4_layout layout) {
   ScaleOut so;
   so.p = scales;
   so.blocks_per_row = (uint32_t)(K / group);
   so.Cp = (uint32_t)((K / group + 3) / 4 * 4);
   so.swizzled = layout == NVFP4_LAYOUT_SWIZZLED;
+  return so;
+}
+
+// NVFP4 quantize of `count` tensors (those with elements) in one launch.
+static nvfp4_status nvfp4_quantize_launch(const char* tag, const nvfp4_quantize_item* items, int count,
+                                          nvfp4_dtype dt, nvfp4_stream_t stream, bool sr, uint64_t seed) {
+  if (!items || count < 1 || count > kMaxSegs)
+    return fail(NVFP4_ERR_INVALID_ARG, "[%s] between 1 and %d tensors, got %d", tag, kMaxSegs, count);
+  QuantSegs q;
+  memset(&q, 0, sizeof(q));
+  q.seed = seed;
+  for (int i = 0; i < count; ++i) {
+    const nvfp4_quantize_item& it = items[i];
+    bool empty = false;
+    nvfp4_status st = check_quantize(tag, 0, it.x, dt, it.rows, it.K, it.g, it.codes, it.scales, it.layout, &empty);
+    if (st != NVFP4_OK) return st;
+    if (empty) continue;
+    QuantSeg& sg = q.s[q.count++];
+    sg.x = it.x;
+    sg.g = it.g;
+    sg.codes = it.codes;
+    sg.so = scale_out(it.scales, it.K, 16, it.layout);
+    sg.rows = (uint32_t)it.rows;
+    sg.n_half = (uint32_t)(it.rows * it.K / 8);
+    sg.first_unit = q.units;
+    q.units += (sg.n_half + kUnitHalf - 1) / kUnitHalf;
+  }
+  if (q.count == 0) return ok();  // nothing to write: no device work, no device query
+  DeviceInfo d;
+  nvfp4_status st = device_info(tag, &d);
+  if (st != NVFP4_OK) return st;
+  const unsigned grid = ew_grid(d, (uint64_t)q.units * 32u);
+  dispatch_dt(dt, [&](auto tag_t) {
+    using T = decltype(tag_t);
+    if (sr) k_nvfp4_quantize<T, true><<<grid, kEwThreads, 0, stream>>>(q);
+    else k_nvfp4_quantize<T><<<grid, kEwThreads, 0, stream>>>(q);
+  });
+  return check_launch(tag);
+}
+
+static nvfp4_status mx_quantize(const char* tag, int kind, const void* x, nvfp4_dtype dt, int64_t rows, int64_t K,
+                                uint32_t* codes, uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
+  bool empty = false;
+  nvfp4_status st = check_quantize(tag, kind, x, dt, rows, K, nullptr, codes, scales, layout, &empty);
+  if (st != NVFP4_OK) return st;
+  if (empty) return ok();  // nothing to write: no device work, no device query
+  DeviceInfo d;
+  st = device_info(tag, &d);
+  if (st != NVFP4_OK) return st;
+  const ScaleOut so = scale_out(scales, K, 32, layout);
   const uint32_t n_half = (uint32_t)(rows * K / 8);
   const unsigned grid = ew_grid(d, ((uint64_t)n_half + kUnroll - 1) / kUnroll);
   dispatch_dt(dt, [&](auto tag_t) {
@@ -207,15 +295,8 @@ static nvfp4_status quantize_common(const char* tag, int kind, const void* x, nv
     if (kind == 1)
       k_mxfp8_quantize<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, codes, so,
                                                            (uint32_t)rows);
-    else if (kind == 2)
-      k_mxfp4_quantize<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, codes, so,
-                                                           (uint32_t)rows);
     else
-      if (sr)
-        k_nvfp4_quantize<T, true><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, g, codes, so,
-                                                                   (uint32_t)rows, seed);
-      else
-        k_nvfp4_quantize<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, g, codes, so,
+      k_mxfp4_quantize<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, codes, so,
                                                            (uint32_t)rows);
   });
   return check_launch(tag);
@@ -223,13 +304,20 @@ static nvfp4_status quantize_common(const char* tag, int kind, const void* x, nv
 
 nvfp4_status nvfp4_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K, const float* g,
                             uint32_t* codes, uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
-  return quantize_common("quantize", 0, x, dt, rows, K, g, codes, scales, layout, stream);
+  const nvfp4_quantize_item it{x, rows, K, g, codes, scales, layout};
+  return nvfp4_quantize_launch("quantize", &it, 1, dt, stream, false, 0);
+}
+
+nvfp4_status nvfp4_quantize_multi(const nvfp4_quantize_item* items, int count, nvfp4_dtype dt,
+                                  nvfp4_stream_t stream) {
+  return nvfp4_quantize_launch("quantize_multi", items, count, dt, stream, false, 0);
 }
 
 nvfp4_status nvfp4_quantize_sr(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K, const float* g,
                                uint64_t seed, uint32_t* codes, uint8_t* scales, nvfp4_layout layout,
                                nvfp4_stream_t stream) {
-  return quantize_common("quantize_sr", 0, x, dt, rows, K, g, codes, scales, layout, stream, true, seed);
+  const nvfp4_quantize_item it{x, rows, K, g, codes, scales, layout};
+  return nvfp4_quantize_launch("quantize_sr", &it, 1, dt, stream, true, seed);
 }
 
 nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, int64_t rows, int64_t cols, const float* g,
@@ -268,12 +356,12 @@ nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, int64_t ro
 
 nvfp4_status mxfp8_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K, uint32_t* codes,
                             uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
-  return quantize_common("mxfp8_quantize", 1, x, dt, rows, K, nullptr, codes, scales, layout, stream);
+  return mx_quantize("mxfp8_quantize", 1, x, dt, rows, K, codes, scales, layout, stream);
 }
 
 nvfp4_status mxfp4_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K, uint32_t* codes,
                             uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
-  return quantize_common("mxfp4_quantize", 2, x, dt, rows, K, nullptr, codes, scales, layout, stream);
+  return mx_quantize("mxfp4_quantize", 2, x, dt, rows, K, codes, scales, layout, stream);
 }
 
 static nvfp4_status dequantize_common(const char* tag, int kind, const uint32_t* codes, const uint8_t* scales,
@@ -401,7 +489,8 @@ nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32
   nvfp4_status st = device_info("qmv", &d);
   if (st != NVFP4_OK) return st;
   cudaError_t e = cudaSuccess;
-  const uint32_t stages = qtc::pick_stages(M, K);
+  const uint32_t esz = x_dt == NVFP4_DT_F32 ? 4u : 2u;
+  const uint32_t stages = qtc::pick_stages(M, K, esz);
   if (stages > 0) {
     // tensor-core path: one CTA per 128 weight rows
     CUtensorMap mw;
@@ -409,7 +498,7 @@ nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32
       return fail(NVFP4_ERR_CUDA, "[qmv] cuTensorMapEncodeTiled failed");
     qtc::Args a{x, g_x, w_codes, w_scales, g_w, y, (uint32_t)M, (uint32_t)N, (uint32_t)K, stages};
     const uint32_t MM = M == 1 ? 1u : 2u;
-    const size_t smem = qtc::smem_needed(stages, MM, (uint32_t)K);
+    const size_t smem = qtc::smem_needed(stages, MM, (uint32_t)K, esz);
     const unsigned grid = (unsigned)((N + qtc::BM - 1) / qtc::BM);
     dispatch_dt(x_dt, [&](auto tag_t) {
       using T = decltype(tag_t);
@@ -511,23 +600,56 @@ nvfp4_status gather_qmm_kn(const void* x, const uint32_t* w_codes, const uint8_t
                            sizeof(t_msg), true);
 }
 
-// Device address of g_noalloc_scratch on the current device, resolved on
-// the first call per device (with that device current) and cached.
+// Identity of the calling thread's current context (0 if none can be read):
+// cuCtxGetCurrent and cuCtxGetId through the runtime's driver entry points,
+// so the library needs no link against the driver library.
+static unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static bool looked = false;
+  if (!looked) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+    looked = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_noalloc_scratch on the current device, resolved with
+// that device current and cached per device together with the context it
+// belongs to: a new context on the device (after cudaDeviceReset, which
+// unloads the library's module and may place the array elsewhere) resolves
+// it again.
 static nvfp4_status noalloc_scratch(void** out) {
   static void* addr[64] = {nullptr};
+  static unsigned long long ctx_of[64] = {0};
   static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(NVFP4_ERR_CUDA, "[gather_qmm_noalloc] cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= 64) return fail(NVFP4_ERR_UNSUPPORTED, "[gather_qmm_noalloc] device ordinal %d", dev);
   std::lock_guard<std::mutex> lk(mu);
-  if (addr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (addr[dev] == nullptr || ctx == 0 || ctx != ctx_of[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr)
       return fail(NVFP4_ERR_CUDA, "[gather_qmm_noalloc] cudaGetSymbolAddress of the static scratch failed: %s",
                   cudaGetErrorString(e));
     addr[dev] = p;
+    ctx_of[dev] = ctx;
   }
   *out = addr[dev];
   return NVFP4_OK;

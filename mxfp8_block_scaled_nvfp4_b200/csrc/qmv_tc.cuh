@@ -29,8 +29,9 @@
 // CTA = 128 weight rows; warps: 0 TMA producer (codes [128 x 128 B] per
 // stage), 1 TMEM allocator + MMA issuer, 4-7 epilogue (TMEM lane quarters;
 // each lane reads its weight row's LINEAR scale bytes straight from global
-// memory, one ring half ahead).  Warps 1-11 compute the x_hat planes first,
-// while warp 0 starts the weight stream.
+// memory, one ring half ahead).  Warp 0 first copies x into shared memory
+// (one bulk copy, ahead of the weight in the memory queues) and then starts
+// the weight stream; warps 1-11 compute the x_hat planes from that copy.
 // TMEM: a 256-column ring of MMA outputs drained in 128-column halves and
 // one tile of unit scales used by both operands.
 //
@@ -64,8 +65,8 @@ constexpr uint32_t T_ONES = 256;     // unit block scales (both operands)
 // shared memory carve-up (bytes, from a 1024-aligned base)
 struct Layout {
   uint32_t stages, M, K;
-  uint32_t ring, planes, uplane, ones, total;
-  __host__ __device__ void init(uint32_t st, uint32_t m, uint32_t k) {
+  uint32_t ring, planes, uplane, ones, xraw, total;
+  __host__ __device__ void init(uint32_t st, uint32_t m, uint32_t k, uint32_t esz) {
     stages = st;
     M = m;
     K = k;
@@ -73,13 +74,14 @@ struct Layout {
     planes = stages * STAGE_BYTES;                 // 4 * M * K bytes (fp32 x_hat in the SIMT fallback)
     uplane = planes + 4u * M * K;                  // 2 * (K / 16) * M floats
     ones = uplane + 2u * (K / 16u) * M * 4u;       // 512 bytes of e4m3 1.0
-    total = ones + 512u;
+    xraw = ones + 512u;                            // x as stored: M * K elements of esz bytes
+    total = xraw + M * K * esz;
   }
 };
 
-__host__ __device__ inline uint32_t smem_needed(uint32_t stages, uint32_t M, uint32_t K) {
+__host__ __device__ inline uint32_t smem_needed(uint32_t stages, uint32_t M, uint32_t K, uint32_t esz) {
   Layout L;
-  L.init(stages, M, K);
+  L.init(stages, M, K, esz);
   return L.total + 1024u;
 }
 
@@ -113,24 +115,13 @@ template <> struct Range<__nv_bfloat16> {
 };
 
 // x_hat = quantize-dequantize(x, g_x) of all M rows as plane codes and
-// plane scales (layout in the header comment).  One lane per half-block;
-// returns false on a thread that met a block outside the exact range.
-// x values of this thread's first half-block, loaded at kernel start.
-// Threads 32.. (warps 1 and up) take part; warp 0 streams the weight.
+// plane scales (layout in the header comment), from x staged in shared
+// memory.  One lane per half-block; threads 32.. (warps 1 and up) take
+// part, warp 0 streams the weight.  Returns false on a thread that met a
+// block outside the exact range.
 template <typename T>
-__device__ __forceinline__ void x_first(const T* __restrict__ x, uint32_t M, uint32_t K, float (&v)[8]) {
-  const uint32_t t = threadIdx.x - 32u;
-  if (threadIdx.x >= 32u && t < M * K / 8u) {
-    load8<T>(x + (size_t)t * 8, v);
-  } else {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = 0.0f;
-  }
-}
-
-template <typename T>
-__device__ __forceinline__ bool x_planes(const T* __restrict__ x, float gx, uint32_t M, uint32_t K, float (&cur)[8],
-                                         uint8_t* planes, float* uplane) {
+__device__ __forceinline__ bool x_planes(const T* xs, float gx, uint32_t M, uint32_t K, uint8_t* planes,
+                                         float* uplane) {
   const float E = kGlobalEncode / gx;
   const float d = gx / kGlobalEncode;
   const uint32_t n_half = M * K / 8u;  // a multiple of 32: whole warps take part in the pair shuffle
@@ -139,10 +130,7 @@ __device__ __forceinline__ bool x_planes(const T* __restrict__ x, float gx, uint
   const uint32_t nthr = blockDim.x - 32u;  // warps 1 and up (a multiple of 32)
   for (uint32_t hb = threadIdx.x - 32u; threadIdx.x >= 32u && hb < n_half; hb += nthr) {
     float v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = cur[j];
-    const uint32_t hn = hb + nthr;  // next half-block's loads in flight during this one
-    if (hn < n_half) load8<T>(x + (size_t)hn * 8, cur);
+    load8_shared<T>(xs + (size_t)hb * 8, v);
     float a = 0.0f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[j]));
@@ -190,17 +178,16 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
   __shared__ __align__(8) uint64_t empty_bar[MAX_STAGES];
   __shared__ __align__(8) uint64_t dfull_bar[2];
   __shared__ __align__(8) uint64_t dempty_bar[2];
+  __shared__ __align__(8) uint64_t xbar;  // x landed in shared memory
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_flag;
 
-  // x and g_x first: these loads must not queue behind the weight stream
-  float xv[8];
-  x_first<T>(static_cast<const T*>(a.x), a.M, a.K, xv);
   const float gx = a.g_x ? __ldg(a.g_x) : kGlobalEncode;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   Layout L;
-  L.init(a.stages, MM, a.K);
+  L.init(a.stages, MM, a.K, (uint32_t)sizeof(T));
+  const uint32_t xbytes = a.M * a.K * (uint32_t)sizeof(T);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t row0 = blockIdx.x * BM;
   const uint32_t S = a.stages;
@@ -243,9 +230,14 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
       mbar_init(smem_u32(&dfull_bar[h]), 1);
       mbar_init(smem_u32(&dempty_bar[h]), 4);
     }
+    mbar_init(smem_u32(&xbar), 1);
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    // the weight stream starts before TMEM allocation and the prologue
+    // x first, one bulk copy (the rows are contiguous, 16-byte aligned and a
+    // multiple of 512 bytes long), so it does not queue behind the weight
+    // stream; then the weight stream, before TMEM allocation and the prologue
+    mbar_expect_tx(smem_u32(&xbar), xbytes);
+    bulk_load(sbase + L.xraw, a.x, xbytes, smem_u32(&xbar));
     for (; issued < S && issued < kb_count; ++issued) issue(issued);
   }
   // zero the plane tiles (a plane row is nonzero only inside its own
@@ -269,8 +261,14 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
 
-  const bool mine = x_planes<T>(static_cast<const T*>(a.x), gx, a.M, a.K, xv, smem + L.planes,
-                                reinterpret_cast<float*>(smem + L.uplane));
+  bool mine = true;
+  if (warp >= 1) {
+    mine = mbar_wait(smem_u32(&xbar), 0);
+    if (!mine) abort_flag = 1;
+    else
+      mine = x_planes<T>(reinterpret_cast<const T*>(smem + L.xraw), gx, a.M, a.K, smem + L.planes,
+                         reinterpret_cast<float*>(smem + L.uplane));
+  }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // planes are read by the tensor core
   const bool exact = __syncthreads_and(mine) != 0;
   const float dw = a.g_w ? __ldg(a.g_w) / kGlobalEncode : 1.0f;
@@ -280,7 +278,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
     // and SIMT rows for this CTA, after the loads in flight have landed
     float4* xs4 = reinterpret_cast<float4*>(smem + L.planes);
     qmv_prologue<T>(static_cast<const T*>(a.x), a.g_x, a.M, a.K, xs4, threadIdx.x, blockDim.x);
-    if (threadIdx.x == 0) drain(issued);
+    if (threadIdx.x == 0) {
+      drain(issued);
+      mbar_wait(smem_u32(&xbar), 0);  // x's copy has landed (a no-op unless its wait above gave up)
+    }
     __syncthreads();
     const uint32_t end = min(row0 + BM, a.N);
     qmv_simt_rows<T, MM>(xs4, a.wc, a.wsc, dw, a.M, a.N, a.K, static_cast<T*>(a.y), row0 + warp,
@@ -436,13 +437,14 @@ inline bool make_map(CUtensorMap* mw, const uint32_t* wc, uint64_t N, uint64_t K
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Stages that fit next to the plane tiles, plane scales and x_hat; 0 if the
-// tensor-core path does not apply (then the caller runs the SIMT kernel).
-inline uint32_t pick_stages(int64_t M, int64_t K) {
+// Stages that fit next to the plane tiles, plane scales and x (elements of
+// esz bytes); 0 if the tensor-core path does not apply (then the caller runs
+// the SIMT kernel).
+inline uint32_t pick_stages(int64_t M, int64_t K, uint32_t esz) {
   if (M < 1 || M > 2 || K % 256 != 0 || K < 256) return 0;
   const uint32_t MM = M == 1 ? 1u : 2u;
   for (uint32_t st = MAX_STAGES; st >= 2; st -= 2)  // even: two groups of st / 2 stages
-    if (smem_needed(st, MM, (uint32_t)K) <= 227u * 1024u) return st;
+    if (smem_needed(st, MM, (uint32_t)K, esz) <= 227u * 1024u) return st;
   return 0;
 }
 

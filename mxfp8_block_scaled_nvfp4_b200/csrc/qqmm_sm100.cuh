@@ -163,8 +163,9 @@ __device__ __forceinline__ uint64_t sf_tile_desc(uint32_t addr) { return smem_de
 // 10-12), K-major A and B, N >> 3 (bits 17-22), scale format (bit 23:
 // 0 = ue4m3, 1 = ue8m0), M >> 4 (bits 24-28), scale-factor byte ids of B
 // (bits 4-5) and A (bits 29-30).
-__host__ __device__ constexpr uint32_t block_scaled_idesc(uint32_t ab_format, uint32_t scale_ue8m0, uint32_t sf_id) {
-  return (sf_id << 4) | (ab_format << 7) | (ab_format << 10) | ((uint32_t)(BN >> 3) << 17) | (scale_ue8m0 << 23) |
+__host__ __device__ constexpr uint32_t block_scaled_idesc(uint32_t ab_format, uint32_t scale_ue8m0, uint32_t sf_id,
+                                                         uint32_t n = BN) {
+  return (sf_id << 4) | (ab_format << 7) | (ab_format << 10) | ((n >> 3) << 17) | (scale_ue8m0 << 23) |
          ((uint32_t)(BM >> 4) << 24) | (sf_id << 29);
 }
 
@@ -251,6 +252,8 @@ struct Params {
   uint32_t sf_groups;   // Cp / 4: scale-tile columns per 128-row block
   uint32_t rows_b_pad;  // ceil128(N)
   int tma_store;        // 1: y is written through tmap_y (row pitch a multiple of 16 bytes)
+  uint32_t nfull;       // work units that are whole 128 x 256 tiles
+  uint32_t units;       // all work units: nfull + 2 x (tiles split into 128 x 128 halves)
 };
 
 template <typename T>
@@ -372,9 +375,32 @@ __device__ __forceinline__ void tile_coords(uint32_t t, uint32_t mt, uint32_t nt
   tn = r / gm;
 }
 
+// Work unit u of the persistent schedule -> output tile.  Units below
+// p.nfull are 128 x 256 tiles in tile_coords order.  The tiles after them
+// (the last, partial wave of wide tiles) are split into their two 128 x 128
+// halves, one unit each, so that wave runs on up to twice as many SMs for
+// about half as long.  n0 is the first output column; false for a half that
+// lies wholly beyond N (every role skips it).
+__device__ __forceinline__ bool unit_coords(uint32_t u, const Params& p, uint32_t mt, uint32_t nt, uint32_t& tm,
+                                            uint32_t& n0, bool& wide) {
+  uint32_t tn;
+  if (u < p.nfull) {
+    tile_coords(u, mt, nt, tm, tn);
+    n0 = tn * BN;
+    wide = true;
+    return true;
+  }
+  const uint32_t s = u - p.nfull;
+  tile_coords(p.nfull + s / 2u, mt, nt, tm, tn);
+  n0 = tn * BN + (s & 1u) * 128u;
+  wide = false;
+  return n0 < (uint32_t)p.N;
+}
+
 template <int KIND>
 __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUtensorMap tmap_a,
                                                      const __grid_constant__ CUtensorMap tmap_b,
+                                                     const __grid_constant__ CUtensorMap tmap_b128,
                                                      const __grid_constant__ CUtensorMap tmap_y, Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
@@ -387,7 +413,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t mt = ((uint32_t)p.M + BM - 1) / BM, nt = ((uint32_t)p.N + BN - 1) / BN, tiles = mt * nt;
+  const uint32_t mt = ((uint32_t)p.M + BM - 1) / BM, nt = ((uint32_t)p.N + BN - 1) / BN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -415,11 +441,12 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t it = 0;  // global stage counter across tiles
-      for (uint32_t t = blockIdx.x; t < tiles && !*(volatile int*)&abort_flag; t += gridDim.x) {
-        uint32_t tm, tn;
-        tile_coords(t, mt, nt, tm, tn);
-        const int tile_m = (int)(tm * BM), tile_n = (int)(tn * BN);
-        const bool b_second = (uint32_t)(tile_n + 128) < p.rows_b_pad;
+      for (uint32_t u = blockIdx.x; u < p.units && !*(volatile int*)&abort_flag; u += gridDim.x) {
+        uint32_t tm, n0;
+        bool wide;
+        if (!unit_coords(u, p, mt, nt, tm, n0, wide)) continue;
+        const int tile_m = (int)(tm * BM), tile_n = (int)n0;
+        const bool b_second = wide && (uint32_t)(tile_n + 128) < p.rows_b_pad;
         for (uint32_t kb = 0; kb < p.kb_count; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           if (!mbar_wait(smem_u32(&empty_bar[s]), ((it / STAGES) & 1u) ^ 1u)) {
@@ -431,9 +458,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
           if (ntl > tiles_per_stage) ntl = tiles_per_stage;
           const uint32_t sfa_bytes = ntl * 512u, sfb_bytes = ntl * 512u * (b_second ? 2u : 1u);
           const uint32_t bar = smem_u32(&full_bar[s]);
-          mbar_expect_tx(bar, A_STAGE + B_STAGE + sfa_bytes + sfb_bytes);
+          mbar_expect_tx(bar, A_STAGE + (wide ? B_STAGE : B_STAGE / 2) + sfa_bytes + sfb_bytes);
           tma_load_2d(sbase + SMEM_A + s * A_STAGE, &tmap_a, (int)(kb * BKB), tile_m, bar);
-          tma_load_2d(sbase + SMEM_B + s * B_STAGE, &tmap_b, (int)(kb * BKB), tile_n, bar);
+          tma_load_2d(sbase + SMEM_B + s * B_STAGE, wide ? &tmap_b : &tmap_b128, (int)(kb * BKB), tile_n, bar);
         }
       }
       // drain: the last STAGES issued stages must have landed before exit
@@ -453,14 +480,16 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
       const uint64_t sfa_base = sf_tile_desc(sbase + SMEM_SFA), sfb_base = sf_tile_desc(sbase + SMEM_SFB);
       const uint32_t a_hi = (uint32_t)(a_base >> 32), b_hi = (uint32_t)(b_base >> 32);
       const uint32_t sfa_hi = (uint32_t)(sfa_base >> 32), sfb_hi = (uint32_t)(sfb_base >> 32);
-      const uint32_t idesc_nv = block_scaled_idesc(1u, 0u, 0u);  // e2m1 x e2m1, ue4m3
       auto mk = [](uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; };
       uint32_t it = 0, tile_i = 0, s = 0, ph = 0;
       bool ok = true;
-      for (uint32_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tile_i) {
-        uint32_t tm, tn;
-        tile_coords(t, mt, nt, tm, tn);
-        const bool b_second = (uint32_t)(tn * BN + 128) < p.rows_b_pad;
+      for (uint32_t u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        uint32_t tm, n0;
+        bool wide;
+        if (!unit_coords(u, p, mt, nt, tm, n0, wide)) continue;
+        const bool b_second = wide && (uint32_t)(n0 + 128) < p.rows_b_pad;
+        const uint32_t nmma = wide ? (uint32_t)BN : 128u;                 // MMA N of this unit
+        const uint32_t idesc_nv = block_scaled_idesc(1u, 0u, 0u, nmma);  // e2m1 x e2m1, ue4m3
         // the epilogue has drained the previous tile's accumulator
         if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&accum_empty), (tile_i & 1u) ^ 1u)) ||
             *(volatile int*)&abort_flag) {
@@ -490,7 +519,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
 #pragma unroll
               for (uint32_t j = 0; j < 4; ++j)
                 mma_block_scaled<kMX8>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi),
-                                       block_scaled_idesc(0u, 1u, j), tsfa, tsfb, (kb | j) != 0);
+                                       block_scaled_idesc(0u, 1u, j, nmma), tsfa, tsfb, (kb | j) != 0);
             } else {
               // NVFP4: one scale tile per k-step; MXFP4: one per two k-steps,
               // the k-step's two scale bytes selected by the scale-factor id
@@ -508,7 +537,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
                                         tsfb + 8 * j, (kb | j) != 0);
                 else
                   mma_block_scaled<kMX4>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi),
-                                         block_scaled_idesc(1u, 1u, (j & 1u) * 2u), tsfa + 4 * (j >> 1),
+                                         block_scaled_idesc(1u, 1u, (j & 1u) * 2u, nmma), tsfa + 4 * (j >> 1),
                                          tsfb + 8 * (j >> 1), (kb | j) != 0);
               }
             }
@@ -525,10 +554,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
               if (kb * BKB + j * 32u >= p.k_bytes) break;
               if constexpr (KIND == kMX8)
                 mma_block_scaled<kMX8>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi),
-                                       block_scaled_idesc(0u, 1u, j), tsfa, tsfb, (kb | j) != 0);
+                                       block_scaled_idesc(0u, 1u, j, nmma), tsfa, tsfb, (kb | j) != 0);
               else if constexpr (KIND == kMX4)
                 mma_block_scaled<kMX4>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi),
-                                       block_scaled_idesc(1u, 1u, (j & 1u) * 2u), tsfa + 4 * (j >> 1),
+                                       block_scaled_idesc(1u, 1u, (j & 1u) * 2u, nmma), tsfa + 4 * (j >> 1),
                                        tsfb + 8 * (j >> 1), (kb | j) != 0);
               else
                 mma_block_scaled<kNV>(tmem, mk(a_lo + 2 * j, a_hi), mk(b_lo + 2 * j, b_hi), idesc_nv, tsfa + 4 * j,
@@ -545,6 +574,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
         }
         if (leader) mma_commit(smem_u32(&accum_full));  // arrives when this tile's MMAs are done
         __syncwarp();
+        ++tile_i;
       }
     }
   } else if (warp == W_SCALES) {
@@ -554,11 +584,12 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
     // phase cannot complete before warp 0's arrival).
     if (lane == 0) {
       uint32_t it = 0;
-      for (uint32_t t = blockIdx.x; t < tiles && !*(volatile int*)&abort_flag; t += gridDim.x) {
-        uint32_t tm, tn;
-        tile_coords(t, mt, nt, tm, tn);
-        const int tile_n = (int)(tn * BN);
-        const bool b_second = (uint32_t)(tile_n + 128) < p.rows_b_pad;
+      for (uint32_t u = blockIdx.x; u < p.units && !*(volatile int*)&abort_flag; u += gridDim.x) {
+        uint32_t tm, n0;
+        bool wide;
+        if (!unit_coords(u, p, mt, nt, tm, n0, wide)) continue;
+        const int tile_n = (int)n0;
+        const bool b_second = wide && (uint32_t)(tile_n + 128) < p.rows_b_pad;
         for (uint32_t kb = 0; kb < p.kb_count; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           if (!mbar_wait(smem_u32(&empty_bar[s]), ((it / STAGES) & 1u) ^ 1u)) {
@@ -586,12 +617,21 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
     float alpha = 1.0f;
     if (KIND == kNV && p.g_x != nullptr) alpha = (__ldg(p.g_x) / kGlobalEncode) * (__ldg(p.g_w) / kGlobalEncode);
     uint32_t tile_i = 0;
-    for (uint32_t t = blockIdx.x; t < tiles; t += gridDim.x, ++tile_i) {
-      uint32_t tm, tn;
-      tile_coords(t, mt, nt, tm, tn);
+    for (uint32_t u = blockIdx.x; u < p.units; u += gridDim.x) {
+      uint32_t tm, n0;
+      bool wide;
+      if (!unit_coords(u, p, mt, nt, tm, n0, wide)) continue;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&accum_full), tile_i & 1u));
       tc_fence_after();
+      ++tile_i;
       if (!ok || *(volatile int*)&abort_flag) break;
+      if (!wide && half == 1) {
+        // a 128 x 128 unit: the second column half holds nothing
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&accum_empty)) : "memory");
+        continue;
+      }
       float v[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -605,7 +645,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&accum_empty)) : "memory");
       epilogue_store(p, &tmap_y, sbase + SMEM_EPI + (uint32_t)(warp - 2) * EPI_BUF, v, alpha,
-                     (int)(tm * BM) + q * 32, (int)(tn * BN) + half * 128, lane);
+                     (int)(tm * BM) + q * 32, (int)n0 + half * 128, lane);
     }
     // the tensor stores of this warp are complete before the CTA exits
     if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -678,8 +718,9 @@ inline nvfp4_status qqmm_launch(int kind, int64_t M, int64_t N, int64_t K, const
   using namespace tc;
   const bool mx = kind == tc::kMX8;
   const uint64_t k_bytes = mx ? (uint64_t)K : (uint64_t)K / 2;
-  CUtensorMap ta, tb;
-  if (!make_tmap(&ta, a_codes, (uint64_t)M, k_bytes, BM) || !make_tmap(&tb, b_codes, (uint64_t)N, k_bytes, BN)) {
+  CUtensorMap ta, tb, tb128;
+  if (!make_tmap(&ta, a_codes, (uint64_t)M, k_bytes, BM) || !make_tmap(&tb, b_codes, (uint64_t)N, k_bytes, BN) ||
+      !make_tmap(&tb128, b_codes, (uint64_t)N, k_bytes, 128)) {
     snprintf(msg, msg_len, "[qqmm] cuTensorMapEncodeTiled failed");
     return NVFP4_ERR_CUDA;
   }
@@ -701,12 +742,18 @@ inline nvfp4_status qqmm_launch(int kind, int64_t M, int64_t N, int64_t K, const
   const int64_t sf_cols = kind == tc::kNV ? K / 16 : K / 32;
   p.sf_groups = (uint32_t)((sf_cols + 3) / 4);
   p.rows_b_pad = (uint32_t)((N + 127) / 128 * 128);
+  // 128 x 256 tiles; when the last wave is at most half full, its tiles run
+  // as 128 x 128 halves (two units each) on up to twice as many SMs
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-  dim3 grid((unsigned)(tiles < sm_count ? tiles : sm_count));  // persistent: one CTA per SM
+  const int64_t rem = tiles % sm_count;
+  const bool split = rem != 0 && 2 * rem <= sm_count;
+  p.nfull = (uint32_t)(split ? tiles - rem : tiles);
+  p.units = (uint32_t)(split ? tiles + rem : tiles);
+  dim3 grid((unsigned)(p.units < (uint32_t)sm_count ? p.units : (uint32_t)sm_count));  // persistent: one CTA per SM
   cudaError_t e;
   auto go = [&](auto kern) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-    if (e == cudaSuccess) kern<<<grid, THREADS, SMEM_ALLOC, stream>>>(ta, tb, ty, p);
+    if (e == cudaSuccess) kern<<<grid, THREADS, SMEM_ALLOC, stream>>>(ta, tb, tb128, ty, p);
   };
   if (kind == kMX8) go(k_qqmm<kMX8>);
   else if (kind == kMX4) go(k_qqmm<kMX4>);

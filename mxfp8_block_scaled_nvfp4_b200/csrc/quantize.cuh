@@ -22,33 +22,59 @@ constexpr int kEwThreads = 256;
 constexpr int kUnroll = 4;
 
 // ---------------------------------------------------------------------------
-// a1: g = max |x|, atomically combined into *out (which the host zeroes).
+// a1: g = max |x| of up to 4 tensors in one launch, each atomically combined
+// into its own output (which the host zeroes).  Each thread keeps 4
+// independent 16-byte loads in flight per iteration.
 // ---------------------------------------------------------------------------
+constexpr int kAmaxSegs = 4;
+
+struct AmaxSegs {
+  const void* x[kAmaxSegs];
+  int64_t n[kAmaxSegs];
+  float* out[kAmaxSegs];
+  uint32_t count;
+};
+
 template <typename T>
-__global__ void __launch_bounds__(kEwThreads) k_amax(const T* __restrict__ x, int64_t n,
-                                                     float* __restrict__ out) {
-  const int64_t nvec = n / 8;
+__global__ void __launch_bounds__(kEwThreads) k_amax(const __grid_constant__ AmaxSegs a) {
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
-  float m = 0.0f;
-  for (int64_t i = tid; i < nvec; i += nthr) {
-    float v[8];
-    load8<T>(x + i * 8, v);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
-  }
-  for (int64_t i = nvec * 8 + tid; i < n; i += nthr) m = fmaxf(m, fabsf(Elem<T>::to_f(x[i])));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   __shared__ float red[kEwThreads / 32];
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    m = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+  for (uint32_t sgi = 0; sgi < a.count; ++sgi) {
+    const T* x = static_cast<const T*>(a.x[sgi]);
+    const int64_t n = a.n[sgi];
+    const int64_t nvec = n / 8;
+    float m = 0.0f;
+    for (int64_t i = tid; i < nvec; i += 4 * nthr) {
+      float v[4][8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int64_t j = i + k * nthr;
+        if (j < nvec) {
+          load8<T>(x + j * 8, v[k]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[k][e] = 0.0f;
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[k][e]));
+    }
+    for (int64_t i = nvec * 8 + tid; i < n; i += nthr) m = fmaxf(m, fabsf(Elem<T>::to_f(x[i])));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    // non-negative floats order like their bit patterns
-    if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned int*>(out), __float_as_uint(m));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      m = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      // non-negative floats order like their bit patterns
+      if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned int*>(a.out[sgi]), __float_as_uint(m));
+    }
+    __syncthreads();  // red is reused by the next tensor
   }
 }
 
@@ -137,32 +163,147 @@ __device__ __forceinline__ uint32_t e2m1_sr(float t, uint32_t r) {
 }
 
 // ---------------------------------------------------------------------------
+// a2-a4: NVFP4 quantize of up to kMaxSegs tensors in one launch (the raw
+// qqmm quantizes both operands, "mlx 0.30.7.2 -> 0.30.7.6" diff, page 8,
+// ops.cpp qqmm; one launch over both keeps every SM busy on what would be
+// two short launches).  Per 16-block: E = 2688 / g (1 without g);
+//   s = e4m3_rne_satfinite((amax / 6) * E);  q_i = e2m1(x_i * (E / f8(s)))
+// ("mlx 0.30.7.2 -> 0.30.7.6" diff, page 7, fp_quantize_rowwise), zero
+// codes for a block whose scale decodes to 0.
+//
+// Work unit: 32 x kUnroll half-blocks of one tensor (one warp iteration).
+// Units of all tensors form one sequence; warp w takes units w, w + nwarps,
+// ...  The loads of a warp's next unit are issued before the current one is
+// computed (two units in flight per warp).  Scale bytes of 4 consecutive
+// blocks are packed into one 32-bit store where they are contiguous (LINEAR
+// layout, or 4 blocks of one row starting at a multiple of 4 in the tile
+// layout); other scales are stored byte by byte.
+// ---------------------------------------------------------------------------
+constexpr int kMaxSegs = 4;
+constexpr uint32_t kUnitHalf = 32u * kUnroll;  // half-blocks per unit
+
+struct QuantSeg {
+  const void* x;
+  const float* g;
+  uint32_t* codes;
+  ScaleOut so;
+  uint32_t rows;
+  uint32_t n_half;
+  uint32_t first_unit;  // index of the segment's first unit in the launch's sequence
+};
+
+struct QuantSegs {
+  QuantSeg s[kMaxSegs];
+  uint32_t count;
+  uint32_t units;  // all units of all segments
+  uint64_t seed;   // stochastic rounding only
+};
+
+// Raw 16-byte words of one half-block (two for fp32).
+template <typename T>
+struct Raw8 {
+  uint4 a, b;
+};
+
+template <typename T>
+__device__ __forceinline__ void load_raw(const T* p, Raw8<T>& r) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+  r.a = __ldg(q);
+  if constexpr (sizeof(T) == 4) r.b = __ldg(q + 1);
+}
+
+__device__ __forceinline__ uint32_t seg_of(const QuantSegs& q, uint32_t unit) {
+  uint32_t i = 0;
+#pragma unroll
+  for (int j = 1; j < kMaxSegs; ++j)
+    if ((uint32_t)j < q.count && unit >= q.s[j].first_unit) i = (uint32_t)j;
+  return i;
+}
+
+template <typename T>
+__device__ __forceinline__ void load_unit(const QuantSegs& q, uint32_t unit, uint32_t lane, Raw8<T> (&r)[kUnroll]) {
+  if (unit >= q.units) return;
+  const QuantSeg& sg = q.s[seg_of(q, unit)];
+  const uint32_t base = (unit - sg.first_unit) * kUnitHalf;
+  const T* x = static_cast<const T*>(sg.x);
+#pragma unroll
+  for (int u = 0; u < kUnroll; ++u) {
+    const uint32_t hb = base + (uint32_t)u * 32u + lane;
+    if (hb < sg.n_half) load_raw<T>(x + (size_t)hb * 8, r[u]);
+    else r[u].a = r[u].b = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Scale bytes s of the even lanes' blocks (block hb >> 1 of lane hb), 4
+// consecutive blocks per 32-bit store where possible.  All lanes call it.
+__device__ __forceinline__ void store_scales(const ScaleOut& so, uint32_t hb, uint32_t n_half, uint32_t s,
+                                             uint32_t lane) {
+  const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 2);
+  const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 4);
+  const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 6);
+  // lane % 8 == 0 owns blocks b0 .. b0 + 3 (b0 a multiple of 4)
+  const uint32_t lead = hb & ~7u;
+  const uint32_t b0 = lead >> 1;
+  bool packed = lead + 8u <= n_half;  // all four blocks exist
+  uint32_t off = b0;
+  if (so.swizzled) {
+    const uint32_t r = b0 / so.blocks_per_row, c = b0 - r * so.blocks_per_row;
+    packed = packed && (c & 3u) == 0 && c + 4u <= so.blocks_per_row;
+    off = swizzled_offset(r, c, so.Cp);
+  }
+  if (packed) {
+    if ((lane & 7u) == 0) *reinterpret_cast<uint32_t*>(so.p + off) = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  } else if ((lane & 1u) == 0 && hb < n_half) {
+    so.store(hb >> 1, s);
+  }
+}
+
 template <typename T, bool SR = false>
-__global__ void __launch_bounds__(kEwThreads) k_nvfp4_quantize(
-    const T* __restrict__ x, uint32_t n_half, const float* __restrict__ g,
-    uint32_t* __restrict__ codes, ScaleOut so, uint32_t rows, uint64_t seed = 0) {
-  const float E = g ? kGlobalEncode / __ldg(g) : 1.0f;
+__global__ void __launch_bounds__(kEwThreads) k_nvfp4_quantize(const __grid_constant__ QuantSegs q) {
   const uint32_t lane = threadIdx.x & 31u;
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-  for (uint32_t base = warp * 32u * kUnroll; base < n_half; base += nwarps * 32u * kUnroll) {
-    float v[kUnroll][8];
+  Raw8<T> nxt[kUnroll];
+  load_unit<T>(q, warp, lane, nxt);
+  for (uint32_t unit = warp; unit < q.units; unit += nwarps) {
+    Raw8<T> cur[kUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const uint32_t hb = base + u * 32u + lane;
-      if (hb < n_half) {
-        load8<T>(x + (size_t)hb * 8, v[u]);
-      } else {
+    for (int u = 0; u < kUnroll; ++u) cur[u] = nxt[u];
+    load_unit<T>(q, unit + nwarps, lane, nxt);  // next unit's loads in flight during this one
+    const QuantSeg& sg = q.s[seg_of(q, unit)];
+    const uint32_t base = (unit - sg.first_unit) * kUnitHalf;
+    const float E = sg.g ? kGlobalEncode / __ldg(sg.g) : 1.0f;
+    // stochastic rounding: half-blocks 2c and 2c + 1 share generator call c
+    // (words x, y for the even one, z, w for the odd one).  Over iterations
+    // (u, u + 1) the even lane of a pair calls the generator for u and the
+    // odd lane for u + 1; each hands its partner the two words it needs.
+    uint32_t wa[kUnroll], wb[kUnroll];
+    if constexpr (SR) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
+      for (int u = 0; u < kUnroll; u += 2) {
+        const uint32_t odd = lane & 1u;
+        const uint64_t c0 = (uint64_t)(base + (uint32_t)(u + (int)odd) * 32u + (lane & ~1u)) >> 1;
+        const uint4 r4 = philox4x32_10(make_uint4((uint32_t)c0, (uint32_t)(c0 >> 32), 0u, 0u), (uint32_t)q.seed,
+                                       (uint32_t)(q.seed >> 32));
+        const uint32_t give0 = odd ? r4.x : r4.z, give1 = odd ? r4.y : r4.w;
+        const uint32_t got0 = __shfl_xor_sync(0xffffffffu, give0, 1);
+        const uint32_t got1 = __shfl_xor_sync(0xffffffffu, give1, 1);
+        // even lane: u from its own call (x, y), u + 1 from the partner's (x, y)
+        // odd lane:  u from the partner's call (z, w), u + 1 from its own (z, w)
+        wa[u] = odd ? got0 : r4.x;
+        wb[u] = odd ? got1 : r4.y;
+        wa[u + 1] = odd ? r4.z : got0;
+        wb[u + 1] = odd ? r4.w : got1;
       }
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const uint32_t hb = base + u * 32u + lane;
+      const uint32_t hb = base + (uint32_t)u * 32u + lane;
+      float v[8];
+      unpack8<T>(cur[u].a, cur[u].b, v);
       float a = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[u][j]));
+      for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[j]));
       a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
       float t = a / kE2M1Max;
       t = t * E;
@@ -171,29 +312,22 @@ __global__ void __launch_bounds__(kEwThreads) k_nvfp4_quantize(
       uint32_t w = 0;
       if (fs != 0.0f) {
         const float k = E / fs;
-        float q[8];
+        float qv[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) q[j] = v[u][j] * k;
+        for (int j = 0; j < 8; ++j) qv[j] = v[j] * k;
         if constexpr (SR) {
-          // elements 8hb..8hb+7 use words 2hb and 2hb+1: outputs 2(hb%2) and
-          // 2(hb%2)+1 of the generator call at counter hb/2
-          const uint64_t c0 = (uint64_t)hb >> 1;
-          const uint4 r4 = philox4x32_10(make_uint4((uint32_t)c0, (uint32_t)(c0 >> 32), 0u, 0u), (uint32_t)seed,
-                                         (uint32_t)(seed >> 32));
-          const uint32_t wa = (hb & 1u) ? r4.z : r4.x, wb = (hb & 1u) ? r4.w : r4.y;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) w |= e2m1_sr(q[j], ((j < 4 ? wa : wb) >> (8 * (j & 3))) & 0xFFu) << (4 * j);
+          for (int j = 0; j < 8; ++j)
+            w |= e2m1_sr(qv[j], ((j < 4 ? wa[u] : wb[u]) >> (8 * (j & 3))) & 0xFFu) << (4 * j);
         } else {
-          w = f32x8_to_e2m1x8(q);
+          w = f32x8_to_e2m1x8(qv);
         }
       }
-      if (hb < n_half) {
-        codes[hb] = w;
-        if ((lane & 1u) == 0) so.store(hb >> 1, s);
-      }
+      if (hb < sg.n_half) sg.codes[hb] = w;
+      store_scales(sg.so, hb, sg.n_half, s, lane);
     }
   }
-  zero_scale_padding(so, rows);
+  for (uint32_t i = 0; i < q.count; ++i) zero_scale_padding(q.s[i].so, q.s[i].rows);
 }
 
 // ---------------------------------------------------------------------------

@@ -26,13 +26,28 @@ MODE = {"nvfp4": 0, "mxfp8": 1, "mxfp4": 2}
 
 # (name, restype, argtypes) of every symbol declared in include/nvfp4.h
 _P, _I64, _I, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+
+
+class AmaxItem(ctypes.Structure):
+    """nvfp4_amax_item"""
+    _fields_ = [("x", _P), ("n", _I64), ("g_out", _P)]
+
+
+class QuantizeItem(ctypes.Structure):
+    """nvfp4_quantize_item (the layout enum is a C int)"""
+    _fields_ = [("x", _P), ("rows", _I64), ("K", _I64), ("g", _P), ("codes", _P), ("scales", _P),
+                ("layout", _I)]
+
+
 SIGNATURES = [
     ("nvfp4_status_string", ctypes.c_char_p, [_I]),
     ("nvfp4_last_error_message", ctypes.c_char_p, []),
     ("nvfp4_check_device_errors", _I, [_P]),
     ("nvfp4_scale_bytes", _SZ, [_I64, _I64, _I]),
     ("nvfp4_amax", _I, [_P, _I, _I64, _P, _P]),
+    ("nvfp4_amax_multi", _I, [ctypes.POINTER(AmaxItem), _I, _I, _P]),
     ("nvfp4_quantize", _I, [_P, _I, _I64, _I64, _P, _P, _P, _I, _P]),
+    ("nvfp4_quantize_multi", _I, [ctypes.POINTER(QuantizeItem), _I, _I, _P]),
     ("nvfp4_quantize_columnwise", _I, [_P, _I, _I64, _I64, _P, _P, _P, _I, _P]),
     ("nvfp4_dequantize", _I, [_P, _P, _I, _I64, _I64, _P, _P, _I, _P]),
     ("nvfp4_quantize_sr", _I, [_P, _I, _I64, _I64, _P, ctypes.c_uint64, _P, _P, _I, _P]),
@@ -176,6 +191,52 @@ def nvfp4_quantize(x: torch.Tensor, g: torch.Tensor | None = None, layout: str =
     return codes, scales
 
 
+def amax_multi(xs, out: torch.Tensor | None = None) -> torch.Tensor:
+    """fp32 [len(xs)] tensor: out[i] = max |xs[i]|, one launch (1 to 4
+    tensors of one dtype)."""
+    n = len(xs)
+    if not 1 <= n <= 4:
+        raise ValueError("amax_multi takes 1 to 4 tensors")
+    if any(x.dtype != xs[0].dtype for x in xs):
+        raise ValueError("amax_multi: every tensor must have the same dtype")
+    _need_g(out, n, "out")
+    _need_cuda(*xs, out)
+    out = torch.empty(n, dtype=torch.float32, device=xs[0].device) if out is None else out
+    items = (AmaxItem * n)(*[AmaxItem(x.data_ptr(), x.numel(), out.data_ptr() + 4 * i) for i, x in enumerate(xs)])
+    _check(lib().nvfp4_amax_multi(items, n, DT[xs[0].dtype], _stream()))
+    return out
+
+
+def nvfp4_quantize_multi(jobs):
+    """nvfp4_quantize of 1 to 4 tensors of one dtype in one launch.  jobs:
+    (x, g, layout[, codes, scales]) tuples, as nvfp4_quantize's arguments.
+    Returns [(codes, scales), ...] in the same order."""
+    n = len(jobs)
+    if not 1 <= n <= 4:
+        raise ValueError("nvfp4_quantize_multi takes 1 to 4 tensors")
+    outs, items = [], []
+    for job in jobs:
+        x, g, layout = job[0], job[1], job[2]
+        codes, scales = (job[3], job[4]) if len(job) > 3 else (None, None)
+        if x.dtype != jobs[0][0].dtype:
+            raise ValueError("nvfp4_quantize_multi: every tensor must have the same dtype")
+        rows, K = x.shape
+        _need_g(g)
+        _need_bytes(codes, rows * (K // 8) * 4, "codes")
+        _need_bytes(scales, _scale_nbytes(rows, K // 16, layout), "scales")
+        _need_cuda(x, g, codes, scales)
+        if codes is None:
+            codes = torch.empty(rows, K // 8, dtype=torch.int32, device=x.device)
+        if scales is None:
+            scales = torch.empty(scale_shape(rows, K // 16, layout), dtype=torch.uint8, device=x.device)
+        outs.append((codes, scales))
+        items.append(QuantizeItem(x.data_ptr(), rows, K, None if g is None else g.data_ptr(), codes.data_ptr(),
+                                  scales.data_ptr(), LAYOUT[layout]))
+    arr = (QuantizeItem * n)(*items)
+    _check(lib().nvfp4_quantize_multi(arr, n, DT[jobs[0][0].dtype], _stream()))
+    return outs
+
+
 def nvfp4_quantize_columnwise(x: torch.Tensor, g: torch.Tensor | None = None, layout: str = "linear",
                               codes: torch.Tensor | None = None, scales: torch.Tensor | None = None):
     """(codes [cols, rows/8], scales) of x^T quantized along the rows of a 2-D x
@@ -304,6 +365,29 @@ def qqmm(a_codes, a_scales, b_codes, b_scales, K: int, mode: str = "nvfp4", g_x=
     _check(lib().qqmm(MODE[mode], M, N, K, _ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales),
                       _ptr(g_x), _ptr(g_w), _ptr(out), DT[out.dtype], _stream()))
     return out
+
+
+def qqmm_raw(x: torch.Tensor, w: torch.Tensor, out_dtype=None, out: torch.Tensor | None = None, buffers=None):
+    """y [M, N] = qqmm of raw operands x [M, K] and w [N, K] (one dtype),
+    NVFP4 with g = amax of each ("mlx 0.30.7.2 -> 0.30.7.6" diff, page 8,
+    ops.cpp qqmm on unquantized inputs): both amaxes in one launch, both
+    quantizations (SWIZZLED scales) in one launch, then the GEMM.  y has x's
+    dtype unless out_dtype or out says otherwise.  buffers: optional
+    preallocated (g [2] fp32, x codes, x scales, w codes, w scales)."""
+    M, K = x.shape
+    N = w.shape[0]
+    if w.shape[1] != K or w.dtype != x.dtype:
+        raise ValueError("x [M, K] and w [N, K] must share K and dtype")
+    if buffers is None:
+        dev = x.device
+        g = torch.empty(2, dtype=torch.float32, device=dev)
+        xc, wc = (torch.empty(r, K // 8, dtype=torch.int32, device=dev) for r in (M, N))
+        xs, ws = (torch.empty(scale_shape(r, K // 16, "swizzled"), dtype=torch.uint8, device=dev) for r in (M, N))
+    else:
+        g, xc, xs, wc, ws = buffers
+    amax_multi([x, w], g)
+    nvfp4_quantize_multi([(x, g[0:1], "swizzled", xc, xs), (w, g[1:2], "swizzled", wc, ws)])
+    return qqmm(xc, xs, wc, ws, K, "nvfp4", g[0:1], g[1:2], out_dtype=out_dtype or x.dtype, out=out)
 
 
 def qqmm_vjp(x: torch.Tensor, w: torch.Tensor, cotan: torch.Tensor, g_x: torch.Tensor, g_w: torch.Tensor):

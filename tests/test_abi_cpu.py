@@ -258,3 +258,38 @@ def test_plain_c_caller(L):
     assert r.returncode == 0, r.stdout + r.stderr
     assert r.stdout.strip().endswith("ok")
     assert "or neither" in r.stdout
+
+
+def test_multi_tensor_entries_check_every_item(L):
+    """nvfp4_amax_multi / nvfp4_quantize_multi: 1 to 4 items, each checked as
+    the single-tensor call checks it; items with no element are skipped, so
+    a call whose items are all empty returns OK without a device, while
+    amax_multi (which zeroes its outputs) always needs one."""
+    from mxfp8_block_scaled_nvfp4_b200.nvfp4 import AmaxItem, QuantizeItem
+    N0 = None
+
+    def q(*items):
+        arr = (QuantizeItem * max(1, len(items)))(*items)
+        return L.nvfp4_quantize_multi(arr, len(items), 2, N0)
+
+    def am(*items):
+        arr = (AmaxItem * max(1, len(items)))(*items)
+        return L.nvfp4_amax_multi(arr, len(items), 2, N0)
+
+    good = QuantizeItem(A, 4, 64, N0, A, A, 0)
+    empty = QuantizeItem(N0, 0, 64, N0, N0, N0, 1)
+    assert q() == 1 and "between 1 and 4" in msg(L)
+    assert q(good, good, good, good, good) == 1
+    assert q(empty, empty) == 0
+    assert q(empty, QuantizeItem(A, 4, 24, N0, A, A, 0)) == 1 and "group size 16" in msg(L)
+    assert q(good, QuantizeItem(A + 8, 4, 64, N0, A, A, 0)) == 1 and "16-byte aligned" in msg(L)
+    assert q(good, QuantizeItem(A, 4, 64, N0, A, A, 7)) == 1 and "layout" in msg(L)
+    assert q(good, empty) not in (0, 1, 2)  # work to do: reaches the device query (no device here)
+    assert L.nvfp4_quantize_multi(None, 1, 2, N0) == 1
+    assert L.nvfp4_quantize_multi((QuantizeItem * 1)(good), 1, 7, N0) == 2
+
+    assert am() == 1
+    assert am(AmaxItem(A, 16, A), AmaxItem(A, 16, A)) == 1 and "share one output" in msg(L)
+    assert am(AmaxItem(A, -1, A)) == 1
+    assert am(AmaxItem(A, 16, A + 2)) == 1 and "4-byte aligned" in msg(L)
+    assert am(AmaxItem(A, 16, A), AmaxItem(A, 0, A + 4)) not in (0, 1, 2)

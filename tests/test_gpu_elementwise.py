@@ -214,3 +214,62 @@ def test_full_size_quantize_sampled_rows(nv, orc):
     assert np.array_equal(sc[off], os_)
     del x, codes, scales
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_amax_multi_parity(nv, orc, dt):
+    """Several tensors in one launch (ragged lengths, an empty one): each
+    output equals the oracle's amax of its tensor, with consecutive and with
+    separate output buffers."""
+    import ctypes
+    xs = [make_x((n,), dt, 300 + n) for n in (100003, 7, 4096 * 3)]
+    xs[1] = xs[1] * 40.0  # the largest values in the shortest tensor
+    want = [orc.amax(raw(x), dt) for x in xs]
+    gs = nv.amax_multi([x.cuda() for x in xs])
+    assert gs.cpu().tolist() == want
+    # separate outputs (one memset each) and an empty tensor, through the C ABI
+    xg = [x.cuda() for x in xs] + [torch.empty(0, dtype=xs[0].dtype, device="cuda")]
+    outs = [torch.full((1,), 7.0, device="cuda") for _ in xg]
+    items = (nv.AmaxItem * 4)(*[nv.AmaxItem(x.data_ptr(), x.numel(), o.data_ptr()) for x, o in zip(xg, outs)])
+    st = nv.lib().nvfp4_amax_multi(items, 4, nv.DT[xg[0].dtype], ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    assert [o.item() for o in outs] == want + [0.0]
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+def test_quantize_multi_parity(nv, orc, dt):
+    """Four tensors of different shapes, layouts and global scales in one
+    launch: every code and scale byte equals the oracle's (as one
+    nvfp4_quantize per tensor), padding of the tile layout zero."""
+    shapes = [(67, 256), (200, 1040), (1, 16), (257, 48)]
+    layouts = ["swizzled", "linear", "linear", "swizzled"]
+    xs = [make_x(s, dt, 500 + i, std=0.02 if dt != "f16" else 1.0) for i, s in enumerate(shapes)]
+    xg = [x.cuda() for x in xs]
+    gs = [nv.amax(xg[0]), None, nv.amax(xg[2]), nv.amax(xg[3])]
+    # poison the outputs: every byte must be written
+    jobs = []
+    for x, g, lay in zip(xg, gs, layouts):
+        rows, K = x.shape
+        codes = torch.full((rows, K // 8), -1, dtype=torch.int32, device="cuda")
+        scales = torch.full(nv.scale_shape(rows, K // 16, lay), 0xAB, dtype=torch.uint8, device="cuda")
+        jobs.append((x, g, lay, codes, scales))
+    outs = nv.nvfp4_quantize_multi(jobs)
+    torch.cuda.synchronize()
+    for x, g, lay, (codes, scales) in zip(xs, gs, layouts, outs):
+        oc, os_ = orc.nvfp4_quantize(raw(x), dt, None if g is None else g.item())
+        assert np.array_equal(raw(codes), oc)
+        assert np.array_equal(raw(scales), os_ if lay == "linear" else orc.swizzle_scales(os_))
+
+
+def test_qqmm_raw_matches_the_separate_calls(nv):
+    """qqmm_raw (amax and quantize of both operands, one launch each, then
+    the GEMM) gives bit for bit the result of the single-tensor calls."""
+    x = make_x((300, 512), "bf16", 71).cuda()
+    w = make_x((520, 512), "bf16", 72, std=0.02).cuda()
+    y = nv.qqmm_raw(x, w)
+    g_x, g_w = nv.amax(x), nv.amax(w)
+    xc, xs = nv.nvfp4_quantize(x, g_x, "swizzled")
+    wc, ws = nv.nvfp4_quantize(w, g_w, "swizzled")
+    y2 = nv.qqmm(xc, xs, wc, ws, 512, "nvfp4", g_x, g_w)
+    nv.check_device_errors()
+    assert y.dtype == torch.bfloat16 and torch.equal(y.view(torch.int16), y2.view(torch.int16))

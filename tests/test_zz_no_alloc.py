@@ -55,8 +55,11 @@ def _close(a, b):
 
 
 def test_noalloc_matches_workspace_entry_point_twice(nv):
-    cases = [(256, 8, 16, 512, 256, 11), (96, 2, 5, 128, 512, 12)]
-    for T, topk, E, N, K, seed in cases:  # two calls in a row, different routing
+    # calls in a row with different routing: the decode path (T <= 16 tokens,
+    # its tile list and permutation in the static scratch) first, then larger
+    # calls that would read any stale tile entries it left
+    cases = [(8, 4, 8, 256, 256, 10), (256, 8, 16, 512, 256, 11), (96, 2, 5, 128, 512, 12)]
+    for T, topk, E, N, K, seed in cases:
         x, wc, ws, g, idx = _case(nv, T, topk, E, N, K, seed)
         want = nv.gather_qmm(x, wc, ws, g, idx)
         got = torch.full_like(want, float("nan"))
@@ -80,3 +83,47 @@ def test_noalloc_rejects_scratch_beyond_its_size(nv):
                               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == nv.ERR_UNSUPPORTED
     assert "static scratch" in L.nvfp4_last_error_message().decode()
+
+
+def test_noalloc_against_the_oracle(nv, orc):
+    """One decode-size and one tensor-core-size call compared with the CPU
+    oracle's gather_qmm on the oracle's own quantization of the same seeded
+    weights (the tolerance of the other GEMM tests)."""
+    import numpy as np
+    from helpers import check_gemm_output, raw
+    from mxfp8_block_scaled_nvfp4_b200 import workloads
+    for T, topk, E, N, K, seed in [(12, 2, 6, 128, 256, 21), (80, 3, 7, 272, 192, 22)]:
+        w = workloads.normal((E, N, K), 0.02, seed, torch.bfloat16)
+        x = workloads.normal((T, K), 1.0, seed + 1, torch.bfloat16)
+        idx = workloads.routing(T, E, topk, seed + 2)
+        wg = w.cuda()
+        g = torch.stack([nv.amax(wg[e]) for e in range(E)]).view(E)
+        wc = torch.empty(E, N, K // 8, dtype=torch.int32, device="cuda")
+        ws = torch.empty(E, N, K // 16, dtype=torch.uint8, device="cuda")
+        for e in range(E):
+            nv.nvfp4_quantize(wg[e], g[e:e + 1], "linear", wc[e], ws[e])
+        y = torch.empty(T, topk, N, dtype=torch.bfloat16, device="cuda")
+        assert _noalloc_raw(nv, x.cuda(), wc, ws, g, idx.cuda(), y) == nv.OK
+        nv.check_device_errors()
+        gs = np.array([orc.amax(raw(w[e]), "bf16") for e in range(E)], dtype=np.float32)
+        q = [orc.nvfp4_quantize(raw(w[e]), "bf16", float(gs[e])) for e in range(E)]
+        oc, os_ = np.stack([c for c, _ in q]), np.stack([s for _, s in q])
+        assert np.array_equal(raw(wc).reshape(oc.shape), oc)
+        r = orc.gather_qmm(raw(x), oc, os_, gs, idx.numpy())
+        check_gemm_output(raw(y), r, "bf16", orc)
+
+
+def test_noalloc_leaves_free_device_memory_unchanged(nv):
+    """After a warm-up call, a call changes nothing in the device's free
+    memory (cudaMemGetInfo): the entry point allocates nothing."""
+    x, wc, ws, g, idx = _case(nv, 64, 4, 8, 256, 256, 31)
+    y = torch.empty(64, 4, 256, dtype=torch.bfloat16, device="cuda")
+    assert _noalloc_raw(nv, x, wc, ws, g, idx, y) == nv.OK
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert _noalloc_raw(nv, x, wc, ws, g, idx, y) == nv.OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    nv.check_device_errors()
