@@ -263,6 +263,23 @@ NVFP4_API nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, co
                  const uint8_t* w_scales, const float* g_w, int64_t M, int64_t N, int64_t K,
                  void* y, nvfp4_stream_t stream);
 
+/* qmv for chains of decode calls whose weights stay fixed (the layers of a
+ * model at decode time): the same arguments, checks and result as qmv, but
+ * launched with programmatic dependent launch.  The kernel starts streaming
+ * w_codes and w_scales (and reads g_w) before the kernel before it on the
+ * stream has finished; it reads x and g_x and writes y only after that
+ * kernel has completed and its writes are visible.  Each call lets the next
+ * launch start at once, so back-to-back calls overlap one weight stream
+ * with the previous call's tail.
+ * Precondition: w_codes, w_scales and g_w are not written by any work still
+ * pending on the device when the call is enqueued (e.g. they were written
+ * and the writer synchronized before, as for weights loaded once).  Sizes
+ * the tensor-core path does not take (see qmv) run the SIMT kernel in plain
+ * stream order. */
+NVFP4_API nvfp4_status qmv_pdl(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32_t* w_codes,
+                               const uint8_t* w_scales, const float* g_w, int64_t M, int64_t N, int64_t K,
+                               void* y, nvfp4_stream_t stream);
+
 /* a10 -- gather_qmm: MoE matmul with per-expert NVFP4 weights and per-expert
  * global scales ([P3]: the global scale multiplies each fp8 block scale
  * inside the dequantization, before the cast to bf16; weights transposed).

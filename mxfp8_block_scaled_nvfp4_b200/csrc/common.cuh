@@ -185,6 +185,54 @@ __device__ __forceinline__ uint32_t f32x8_to_e2m1x8(const float (&v)[8]) {
   return out;
 }
 
+// e2m1 codes of v[i] * k (each product rounded to fp32, as v[i] * k is;
+// computed two at a time by the packed fp32x2 multiply), element i in bits
+// 4i..4i+3.
+__device__ __forceinline__ uint32_t scaled_e2m1x8(const float (&v)[8], float k) {
+  uint32_t out;
+  asm("{\n\t"
+      ".reg .b64 kk, p0, p1, p2, p3;\n\t"
+      ".reg .f32 q0, q1, q2, q3, q4, q5, q6, q7;\n\t"
+      ".reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b64 kk, {%9, %9};\n\t"
+      "mov.b64 p0, {%1, %2};\n\t"
+      "mov.b64 p1, {%3, %4};\n\t"
+      "mov.b64 p2, {%5, %6};\n\t"
+      "mov.b64 p3, {%7, %8};\n\t"
+      "mul.rn.f32x2 p0, p0, kk;\n\t"
+      "mul.rn.f32x2 p1, p1, kk;\n\t"
+      "mul.rn.f32x2 p2, p2, kk;\n\t"
+      "mul.rn.f32x2 p3, p3, kk;\n\t"
+      "mov.b64 {q0, q1}, p0;\n\t"
+      "mov.b64 {q2, q3}, p1;\n\t"
+      "mov.b64 {q4, q5}, p2;\n\t"
+      "mov.b64 {q6, q7}, p3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, q1, q0;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, q3, q2;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, q5, q4;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, q7, q6;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t"
+      "}"
+      : "=r"(out)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(k));
+  return out;
+}
+
+// n / d for a fixed divisor d >= 1 and n < 2^31 with one multiply-high
+// (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", PLDI 1994): with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (umulhi(n, m) + n) >> l.
+struct FastDiv {
+  uint32_t d, m, l;
+  __host__ __device__ void init(uint32_t dd) {
+    d = dd;
+    l = 0;
+    while ((1ull << l) < (unsigned long long)d) ++l;
+    m = (uint32_t)((((1ull << 32) * ((1ull << l) - d)) / d) + 1ull);
+  }
+  __device__ __forceinline__ uint32_t div(uint32_t n) const { return (__umulhi(n, m) + n) >> l; }
+};
+
 // Four fp32 values to four e4m3 bytes (RNE, satfinite), element i in byte i.
 __device__ __forceinline__ uint32_t f32x4_to_e4m3x4(float a, float b, float c, float d) {
   uint16_t lo, hi;

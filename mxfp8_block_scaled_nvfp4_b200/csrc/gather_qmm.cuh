@@ -635,7 +635,105 @@ constexpr int kQmvPairs = 4;     // routed x rows per pass
 constexpr int QV_THREADS = 256;
 constexpr int QV_ROWS = 16;      // weight rows per CTA (2 per warp)
 
-// CTA (row block, tile): weight rows n0..n0+15 of the tile's expert against
+// a0 += w0 * x0, a1 += w1 * x1 (one packed fp32x2 fused multiply-add,
+// each lane rounded as fmaf rounds).
+__device__ __forceinline__ void ffma2(float& a0, float& a1, float w0, float w1, float x0, float x1) {
+  asm("{\n\t.reg .b64 acc, w, x;\n\t"
+      "mov.b64 acc, {%0, %1};\n\t"
+      "mov.b64 w, {%2, %3};\n\t"
+      "mov.b64 x, {%4, %5};\n\t"
+      "fma.rn.f32x2 acc, w, x, acc;\n\t"
+      "mov.b64 {%0, %1}, acc;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(w0), "f"(w1), "f"(x0), "f"(x1));
+}
+
+// Weight row r (< QV_ROWS) of this CTA's block: lane l loads 128-bit code
+// chunks g*128 + 32i + l (i < 4) and their two scale bytes.
+__device__ __forceinline__ void gqmv_load(const uint32_t* __restrict__ wc, const Args& a, int e, int nr, uint32_t chunks,
+                                          int r, uint32_t g, uint4 (&qb)[4], uint32_t (&sb)[4]) {
+  const uint32_t lane = threadIdx.x & 31u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t c = g * 128u + (uint32_t)i * 32u + lane;
+    if (r < nr && c < chunks) {
+      const size_t wrow = (size_t)e * a.N + blockIdx.x * QV_ROWS + r;
+      qb[i] = __ldg(reinterpret_cast<const uint4*>(wc + wrow * (size_t)(a.K / 8)) + c);
+      sb[i] = __ldg(reinterpret_cast<const unsigned short*>(a.wsc + wrow * (size_t)(a.K / 16)) + c);
+    } else {
+      qb[i] = make_uint4(0, 0, 0, 0);
+      sb[i] = 0;
+    }
+  }
+}
+
+// The rows of one pass against NQ routed x rows held in shared memory: each
+// 8-weight word is dequantized once (the bf16 rounding of the tensor-core
+// path) and multiplied into NQ pairs of fp32 accumulators by packed fp32x2
+// fused multiply-adds.  qb / sb hold the first unit's loads on entry; the
+// next unit's loads are issued before the current unit is computed.
+template <int NQ>
+__device__ __forceinline__ void gqmv_rows(const uint32_t* __restrict__ wc, const Args& a, const float* xs,
+                                          const int* perm, int e, int nr, float d, uint32_t groups, uint32_t chunks,
+                                          uint4 (&qb)[4], uint32_t (&sb)[4], int& ur, uint32_t& ug) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t K = (uint32_t)a.K;
+  float acc[NQ][2];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) acc[q][0] = acc[q][1] = 0.0f;
+  while (ur < nr) {
+    uint4 qc[4];
+    uint32_t sc4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      qc[i] = qb[i];
+      sc4[i] = sb[i];
+    }
+    const int cr = ur;
+    const uint32_t cg = ug;
+    if (++ug == groups) {
+      ug = 0;
+      ur += QV_THREADS / 32;
+    }
+    gqmv_load(wc, a, e, nr, chunks, ur, ug, qb, sb);  // next unit in flight
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t c = cg * 128u + (uint32_t)i * 32u + lane;
+      if (c < chunks) {
+        const uint32_t words[4] = {qc[i].x, qc[i].y, qc[i].z, qc[i].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {  // 8 weights per word, block h / 2 of the chunk
+          const uint4 wb = dequant8_bf16(words[h], e4m3_to_f32((sc4[i] >> (8 * (h >> 1))) & 0xFFu) * d);
+          const uint32_t pw[4] = {wb.x, wb.y, wb.z, wb.w};
+          const uint32_t k0 = c * 32u + (uint32_t)h * 8u;
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            const float4 xa = *reinterpret_cast<const float4*>(xs + xs_index((uint32_t)q, K, k0));
+            const float4 xb = *reinterpret_cast<const float4*>(xs + xs_index((uint32_t)q, K, k0 + 4u));
+            const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              ffma2(acc[q][0], acc[q][1], __uint_as_float(pw[j] << 16), __uint_as_float(pw[j] & 0xFFFF0000u),
+                    xv[2 * j], xv[2 * j + 1]);
+          }
+        }
+      }
+    }
+    if (cg + 1 == groups) {  // row finished: reduce across the warp and store
+      const int n = (int)blockIdx.x * QV_ROWS + cr;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        float t = acc[q][0] + acc[q][1];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (lane == 0) a.y[(size_t)perm[q] * a.N + n] = __float2bfloat16_rn(t);
+        acc[q][0] = acc[q][1] = 0.0f;
+      }
+    }
+  }
+}
+
+// CTA (row block, tile): weight rows n0..n0+15 of the tile's expert against// CTA (row block, tile): weight rows n0..n0+15 of the tile's expert against
 // every pair of the tile, kQmvPairs pairs per pass; x of those pairs in
 // shared memory as fp32 [kQmvPairs][K] in qmv's swizzled 32-element chunks
 // (xs_index): lane l reads chunk l, and the swizzle puts the 8 lanes of a
@@ -646,7 +744,7 @@ __global__ void __launch_bounds__(QV_THREADS) k_gather_qmv(const __nv_bfloat16* 
   const int tile = blockIdx.y;
   if (tile >= *a.ws.ntiles) return;  // uniform per CTA
   const int e = a.ws.tile_expert[tile], row0 = a.ws.tile_row0[tile], nrows = a.ws.tile_rows[tile];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   const int K = a.K, N = a.N;
   const uint32_t chunks = (uint32_t)K / 32u;  // 32 codes (16 bytes) per lane and chunk
   const float d = a.g ? __ldg(a.g + e) / kGlobalEncode : 1.0f;
@@ -657,25 +755,11 @@ __global__ void __launch_bounds__(QV_THREADS) k_gather_qmv(const __nv_bfloat16* 
   const int nr = min(QV_ROWS, N - (int)blockIdx.x * QV_ROWS);
   uint4 qb[4];
   uint32_t sb[4];
-  auto load_unit = [&](int r, uint32_t g) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t c = g * 128u + (uint32_t)i * 32u + (uint32_t)lane;
-      if (r < nr && c < chunks) {
-        const size_t wrow = (size_t)e * N + blockIdx.x * QV_ROWS + r;
-        qb[i] = __ldg(reinterpret_cast<const uint4*>(wc + wrow * (size_t)(K / 8)) + c);
-        sb[i] = __ldg(reinterpret_cast<const unsigned short*>(a.wsc + wrow * (size_t)(K / 16)) + c);
-      } else {
-        qb[i] = make_uint4(0, 0, 0, 0);
-        sb[i] = 0;
-      }
-    }
-  };
   for (int q0 = 0; q0 < nrows; q0 += kQmvPairs) {
     const int nq = min(kQmvPairs, nrows - q0);
     int ur = warp;
     uint32_t ug = 0;
-    load_unit(ur, ug);
+    gqmv_load(wc, a, e, nr, chunks, ur, ug, qb, sb);
     __syncthreads();  // the previous pass is done with xs
     for (int q = 0; q < nq; ++q) {
       const int tok = a.ws.perm[row0 + q0 + q] / a.topk;
@@ -690,71 +774,12 @@ __global__ void __launch_bounds__(QV_THREADS) k_gather_qmv(const __nv_bfloat16* 
       }
     }
     __syncthreads();
-    float acc[kQmvPairs];
-#pragma unroll
-    for (int q = 0; q < kQmvPairs; ++q) acc[q] = 0.0f;
-    while (ur < nr) {
-      uint4 qc[4];
-      uint32_t sc4[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        qc[i] = qb[i];
-        sc4[i] = sb[i];
-      }
-      const int cr = ur;
-      const uint32_t cg = ug;
-      if (++ug == groups) {
-        ug = 0;
-        ur += QV_THREADS / 32;
-      }
-      load_unit(ur, ug);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t c = cg * 128u + (uint32_t)i * 32u + (uint32_t)lane;
-        if (c < chunks) {
-          const uint32_t words[4] = {qc[i].x, qc[i].y, qc[i].z, qc[i].w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {  // 8 weights per word, block h / 2 of the chunk
-            const uint4 wb = dequant8_bf16(words[h], e4m3_to_f32((sc4[i] >> (8 * (h >> 1))) & 0xFFu) * d);
-            const uint32_t pw[4] = {wb.x, wb.y, wb.z, wb.w};
-            float wv[8];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              wv[2 * j] = __uint_as_float(pw[j] << 16);
-              wv[2 * j + 1] = __uint_as_float(pw[j] & 0xFFFF0000u);
-            }
-            const uint32_t k0 = c * 32u + (uint32_t)h * 8u;
-#pragma unroll
-            for (int q = 0; q < kQmvPairs; ++q) {
-              if (q < nq) {
-                const float4 xa = *reinterpret_cast<const float4*>(xs + xs_index((uint32_t)q, (uint32_t)K, k0));
-                const float4 xb = *reinterpret_cast<const float4*>(xs + xs_index((uint32_t)q, (uint32_t)K, k0 + 4u));
-                float t = acc[q];
-                t = fmaf(wv[0], xa.x, t);
-                t = fmaf(wv[1], xa.y, t);
-                t = fmaf(wv[2], xa.z, t);
-                t = fmaf(wv[3], xa.w, t);
-                t = fmaf(wv[4], xb.x, t);
-                t = fmaf(wv[5], xb.y, t);
-                t = fmaf(wv[6], xb.z, t);
-                t = fmaf(wv[7], xb.w, t);
-                acc[q] = t;
-              }
-            }
-          }
-        }
-      }
-      if (cg + 1 == groups) {  // row finished: reduce across the warp and store
-        const int n = (int)blockIdx.x * QV_ROWS + cr;
-#pragma unroll
-        for (int q = 0; q < kQmvPairs; ++q) {
-          float t = acc[q];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-          if (lane == 0 && q < nq) a.y[(size_t)a.ws.perm[row0 + q0 + q] * N + n] = __float2bfloat16_rn(t);
-          acc[q] = 0.0f;
-        }
-      }
+    const int* perm = a.ws.perm + row0 + q0;
+    switch (nq) {
+      case 1: gqmv_rows<1>(wc, a, xs, perm, e, nr, d, groups, chunks, qb, sb, ur, ug); break;
+      case 2: gqmv_rows<2>(wc, a, xs, perm, e, nr, d, groups, chunks, qb, sb, ur, ug); break;
+      case 3: gqmv_rows<3>(wc, a, xs, perm, e, nr, d, groups, chunks, qb, sb, ur, ug); break;
+      default: gqmv_rows<4>(wc, a, xs, perm, e, nr, d, groups, chunks, qb, sb, ur, ug); break;
     }
   }
 }

@@ -91,11 +91,31 @@ nvfp4_status device_info(const char* tag, DeviceInfo* out) {
 
 bool valid_dt(nvfp4_dtype dt) { return dt == NVFP4_DT_F32 || dt == NVFP4_DT_F16 || dt == NVFP4_DT_BF16; }
 
-// Persistent elementwise grid: enough CTAs to fill every SM, never more than
-// the work needs.
-unsigned ew_grid(const DeviceInfo& d, uint64_t work_threads) {
+// CTAs of `fn` (threads per CTA, dynamic shared memory) that fit on one SM
+// at once, cached per kernel.
+int resident_ctas(const void* fn, int threads, size_t smem) {
+  static std::mutex mu;
+  static const void* keys[128];
+  static int vals[128];
+  static int n = 0;
+  std::lock_guard<std::mutex> lk(mu);
+  for (int i = 0; i < n; ++i)
+    if (keys[i] == fn) return vals[i];
+  int b = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, fn, threads, smem) != cudaSuccess || b < 1) b = 1;
+  if (n < 128) {
+    keys[n] = fn;
+    vals[n] = b;
+    ++n;
+  }
+  return b;
+}
+
+// Persistent elementwise grid: every SM filled with as many CTAs of the
+// kernel as are resident at once (one wave), never more than the work needs.
+unsigned ew_grid(const DeviceInfo& d, uint64_t work_threads, int per_sm) {
   uint64_t want = (work_threads + kEwThreads - 1) / kEwThreads;
-  uint64_t cap = (uint64_t)d.sm_count * 8;  // 8 x 256 threads resident per SM
+  uint64_t cap = (uint64_t)d.sm_count * (uint64_t)per_sm;
   if (want > cap) want = cap;
   if (want < 1) want = 1;
   return (unsigned)want;
@@ -191,9 +211,9 @@ static nvfp4_status amax_launch(const char* tag, const nvfp4_amax_item* items, i
     vecs += (uint64_t)(items[i].n / 8 + 1);
   }
   if (a.count == 0) return ok();
-  const unsigned grid = ew_grid(d, (vecs + 3) / 4);
   dispatch_dt(dt, [&](auto tag_t) {
     using T = decltype(tag_t);
+    const unsigned grid = ew_grid(d, (vecs + 3) / 4, resident_ctas((const void*)k_amax<T>, kEwThreads, 0));
     k_amax<T><<<grid, kEwThreads, 0, stream>>>(a);
   });
   return check_launch(tag);
@@ -234,10 +254,7 @@ static nvfp4_status check_quantize(const char* tag, int kind, const void* x, nvf
 
 static ScaleOut scale_out(uint8_t* scales, int64_t K, int group, nvfp4_layout layout) {
   ScaleOut so;
-  so.p = scales;
-  so.blocks_per_row = (uint32_t)(K / group);
-  so.Cp = (uint32_t)((K / group + 3) / 4 * 4);
-  so.swizzled = layout == NVFP4_LAYOUT_SWIZZLED;
+  so.init(scales, (uint32_t)(K / group), layout == NVFP4_LAYOUT_SWIZZLED);
   return so;
 }
 
@@ -269,9 +286,10 @@ static nvfp4_status nvfp4_quantize_launch(const char* tag, const nvfp4_quantize_
   DeviceInfo d;
   nvfp4_status st = device_info(tag, &d);
   if (st != NVFP4_OK) return st;
-  const unsigned grid = ew_grid(d, (uint64_t)q.units * 32u);
   dispatch_dt(dt, [&](auto tag_t) {
     using T = decltype(tag_t);
+    const void* fn = sr ? (const void*)k_nvfp4_quantize<T, true> : (const void*)k_nvfp4_quantize<T, false>;
+    const unsigned grid = ew_grid(d, (uint64_t)q.units * 32u, resident_ctas(fn, kEwThreads, 0));
     if (sr) k_nvfp4_quantize<T, true><<<grid, kEwThreads, 0, stream>>>(q);
     else k_nvfp4_quantize<T><<<grid, kEwThreads, 0, stream>>>(q);
   });
@@ -289,9 +307,10 @@ static nvfp4_status mx_quantize(const char* tag, int kind, const void* x, nvfp4_
   if (st != NVFP4_OK) return st;
   const ScaleOut so = scale_out(scales, K, 32, layout);
   const uint32_t n_half = (uint32_t)(rows * K / 8);
-  const unsigned grid = ew_grid(d, ((uint64_t)n_half + kUnroll - 1) / kUnroll);
   dispatch_dt(dt, [&](auto tag_t) {
     using T = decltype(tag_t);
+    const void* fn = kind == 1 ? (const void*)k_mxfp8_quantize<T> : (const void*)k_mxfp4_quantize<T>;
+    const unsigned grid = ew_grid(d, ((uint64_t)n_half + kUnroll - 1) / kUnroll, resident_ctas(fn, kEwThreads, 0));
     if (kind == 1)
       k_mxfp8_quantize<T><<<grid, kEwThreads, 0, stream>>>(static_cast<const T*>(x), n_half, codes, so,
                                                            (uint32_t)rows);
@@ -341,10 +360,7 @@ nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, int64_t ro
   nvfp4_status st = device_info(tag, &d);
   if (st != NVFP4_OK) return st;
   ScaleOut so;
-  so.p = scales;
-  so.blocks_per_row = (uint32_t)(rows / 16);
-  so.Cp = (uint32_t)((rows / 16 + 3) / 4 * 4);
-  so.swizzled = layout == NVFP4_LAYOUT_SWIZZLED;
+  so.init(scales, (uint32_t)(rows / 16), layout == NVFP4_LAYOUT_SWIZZLED);
   dim3 grid((unsigned)((rows + kColR - 1) / kColR), (unsigned)((cols + kColC - 1) / kColC));
   dispatch_dt(dt, [&](auto tag_t) {
     using T = decltype(tag_t);
@@ -387,9 +403,11 @@ static nvfp4_status dequantize_common(const char* tag, int kind, const uint32_t*
   si.Cp = (uint32_t)((K / group + 3) / 4 * 4);
   si.swizzled = layout == NVFP4_LAYOUT_SWIZZLED;
   const uint32_t n_half = (uint32_t)(rows * K / 8);
-  const unsigned grid = ew_grid(d, n_half);
   dispatch_dt(out_dt, [&](auto tag_t) {
     using T = decltype(tag_t);
+    const void* fn = kind == 1 ? (const void*)k_mxfp8_dequantize<T>
+                     : kind == 2 ? (const void*)k_mxfp4_dequantize<T> : (const void*)k_nvfp4_dequantize<T>;
+    const unsigned grid = ew_grid(d, n_half, resident_ctas(fn, kEwThreads, 0));
     if (kind == 1)
       k_mxfp8_dequantize<T><<<grid, kEwThreads, 0, stream>>>(codes, si, n_half, static_cast<T*>(out));
     else if (kind == 2)
@@ -427,7 +445,7 @@ nvfp4_status nvfp4_swizzle_scales(const uint8_t* lin, int64_t rows, int64_t cols
   nvfp4_status st = device_info("swizzle_scales", &d);
   if (st != NVFP4_OK) return st;
   const uint32_t Rp = (uint32_t)((rows + 127) / 128 * 128), Cp = (uint32_t)((cols + 3) / 4 * 4);
-  const unsigned grid = ew_grid(d, (uint64_t)Rp * Cp);
+  const unsigned grid = ew_grid(d, (uint64_t)Rp * Cp, resident_ctas((const void*)k_swizzle_scales, kEwThreads, 0));
   k_swizzle_scales<<<grid, kEwThreads, 0, stream>>>(lin, (uint32_t)rows, (uint32_t)cols, Rp, Cp, swz);
   return check_launch("swizzle_scales");
 }
@@ -469,8 +487,11 @@ nvfp4_status qqmm(nvfp4_mode mode, int64_t M, int64_t N, int64_t K, const uint32
                      (int)y_dt, d.sm_count, stream, t_msg, sizeof(t_msg));
 }
 
-nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32_t* w_codes, const uint8_t* w_scales,
-                 const float* g_w, int64_t M, int64_t N, int64_t K, void* y, nvfp4_stream_t stream) {
+// pdl: the tensor-core kernel's PDL form (qmv_pdl); the SIMT kernel always
+// launches in plain stream order.
+static nvfp4_status qmv_launch(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32_t* w_codes,
+                               const uint8_t* w_scales, const float* g_w, int64_t M, int64_t N, int64_t K, void* y,
+                               nvfp4_stream_t stream, bool pdl) {
   if (!valid_dt(x_dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[qmv] dtype must be float32, float16 or bfloat16");
   if ((g_x == nullptr) != (g_w == nullptr))
     return fail(NVFP4_ERR_INVALID_ARG,
@@ -504,10 +525,26 @@ nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32
       using T = decltype(tag_t);
       auto go = [&](auto kern) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess) kern<<<grid, qtc::THREADS, smem, stream>>>(mw, a);
+        if (e != cudaSuccess) return;
+        if (!pdl) {
+          kern<<<grid, qtc::THREADS, smem, stream>>>(mw, a);
+          return;
+        }
+        cudaLaunchConfig_t cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(qtc::THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, kern, mw, a);
       };
-      if (M == 1) go(qtc::k_qmv_tc<T, 1>);
-      else go(qtc::k_qmv_tc<T, 2>);
+      if (M == 1) pdl ? go(qtc::k_qmv_tc<T, 1, true>) : go(qtc::k_qmv_tc<T, 1>);
+      else pdl ? go(qtc::k_qmv_tc<T, 2, true>) : go(qtc::k_qmv_tc<T, 2>);
     });
   } else {
     const size_t smem = (size_t)M * K * sizeof(float);
@@ -532,6 +569,17 @@ nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32
   }
   if (e != cudaSuccess) return fail(NVFP4_ERR_CUDA, "[qmv] %s", cudaGetErrorString(e));
   return check_launch("qmv");
+}
+
+nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32_t* w_codes, const uint8_t* w_scales,
+                 const float* g_w, int64_t M, int64_t N, int64_t K, void* y, nvfp4_stream_t stream) {
+  return qmv_launch(x, x_dt, g_x, w_codes, w_scales, g_w, M, N, K, y, stream, false);
+}
+
+nvfp4_status qmv_pdl(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32_t* w_codes,
+                     const uint8_t* w_scales, const float* g_w, int64_t M, int64_t N, int64_t K, void* y,
+                     nvfp4_stream_t stream) {
+  return qmv_launch(x, x_dt, g_x, w_codes, w_scales, g_w, M, N, K, y, stream, true);
 }
 
 size_t gather_qmm_workspace_size(int64_t T, int64_t topk, int64_t E) {

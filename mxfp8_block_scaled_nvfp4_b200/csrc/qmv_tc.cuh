@@ -170,7 +170,14 @@ __device__ __forceinline__ bool x_planes(const T* xs, float gx, uint32_t M, uint
   return exact;
 }
 
-template <typename T, int MM>
+// PDL = true: the kernel is launched with programmatic stream serialization
+// (qmv_pdl).  Its weight codes, weight scales and g_w are read without
+// waiting for the previous kernel of the stream (the caller guarantees that
+// no pending work writes them); x, g_x and y only after griddepcontrol.wait
+// (all prerequisite grids complete, their writes visible).  Each CTA lets
+// the next launch begin at once (launch_dependents), so a chain of calls
+// streams the next weight while the previous call drains.
+template <typename T, int MM, bool PDL = false>
 __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ CUtensorMap tmap_w, Args a) {
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -182,7 +189,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_flag;
 
-  const float gx = a.g_x ? __ldg(a.g_x) : kGlobalEncode;
+  float gx = kGlobalEncode;
+  if (!PDL) gx = a.g_x ? __ldg(a.g_x) : kGlobalEncode;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   Layout L;
@@ -233,12 +241,26 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
     mbar_init(smem_u32(&xbar), 1);
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    // x first, one bulk copy (the rows are contiguous, 16-byte aligned and a
-    // multiple of 512 bytes long), so it does not queue behind the weight
-    // stream; then the weight stream, before TMEM allocation and the prologue
-    mbar_expect_tx(smem_u32(&xbar), xbytes);
-    bulk_load(sbase + L.xraw, a.x, xbytes, smem_u32(&xbar));
-    for (; issued < S && issued < kb_count; ++issued) issue(issued);
+    if (PDL) {
+      // the weight before the wait for the previous kernel, x after it
+      asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+      for (; issued < S && issued < kb_count; ++issued) issue(issued);
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      mbar_expect_tx(smem_u32(&xbar), xbytes);
+      bulk_load(sbase + L.xraw, a.x, xbytes, smem_u32(&xbar));
+    } else {
+      // x first, one bulk copy (the rows are contiguous, 16-byte aligned and
+      // a multiple of 512 bytes long), so it does not queue behind the weight
+      // stream; then the weight stream, before TMEM allocation and the prologue
+      mbar_expect_tx(smem_u32(&xbar), xbytes);
+      bulk_load(sbase + L.xraw, a.x, xbytes, smem_u32(&xbar));
+      for (; issued < S && issued < kb_count; ++issued) issue(issued);
+    }
+  }
+  if (PDL) {
+    // every thread that reads g_x, or later x_hat's inputs or writes y
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    gx = a.g_x ? __ldg(a.g_x) : kGlobalEncode;
   }
   // zero the plane tiles (a plane row is nonzero only inside its own
   // 16-block: the prologue writes those bytes alone), fill the unit scale tile

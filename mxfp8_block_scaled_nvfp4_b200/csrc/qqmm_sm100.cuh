@@ -78,7 +78,27 @@ constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_SF = 256;       // scale-factor columns start here
 constexpr uint32_t TMEM_SF_STAGE = 48;  // 16 (A) + 32 (B) columns per stage
-constexpr uint32_t kWaitLimit = 1u << 26;
+// Polls of a bounded mbarrier wait before it gives up.  A test build of the
+// library lowers it (-DNVFP4_WAIT_LIMIT=...) so that a withheld stage (below)
+// times out within milliseconds.
+#ifndef NVFP4_WAIT_LIMIT
+#define NVFP4_WAIT_LIMIT (1u << 26)
+#endif
+constexpr uint32_t kWaitLimit = NVFP4_WAIT_LIMIT;
+
+// Test builds only (-DNVFP4_TEST_WITHHOLD_STAGE=s): CTA 0 of the dense GEMM
+// issues neither the arrival nor any copy of its stage s, so the MMA warp's
+// bounded wait on that stage runs out and the kernel takes its timeout path
+// (error word, drain, TMEM freed).  No copy is left in flight: nothing is
+// issued for the withheld stage.  The library itself is built without it.
+__device__ __forceinline__ bool withheld_stage(uint32_t it) {
+#ifdef NVFP4_TEST_WITHHOLD_STAGE
+  return blockIdx.x == 0 && it == (uint32_t)(NVFP4_TEST_WITHHOLD_STAGE);
+#else
+  (void)it;
+  return false;
+#endif
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -458,6 +478,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
           if (ntl > tiles_per_stage) ntl = tiles_per_stage;
           const uint32_t sfa_bytes = ntl * 512u, sfb_bytes = ntl * 512u * (b_second ? 2u : 1u);
           const uint32_t bar = smem_u32(&full_bar[s]);
+          if (withheld_stage(it)) continue;
           mbar_expect_tx(bar, A_STAGE + (wide ? B_STAGE : B_STAGE / 2) + sfa_bytes + sfb_bytes);
           tma_load_2d(sbase + SMEM_A + s * A_STAGE, &tmap_a, (int)(kb * BKB), tile_m, bar);
           tma_load_2d(sbase + SMEM_B + s * B_STAGE, wide ? &tmap_b : &tmap_b128, (int)(kb * BKB), tile_n, bar);
@@ -599,7 +620,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qqmm(const __grid_constant__ CUt
           const uint32_t g0 = kb * tiles_per_stage;
           uint32_t ntl = p.sf_groups > g0 ? p.sf_groups - g0 : 0;
           if (ntl > tiles_per_stage) ntl = tiles_per_stage;
-          if (ntl == 0) continue;
+          if (ntl == 0 || withheld_stage(it)) continue;
           const uint32_t bytes = ntl * 512u, bar = smem_u32(&full_bar[s]);
           bulk_load(sbase + SMEM_SFA + s * SFA_STAGE, p.sfa + ((size_t)tm * p.sf_groups + g0) * 512u, bytes, bar);
           bulk_load(sbase + SMEM_SFB + s * SFB_STAGE, p.sfb + ((size_t)(tile_n / 128) * p.sf_groups + g0) * 512u,

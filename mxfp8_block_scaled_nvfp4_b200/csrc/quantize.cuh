@@ -86,14 +86,21 @@ struct ScaleOut {
   uint32_t blocks_per_row;  // K / group
   uint32_t Cp;              // padded columns (swizzled) = ceil4(blocks_per_row)
   bool swizzled;
-  __device__ __forceinline__ void store(uint32_t block, uint32_t byte) const {
-    if (!swizzled) {
-      p[block] = (uint8_t)byte;
-    } else {
-      uint32_t r = block / blocks_per_row, c = block - r * blocks_per_row;
-      p[swizzled_offset(r, c, Cp)] = (uint8_t)byte;
-    }
+  FastDiv bpr;              // division by blocks_per_row (block index -> row)
+  __host__ void init(uint8_t* scales, uint32_t bpr_, bool swz) {
+    p = scales;
+    blocks_per_row = bpr_;
+    Cp = (bpr_ + 3u) / 4u * 4u;
+    swizzled = swz;
+    bpr.init(bpr_ ? bpr_ : 1u);
   }
+  // byte offset of block `block` (flat index over [rows, blocks_per_row])
+  __device__ __forceinline__ uint32_t offset(uint32_t block) const {
+    if (!swizzled) return block;
+    const uint32_t r = bpr.div(block), c = block - r * blocks_per_row;
+    return swizzled_offset(r, c, Cp);
+  }
+  __device__ __forceinline__ void store(uint32_t block, uint32_t byte) const { p[offset(block)] = (uint8_t)byte; }
 };
 
 // Zero the padding bytes of a 128x4-tile scale buffer: rows [rows, Rp) and
@@ -247,12 +254,12 @@ __device__ __forceinline__ void store_scales(const ScaleOut& so, uint32_t hb, ui
   bool packed = lead + 8u <= n_half;  // all four blocks exist
   uint32_t off = b0;
   if (so.swizzled) {
-    const uint32_t r = b0 / so.blocks_per_row, c = b0 - r * so.blocks_per_row;
+    const uint32_t r = so.bpr.div(b0), c = b0 - r * so.blocks_per_row;
     packed = packed && (c & 3u) == 0 && c + 4u <= so.blocks_per_row;
     off = swizzled_offset(r, c, so.Cp);
   }
   if (packed) {
-    if ((lane & 7u) == 0) *reinterpret_cast<uint32_t*>(so.p + off) = s | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    if ((lane & 7u) == 0) *reinterpret_cast<uint32_t*>(so.p + off) = __byte_perm(s | (s1 << 8), s2 | (s3 << 8), 0x5410);
   } else if ((lane & 1u) == 0 && hb < n_half) {
     so.store(hb >> 1, s);
   }
@@ -260,19 +267,34 @@ __device__ __forceinline__ void store_scales(const ScaleOut& so, uint32_t hb, ui
 
 template <typename T, bool SR = false>
 __global__ void __launch_bounds__(kEwThreads) k_nvfp4_quantize(const __grid_constant__ QuantSegs q) {
+  // k = E / f8(s) for every scale byte s a block can get (0 <= s <= 0x7E:
+  // t >= 0 and the conversion saturates), per tensor: the IEEE quotient the
+  // method takes per block, computed once per CTA instead of once per block
+  __shared__ float ktab[kMaxSegs][128];
+  __shared__ float etab[kMaxSegs];
   const uint32_t lane = threadIdx.x & 31u;
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
   Raw8<T> nxt[kUnroll];
-  load_unit<T>(q, warp, lane, nxt);
+  load_unit<T>(q, warp, lane, nxt);  // the first unit's loads before the table
+  for (uint32_t i = threadIdx.x; i < q.count * 128u; i += blockDim.x) {
+    const QuantSeg& sg = q.s[i >> 7];
+    const float E = sg.g ? kGlobalEncode / __ldg(sg.g) : 1.0f;
+    const float fs = e4m3_to_f32(i & 127u);
+    ktab[i >> 7][i & 127u] = fs != 0.0f ? E / fs : 0.0f;
+    if ((i & 127u) == 0) etab[i >> 7] = E;
+  }
+  __syncthreads();
   for (uint32_t unit = warp; unit < q.units; unit += nwarps) {
     Raw8<T> cur[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) cur[u] = nxt[u];
     load_unit<T>(q, unit + nwarps, lane, nxt);  // next unit's loads in flight during this one
-    const QuantSeg& sg = q.s[seg_of(q, unit)];
+    const uint32_t si = seg_of(q, unit);
+    const QuantSeg& sg = q.s[si];
     const uint32_t base = (unit - sg.first_unit) * kUnitHalf;
-    const float E = sg.g ? kGlobalEncode / __ldg(sg.g) : 1.0f;
+    const float E = etab[si];
+    const float* kt = ktab[si];
     // stochastic rounding: half-blocks 2c and 2c + 1 share generator call c
     // (words x, y for the even one, z, w for the odd one).  Over iterations
     // (u, u + 1) the even lane of a pair calls the generator for u and the
@@ -308,19 +330,15 @@ __global__ void __launch_bounds__(kEwThreads) k_nvfp4_quantize(const __grid_cons
       float t = a / kE2M1Max;
       t = t * E;
       const uint32_t s = f32_to_e4m3(t);
-      const float fs = e4m3_to_f32(s);
       uint32_t w = 0;
-      if (fs != 0.0f) {
-        const float k = E / fs;
-        float qv[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) qv[j] = v[j] * k;
+      if (s != 0u) {  // f8(s) != 0
+        const float k = kt[s];
         if constexpr (SR) {
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            w |= e2m1_sr(qv[j], ((j < 4 ? wa[u] : wb[u]) >> (8 * (j & 3))) & 0xFFu) << (4 * j);
+            w |= e2m1_sr(v[j] * k, ((j < 4 ? wa[u] : wb[u]) >> (8 * (j & 3))) & 0xFFu) << (4 * j);
         } else {
-          w = f32x8_to_e2m1x8(qv);
+          w = scaled_e2m1x8(v, k);
         }
       }
       if (hb < sg.n_half) sg.codes[hb] = w;

@@ -58,6 +58,7 @@ SIGNATURES = [
     ("nvfp4_swizzle_scales", _I, [_P, _I64, _I64, _P, _P]),
     ("qqmm", _I, [_I, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
     ("qmv", _I, [_P, _I, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    ("qmv_pdl", _I, [_P, _I, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     ("gather_qmm", _I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     ("gather_qmm_kn", _I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     ("gather_qmm_workspace_size", _SZ, [_I64, _I64, _I64]),
@@ -409,8 +410,10 @@ def qqmm_vjp(x: torch.Tensor, w: torch.Tensor, cotan: torch.Tensor, g_x: torch.T
     return dx, dw
 
 
-def qmv(x: torch.Tensor, w_codes, w_scales, g_x=None, g_w=None, out=None) -> torch.Tensor:
-    """y [M, N] (x's dtype) = x_hat . w_hat^T, M <= 8, w pre-quantized (LINEAR scales)."""
+def qmv(x: torch.Tensor, w_codes, w_scales, g_x=None, g_w=None, out=None, pdl: bool = False) -> torch.Tensor:
+    """y [M, N] (x's dtype) = x_hat . w_hat^T, M <= 8, w pre-quantized (LINEAR scales).
+    pdl=True calls qmv_pdl: for chains of decode calls whose weight (codes,
+    scales, g_w) is not written by work still pending on the device."""
     M, K = x.shape
     N = w_codes.shape[0]
     _need_bytes(w_codes, N * (K // 8) * 4, "w_codes")
@@ -422,8 +425,9 @@ def qmv(x: torch.Tensor, w_codes, w_scales, g_x=None, g_w=None, out=None) -> tor
     _need_cuda(x, w_codes, w_scales, g_x, g_w, out)
     if out is None:
         out = torch.empty(M, N, dtype=x.dtype, device=x.device)
-    _check(lib().qmv(_ptr(x), DT[x.dtype], _ptr(g_x), _ptr(w_codes), _ptr(w_scales), _ptr(g_w), M, N, K,
-                     _ptr(out), _stream()))
+    fn = lib().qmv_pdl if pdl else lib().qmv
+    _check(fn(_ptr(x), DT[x.dtype], _ptr(g_x), _ptr(w_codes), _ptr(w_scales), _ptr(g_w), M, N, K, _ptr(out),
+              _stream()))
     return out
 
 

@@ -98,3 +98,49 @@ def test_qmv_tensor_path_falls_back_on_subnormal_x_hat(nv, orc):
     xh = orc.to_f64(orc.nvfp4_quantize_dequantize(raw(x), "f16", g_x.item()), "f16")
     assert np.any((np.abs(xh) < 2.0 ** -14) & (xh != 0))
     check_gemm_output(raw(y), r, "f16", orc)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("M,N,K", [(1, 200, 1024), (2, 130, 512), (1, 14336, 4096)])
+def test_qmv_pdl_equals_qmv(nv, dt, M, N, K):
+    """qmv_pdl (programmatic dependent launch, weight streamed before the
+    previous kernel finishes) computes exactly what qmv computes."""
+    from mxfp8_block_scaled_nvfp4_b200 import workloads
+    x = workloads.normal((M, K), 1.0, 60 + M, TORCH_DT[dt]).cuda()
+    w = workloads.normal((N, K), 0.02, 61, TORCH_DT[dt]).cuda()
+    g_x, g_w = nv.amax(x), nv.amax(w)
+    wc, ws = nv.nvfp4_quantize(w, g_w, "linear")
+    torch.cuda.synchronize()  # the weight is written before any qmv_pdl call
+    y = nv.qmv(x, wc, ws, g_x, g_w)
+    y2 = nv.qmv(x, wc, ws, g_x, g_w, pdl=True)
+    nv.check_device_errors()
+    assert torch.equal(y.view(torch.int16) if dt == "bf16" else y, y2.view(torch.int16) if dt == "bf16" else y2)
+
+
+def test_qmv_pdl_chain_orders_reads_and_writes(nv):
+    """A chain of qmv_pdl calls where each call's x is the previous call's
+    output (read after write) and the last call writes over the first
+    call's input (write after read), launched back to back: the same bits as
+    the same chain of qmv calls."""
+    from mxfp8_block_scaled_nvfp4_b200 import workloads
+    K = 4096
+    ws_ = [workloads.normal((K, K), 0.02, 70 + i, torch.bfloat16).cuda() for i in range(3)]
+    q = [nv.nvfp4_quantize(w, None, "linear") for w in ws_]
+    torch.cuda.synchronize()
+
+    def chain(pdl):
+        a = workloads.normal((1, K), 1.0, 80, torch.bfloat16).cuda()
+        b = torch.empty_like(a)
+        c = torch.empty_like(a)
+        torch.cuda.synchronize()
+        for _ in range(4):
+            nv.qmv(a, *q[0], out=b, pdl=pdl)   # b = f(a)
+            nv.qmv(b, *q[1], out=c, pdl=pdl)   # c = f(b): reads what the call before wrote
+            nv.qmv(c, *q[2], out=a, pdl=pdl)   # a = f(c): overwrites the first call's input
+        torch.cuda.synchronize()
+        return a, b, c
+    want = chain(False)
+    got = chain(True)
+    nv.check_device_errors()
+    for u, v in zip(want, got):
+        assert torch.equal(u.view(torch.int16), v.view(torch.int16))
