@@ -176,6 +176,16 @@ NVFP4_API nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, 
                                                  const float* g, uint32_t* codes, uint8_t* scales,
                                                  nvfp4_layout layout, nvfp4_stream_t stream);
 
+/* nvfp4_quantize_columnwise with stochastic rounding of the codes: equal to
+ * nvfp4_quantize_sr of the transposed, contiguous matrix x^T [cols, rows]
+ * with the same seed (its random bits indexed by the flat position in x^T).
+ * The backward pass quantizes the transposed upstream gradient this way
+ * ([P1] QQMatmul::vjp).  Arguments and errors as nvfp4_quantize_columnwise,
+ * plus the 64-bit seed. */
+NVFP4_API nvfp4_status nvfp4_quantize_columnwise_sr(const void* x, nvfp4_dtype dt, int64_t rows, int64_t cols,
+                                                    const float* g, uint64_t seed, uint32_t* codes, uint8_t* scales,
+                                                    nvfp4_layout layout, nvfp4_stream_t stream);
+
 /* f4 -- NVFP4 quantize with stochastic rounding of the codes (the pages
  * reserve it: [P2] fp_quantize_rowwise<..., USE_SR> with rbits "reserved for
  * future use"; this library's reading).  Scales exactly as nvfp4_quantize;
@@ -262,6 +272,21 @@ NVFP4_API nvfp4_status qqmm(nvfp4_mode mode, int64_t M, int64_t N, int64_t K, co
 NVFP4_API nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32_t* w_codes,
                  const uint8_t* w_scales, const float* g_w, int64_t M, int64_t N, int64_t K,
                  void* y, nvfp4_stream_t stream);
+
+/* f3 -- qmv in the MX modes ([P2] QQMatmul::eval_gpu, M = 1 branch, which
+ * quantize-dequantizes x with the mode's group size and bits before fp_qmv):
+ *   x_hat = T(code(q) * 2^(s-127)) per 32-block of x (s = ue8m0_round_up(
+ *   amax / 448) for MXFP8, amax / 6 for MXFP4, codes as mxfp8_quantize /
+ *   mxfp4_quantize);  y[m,n] = T(sum_k x_hat[m,k] * code(q[n,k]) *
+ *   2^(sw[n,k/32]-127)), fp32 accumulation.  No global scales ([P1]
+ *   validate_global_scale: nvfp4 only).
+ * mode NVFP4_MODE_MXFP8 (w_codes [N, K/4], e4m3 bytes) or NVFP4_MODE_MXFP4
+ * (w_codes [N, K/8], e2m1 nibbles); w_scales LINEAR e8m0 [N, K/32]; x [M, K]
+ * of x_dt, 1 <= M <= 8, K % 32 == 0, M*K*4 bytes <= 160 KiB; y [M, N] of
+ * x_dt.  A SIMT kernel (a warp per weight row). */
+NVFP4_API nvfp4_status qmv_mx(nvfp4_mode mode, const void* x, nvfp4_dtype x_dt, const uint32_t* w_codes,
+                              const uint8_t* w_scales, int64_t M, int64_t N, int64_t K, void* y,
+                              nvfp4_stream_t stream);
 
 /* qmv for chains of decode calls whose weights stay fixed (the layers of a
  * model at decode time): the same arguments, checks and result as qmv, but

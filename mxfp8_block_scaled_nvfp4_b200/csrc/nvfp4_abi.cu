@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "nvfp4.h"
 #include "common.cuh"
@@ -266,6 +267,7 @@ static nvfp4_status nvfp4_quantize_launch(const char* tag, const nvfp4_quantize_
   QuantSegs q;
   memset(&q, 0, sizeof(q));
   q.seed = seed;
+  bool v8 = true;  // 256-bit loads need every input 32-byte aligned
   for (int i = 0; i < count; ++i) {
     const nvfp4_quantize_item& it = items[i];
     bool empty = false;
@@ -278,9 +280,10 @@ static nvfp4_status nvfp4_quantize_launch(const char* tag, const nvfp4_quantize_
     sg.codes = it.codes;
     sg.so = scale_out(it.scales, it.K, 16, it.layout);
     sg.rows = (uint32_t)it.rows;
-    sg.n_half = (uint32_t)(it.rows * it.K / 8);
+    sg.n_blk = (uint32_t)(it.rows * it.K / 16);
     sg.first_unit = q.units;
-    q.units += (sg.n_half + kUnitHalf - 1) / kUnitHalf;
+    q.units += (sg.n_blk + kUnitBlk - 1) / kUnitBlk;
+    v8 = v8 && (reinterpret_cast<uintptr_t>(it.x) & 31u) == 0;
   }
   if (q.count == 0) return ok();  // nothing to write: no device work, no device query
   DeviceInfo d;
@@ -288,10 +291,12 @@ static nvfp4_status nvfp4_quantize_launch(const char* tag, const nvfp4_quantize_
   if (st != NVFP4_OK) return st;
   dispatch_dt(dt, [&](auto tag_t) {
     using T = decltype(tag_t);
-    const void* fn = sr ? (const void*)k_nvfp4_quantize<T, true> : (const void*)k_nvfp4_quantize<T, false>;
-    const unsigned grid = ew_grid(d, (uint64_t)q.units * 32u, resident_ctas(fn, kEwThreads, 0));
-    if (sr) k_nvfp4_quantize<T, true><<<grid, kEwThreads, 0, stream>>>(q);
-    else k_nvfp4_quantize<T><<<grid, kEwThreads, 0, stream>>>(q);
+    auto go = [&](auto kern) {
+      const unsigned grid = ew_grid(d, (uint64_t)q.units * 32u, resident_ctas((const void*)kern, kEwThreads, 0));
+      kern<<<grid, kEwThreads, 0, stream>>>(q);
+    };
+    if (sr) v8 ? go(k_nvfp4_quantize<T, true, true>) : go(k_nvfp4_quantize<T, true, false>);
+    else v8 ? go(k_nvfp4_quantize<T, false, true>) : go(k_nvfp4_quantize<T, false, false>);
   });
   return check_launch(tag);
 }
@@ -339,9 +344,9 @@ nvfp4_status nvfp4_quantize_sr(const void* x, nvfp4_dtype dt, int64_t rows, int6
   return nvfp4_quantize_launch("quantize_sr", &it, 1, dt, stream, true, seed);
 }
 
-nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, int64_t rows, int64_t cols, const float* g,
-                                       uint32_t* codes, uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
-  const char* tag = "quantize_columnwise";
+static nvfp4_status columnwise_launch(const char* tag, const void* x, nvfp4_dtype dt, int64_t rows, int64_t cols,
+                                      const float* g, uint32_t* codes, uint8_t* scales, nvfp4_layout layout,
+                                      nvfp4_stream_t stream, bool sr, uint64_t seed) {
   if (!valid_dt(dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[%s] dtype must be float32, float16 or bfloat16", tag);
   if (layout != NVFP4_LAYOUT_LINEAR && layout != NVFP4_LAYOUT_SWIZZLED)
     return fail(NVFP4_ERR_INVALID_ARG, "[%s] unknown scale layout", tag);
@@ -364,10 +369,25 @@ nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, int64_t ro
   dim3 grid((unsigned)((rows + kColR - 1) / kColR), (unsigned)((cols + kColC - 1) / kColC));
   dispatch_dt(dt, [&](auto tag_t) {
     using T = decltype(tag_t);
-    k_nvfp4_quantize_columnwise<T><<<grid, kColThreads, 0, stream>>>(static_cast<const T*>(x), (uint32_t)rows,
-                                                                      (uint32_t)cols, g, codes, so);
+    if (sr)
+      k_nvfp4_quantize_columnwise<T, true><<<grid, kColThreads, 0, stream>>>(static_cast<const T*>(x), (uint32_t)rows,
+                                                                            (uint32_t)cols, g, codes, so, seed);
+    else
+      k_nvfp4_quantize_columnwise<T><<<grid, kColThreads, 0, stream>>>(static_cast<const T*>(x), (uint32_t)rows,
+                                                                        (uint32_t)cols, g, codes, so);
   });
   return check_launch(tag);
+}
+
+nvfp4_status nvfp4_quantize_columnwise(const void* x, nvfp4_dtype dt, int64_t rows, int64_t cols, const float* g,
+                                       uint32_t* codes, uint8_t* scales, nvfp4_layout layout, nvfp4_stream_t stream) {
+  return columnwise_launch("quantize_columnwise", x, dt, rows, cols, g, codes, scales, layout, stream, false, 0);
+}
+
+nvfp4_status nvfp4_quantize_columnwise_sr(const void* x, nvfp4_dtype dt, int64_t rows, int64_t cols, const float* g,
+                                          uint64_t seed, uint32_t* codes, uint8_t* scales, nvfp4_layout layout,
+                                          nvfp4_stream_t stream) {
+  return columnwise_launch("quantize_columnwise_sr", x, dt, rows, cols, g, codes, scales, layout, stream, true, seed);
 }
 
 nvfp4_status mxfp8_quantize(const void* x, nvfp4_dtype dt, int64_t rows, int64_t K, uint32_t* codes,
@@ -574,6 +594,50 @@ static nvfp4_status qmv_launch(const void* x, nvfp4_dtype x_dt, const float* g_x
 nvfp4_status qmv(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32_t* w_codes, const uint8_t* w_scales,
                  const float* g_w, int64_t M, int64_t N, int64_t K, void* y, nvfp4_stream_t stream) {
   return qmv_launch(x, x_dt, g_x, w_codes, w_scales, g_w, M, N, K, y, stream, false);
+}
+
+nvfp4_status qmv_mx(nvfp4_mode mode, const void* x, nvfp4_dtype x_dt, const uint32_t* w_codes,
+                    const uint8_t* w_scales, int64_t M, int64_t N, int64_t K, void* y, nvfp4_stream_t stream) {
+  if (mode != NVFP4_MODE_MXFP8 && mode != NVFP4_MODE_MXFP4)
+    return fail(NVFP4_ERR_INVALID_ARG, "[qmv_mx] mode must be mxfp8 or mxfp4 (nvfp4: use qmv)");
+  if (!valid_dt(x_dt)) return fail(NVFP4_ERR_UNSUPPORTED, "[qmv_mx] dtype must be float32, float16 or bfloat16");
+  if (M < 1 || M > kQmvMaxM)
+    return fail(NVFP4_ERR_INVALID_ARG, "[qmv_mx] M must be in [1, %d], got %lld", kQmvMaxM, (long long)M);
+  if (N < 0 || K < 32 || K % 32 != 0 || N > (1 << 30))
+    return fail(NVFP4_ERR_INVALID_ARG, "[qmv_mx] bad shape N=%lld K=%lld (K %% 32 == 0)", (long long)N, (long long)K);
+  if (M * K * 4 > 160 * 1024)
+    return fail(NVFP4_ERR_UNSUPPORTED, "[qmv_mx] M*K*4 bytes of x_hat must fit 160 KiB of shared memory");
+  if (N > 0 && (!x || !w_codes || !w_scales || !y)) return fail(NVFP4_ERR_INVALID_ARG, "[qmv_mx] null pointer");
+  if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y))
+    return fail(NVFP4_ERR_INVALID_ARG, "[qmv_mx] tensor pointers must be 16-byte aligned");
+  if (N == 0) return ok();
+  DeviceInfo d;
+  nvfp4_status st = device_info("qmv_mx", &d);
+  if (st != NVFP4_OK) return st;
+  const size_t smem = (size_t)M * K * sizeof(float);
+  uint64_t grid = ((uint64_t)N + (kQmvThreads / 32) - 1) / (kQmvThreads / 32);
+  if (grid > (uint64_t)d.sm_count) grid = d.sm_count;
+  cudaError_t e = cudaSuccess;
+  dispatch_dt(x_dt, [&](auto tag_t) {
+    using T = decltype(tag_t);
+    auto go = [&](auto kern) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess)
+        kern<<<(unsigned)grid, kQmvThreads, smem, stream>>>(static_cast<const T*>(x), w_codes, w_scales, (int)M,
+                                                            (int)N, (int)K, static_cast<T*>(y));
+    };
+    auto pick = [&](auto mode_tag) {
+      constexpr int MD = decltype(mode_tag)::value;
+      if (M == 1) go(k_qmv_mx<T, MD, 1>);
+      else if (M == 2) go(k_qmv_mx<T, MD, 2>);
+      else if (M <= 4) go(k_qmv_mx<T, MD, 4>);
+      else go(k_qmv_mx<T, MD, 8>);
+    };
+    if (mode == NVFP4_MODE_MXFP8) pick(std::integral_constant<int, 1>{});
+    else pick(std::integral_constant<int, 2>{});
+  });
+  if (e != cudaSuccess) return fail(NVFP4_ERR_CUDA, "[qmv_mx] %s", cudaGetErrorString(e));
+  return check_launch("qmv_mx");
 }
 
 nvfp4_status qmv_pdl(const void* x, nvfp4_dtype x_dt, const float* g_x, const uint32_t* w_codes,

@@ -197,3 +197,183 @@ __global__ void __launch_bounds__(kQmvThreads) k_qmv(
 }
 
 }  // namespace nvfp4
+
+namespace nvfp4 {
+
+// ---------------------------------------------------------------------------
+// qmv in the MX modes: the same M = 1 route ("mlx 0.30.7.2 -> 0.30.7.6"
+// diff, page 7, qqmm.cpp, QQMatmul::eval_gpu: fp_quantize_dequantize of x
+// with the mode's group size and bits, then fp_qmv), with 32-element blocks
+// and e8m0 scales rounded up, no global scales:
+//   MODE 1 (MXFP8): codes e4m3 (4 per uint32), x_hat[k] = T(e4m3(qx) * 2^(sx-127))
+//   MODE 2 (MXFP4): codes e2m1 (8 per uint32), x_hat[k] = T(e2m1(qx) * 2^(sx-127))
+//   y[m, n] = T( sum_b 2^(sw[n,b]-127) * sum_{k in b} x_hat[m, k] * code(q[n, k]) ),
+// fp32 accumulation (the per-block power of two is exact in fp32).
+// Same kernel shape as k_qmv: x_hat for all M rows in shared memory (fp32,
+// swizzled 32-element chunks), a warp per weight row, 128-bit coalesced
+// code loads with the next unit's loads in flight.
+// ---------------------------------------------------------------------------
+template <typename T, int MODE>
+__device__ __forceinline__ void qmv_mx_prologue(const T* __restrict__ x, uint32_t M, uint32_t K, float4* xs4) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t n_half = M * K / 8u;  // 4 half-blocks per 32-block, 8 per warp step
+  for (uint32_t base = (threadIdx.x & ~31u); base < n_half; base += blockDim.x) {
+    const uint32_t hb = base + lane;
+    float v[8];
+    if (hb < n_half) {
+      load8<T>(x + (size_t)hb * 8, v);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = 0.0f;
+    }
+    float a = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[j]));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+    const uint32_t s = f32_to_ue8m0_rp(a / (MODE == 1 ? kE4M3Max : kE2M1Max));
+    const float sc = ue8m0_to_f32(s);
+    const float k = 1.0f / sc;
+    float dq[8];
+    if constexpr (MODE == 1) {
+      float c0[4], c1[4];
+      e4m3x4_to_f32(f32x4_to_e4m3x4(v[0] * k, v[1] * k, v[2] * k, v[3] * k), c0);
+      e4m3x4_to_f32(f32x4_to_e4m3x4(v[4] * k, v[5] * k, v[6] * k, v[7] * k), c1);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        dq[j] = Elem<T>::to_f(Elem<T>::from_f(c0[j] * sc));
+        dq[4 + j] = Elem<T>::to_f(Elem<T>::from_f(c1[j] * sc));
+      }
+    } else {
+      float q[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) q[j] = v[j] * k;
+      const uint32_t w = f32x8_to_e2m1x8(q);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dq[j] = Elem<T>::to_f(Elem<T>::from_f(e2m1_value(w >> (4 * j)) * sc));
+    }
+    if (hb < n_half) {
+      const uint32_t m = (hb * 8u) / K, k0 = hb * 8u - m * K;
+      const uint32_t i0 = xs_index(m, K, k0), i1 = xs_index(m, K, k0 + 4);
+      xs4[i0 >> 2] = make_float4(dq[0], dq[1], dq[2], dq[3]);
+      xs4[i1 >> 2] = make_float4(dq[4], dq[5], dq[6], dq[7]);
+    }
+  }
+}
+
+// Weight row n's chunk c of 128 bits: 32 e2m1 codes (MXFP4, one 32-block)
+// or 16 e4m3 codes (MXFP8, half a block) starting at element kc; values
+// into v (the codes' values, unscaled).
+template <int MODE>
+__device__ __forceinline__ void mx_chunk_values(uint4 q, float (&v)[32]) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  if constexpr (MODE == 2) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float t[8];
+      e2m1x8_to_f32(w[i], t);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[8 * i + j] = t[j];
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float t[4];
+      e4m3x4_to_f32(w[i], t);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[4 * i + j] = t[j];
+    }
+  }
+}
+
+template <typename T, int MODE, int MM>
+__global__ void __launch_bounds__(kQmvThreads) k_qmv_mx(const T* __restrict__ x, const uint32_t* __restrict__ wc,
+                                                      const uint8_t* __restrict__ ws, int M_, int N, int K,
+                                                      T* __restrict__ y) {
+  extern __shared__ float4 xs4[];
+  const uint32_t M = (uint32_t)M_;
+  qmv_mx_prologue<T, MODE>(x, M, (uint32_t)K, xs4);
+  __syncthreads();
+  constexpr uint32_t kPerChunk = MODE == 2 ? 32u : 16u;  // codes per 128-bit chunk
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t chunks = (uint32_t)K / kPerChunk;
+  const uint32_t groups = (chunks + 32u * kQmvCH - 1) / (32u * kQmvCH);
+  const uint32_t nb = (uint32_t)K / 32u;  // scale bytes per row
+  const uint4* wc4 = reinterpret_cast<const uint4*>(wc);
+  const uint32_t first = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const uint32_t step = (gridDim.x * blockDim.x) >> 5;
+  uint32_t un = first, ug = 0;
+  uint4 qb[kQmvCH];
+  uint32_t sb[kQmvCH];
+  auto load_unit = [&](uint32_t n, uint32_t g) {
+#pragma unroll
+    for (int i = 0; i < kQmvCH; ++i) {
+      const uint32_t c = g * 32u * kQmvCH + (uint32_t)i * 32u + lane;
+      if (n < (uint32_t)N && c < chunks) {
+        qb[i] = __ldg(wc4 + (size_t)n * chunks + c);
+        sb[i] = __ldg(ws + (size_t)n * nb + (c * kPerChunk) / 32u);
+      } else {
+        qb[i] = make_uint4(0, 0, 0, 0);
+        sb[i] = 127;
+      }
+    }
+  };
+  load_unit(un, ug);
+  float acc[MM];
+#pragma unroll
+  for (int m = 0; m < MM; ++m) acc[m] = 0.0f;
+  while (un < (uint32_t)N) {
+    uint4 q[kQmvCH];
+    uint32_t s[kQmvCH];
+#pragma unroll
+    for (int i = 0; i < kQmvCH; ++i) {
+      q[i] = qb[i];
+      s[i] = sb[i];
+    }
+    const uint32_t cn = un, cg = ug;
+    if (++ug == groups) {
+      ug = 0;
+      un += step;
+    }
+    load_unit(un, ug);  // next unit's loads in flight while this one computes
+#pragma unroll
+    for (int i = 0; i < kQmvCH; ++i) {
+      const uint32_t c = cg * 32u * kQmvCH + (uint32_t)i * 32u + lane;
+      if (c < chunks) {
+        float v[32];
+        mx_chunk_values<MODE>(q[i], v);
+        const float sw = ue8m0_to_f32(s[i]);
+#pragma unroll
+        for (int m = 0; m < MM; ++m) {
+          if ((uint32_t)m < M) {
+            float bs = 0.0f;
+#pragma unroll
+            for (int j = 0; j < (int)kPerChunk; j += 4) {
+              const uint32_t k = c * kPerChunk + (uint32_t)j;
+              const float4 xv = xs4[xs_index(m, (uint32_t)K, k) >> 2];
+              bs = fmaf(xv.x, v[j], bs);
+              bs = fmaf(xv.y, v[j + 1], bs);
+              bs = fmaf(xv.z, v[j + 2], bs);
+              bs = fmaf(xv.w, v[j + 3], bs);
+            }
+            acc[m] = fmaf(bs, sw, acc[m]);
+          }
+        }
+      }
+    }
+    if (cg + 1 == groups) {  // row finished: reduce across the warp and store
+#pragma unroll
+      for (int m = 0; m < MM; ++m) {
+        if ((uint32_t)m < M) {
+          float a = acc[m];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+          if (lane == 0) y[(size_t)m * N + cn] = Elem<T>::from_f(a);
+        }
+        acc[m] = 0.0f;
+      }
+    }
+  }
+}
+
+}  // namespace nvfp4

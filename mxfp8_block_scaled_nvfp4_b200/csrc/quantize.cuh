@@ -178,16 +178,22 @@ __device__ __forceinline__ uint32_t e2m1_sr(float t, uint32_t r) {
 // ("mlx 0.30.7.2 -> 0.30.7.6" diff, page 7, fp_quantize_rowwise), zero
 // codes for a block whose scale decodes to 0.
 //
-// Work unit: 32 x kUnroll half-blocks of one tensor (one warp iteration).
-// Units of all tensors form one sequence; warp w takes units w, w + nwarps,
-// ...  The loads of a warp's next unit are issued before the current one is
-// computed (two units in flight per warp).  Scale bytes of 4 consecutive
-// blocks are packed into one 32-bit store where they are contiguous (LINEAR
+// A lane quantizes whole 16-element blocks (K % 16 == 0: a block never
+// leaves its row): one 32-byte load (bf16 / fp16; two for fp32, 256-bit
+// vector loads when every input is 32-byte aligned), the block maximum in
+// registers, one scale, two code words in one 8-byte store (a warp writes
+// 256 contiguous bytes).  Work unit: 32 x kBlkU consecutive blocks of one
+// tensor (one warp iteration); units of all tensors form one sequence, warp
+// w takes units w, w + nwarps, ..., and the loads of its next unit are in
+// flight while it computes the current one.  Scale bytes of 4 consecutive
+// blocks go out as one 32-bit store where they are contiguous (LINEAR
 // layout, or 4 blocks of one row starting at a multiple of 4 in the tile
-// layout); other scales are stored byte by byte.
+// layout); other scales are stored byte by byte.  E / f8(s) comes from a
+// per-CTA table of those IEEE quotients (0 <= s <= 0x7E).
 // ---------------------------------------------------------------------------
 constexpr int kMaxSegs = 4;
-constexpr uint32_t kUnitHalf = 32u * kUnroll;  // half-blocks per unit
+constexpr int kBlkU = 2;                          // blocks per lane per unit
+constexpr uint32_t kUnitBlk = 32u * kBlkU;        // blocks per unit
 
 struct QuantSeg {
   const void* x;
@@ -195,7 +201,7 @@ struct QuantSeg {
   uint32_t* codes;
   ScaleOut so;
   uint32_t rows;
-  uint32_t n_half;
+  uint32_t n_blk;       // 16-element blocks
   uint32_t first_unit;  // index of the segment's first unit in the launch's sequence
 };
 
@@ -206,17 +212,46 @@ struct QuantSegs {
   uint64_t seed;   // stochastic rounding only
 };
 
-// Raw 16-byte words of one half-block (two for fp32).
+// Raw bytes of one 16-element block: 32 (2-byte types) or 64 (fp32).
 template <typename T>
-struct Raw8 {
-  uint4 a, b;
+struct RawBlk {
+  uint4 w[sizeof(T) == 4 ? 4 : 2];
 };
 
+template <bool V8>
+__device__ __forceinline__ void ld32(const void* p, uint4& a, uint4& b) {
+  if constexpr (V8) {
+    asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p));
+  } else {
+    const uint4* q = static_cast<const uint4*>(p);
+    a = __ldg(q);
+    b = __ldg(q + 1);
+  }
+}
+
+template <typename T, bool V8>
+__device__ __forceinline__ void load_blk(const T* p, RawBlk<T>& r) {
+  ld32<V8>(p, r.w[0], r.w[1]);
+  if constexpr (sizeof(T) == 4) ld32<V8>(reinterpret_cast<const uint8_t*>(p) + 32, r.w[2], r.w[3]);
+}
+
 template <typename T>
-__device__ __forceinline__ void load_raw(const T* p, Raw8<T>& r) {
-  const uint4* q = reinterpret_cast<const uint4*>(p);
-  r.a = __ldg(q);
-  if constexpr (sizeof(T) == 4) r.b = __ldg(q + 1);
+__device__ __forceinline__ void unpack16(const RawBlk<T>& r, float (&v)[16]) {
+  float lo[8], hi[8];
+  if constexpr (sizeof(T) == 4) {
+    unpack8<T>(r.w[0], r.w[1], lo);
+    unpack8<T>(r.w[2], r.w[3], hi);
+  } else {
+    unpack8<T>(r.w[0], r.w[0], lo);
+    unpack8<T>(r.w[1], r.w[1], hi);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    v[j] = lo[j];
+    v[8 + j] = hi[j];
+  }
 }
 
 __device__ __forceinline__ uint32_t seg_of(const QuantSegs& q, uint32_t unit) {
@@ -227,31 +262,34 @@ __device__ __forceinline__ uint32_t seg_of(const QuantSegs& q, uint32_t unit) {
   return i;
 }
 
-template <typename T>
-__device__ __forceinline__ void load_unit(const QuantSegs& q, uint32_t unit, uint32_t lane, Raw8<T> (&r)[kUnroll]) {
+template <typename T, bool V8>
+__device__ __forceinline__ void load_unit(const QuantSegs& q, uint32_t unit, uint32_t lane, RawBlk<T> (&r)[kBlkU]) {
   if (unit >= q.units) return;
   const QuantSeg& sg = q.s[seg_of(q, unit)];
-  const uint32_t base = (unit - sg.first_unit) * kUnitHalf;
+  const uint32_t base = (unit - sg.first_unit) * kUnitBlk;
   const T* x = static_cast<const T*>(sg.x);
 #pragma unroll
-  for (int u = 0; u < kUnroll; ++u) {
-    const uint32_t hb = base + (uint32_t)u * 32u + lane;
-    if (hb < sg.n_half) load_raw<T>(x + (size_t)hb * 8, r[u]);
-    else r[u].a = r[u].b = make_uint4(0, 0, 0, 0);
+  for (int u = 0; u < kBlkU; ++u) {
+    const uint32_t b = base + (uint32_t)u * 32u + lane;
+    if (b < sg.n_blk) {
+      load_blk<T, V8>(x + (size_t)b * 16, r[u]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < (int)(sizeof(r[u].w) / 16); ++i) r[u].w[i] = make_uint4(0, 0, 0, 0);
+    }
   }
 }
 
-// Scale bytes s of the even lanes' blocks (block hb >> 1 of lane hb), 4
-// consecutive blocks per 32-bit store where possible.  All lanes call it.
-__device__ __forceinline__ void store_scales(const ScaleOut& so, uint32_t hb, uint32_t n_half, uint32_t s,
+// Scale byte s of this lane's block b, 4 consecutive blocks per 32-bit
+// store where possible.  All lanes call it.
+__device__ __forceinline__ void store_scales(const ScaleOut& so, uint32_t b, uint32_t n_blk, uint32_t s,
                                              uint32_t lane) {
-  const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 2);
-  const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 4);
-  const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 6);
-  // lane % 8 == 0 owns blocks b0 .. b0 + 3 (b0 a multiple of 4)
-  const uint32_t lead = hb & ~7u;
-  const uint32_t b0 = lead >> 1;
-  bool packed = lead + 8u <= n_half;  // all four blocks exist
+  const uint32_t s1 = __shfl_down_sync(0xffffffffu, s, 1);
+  const uint32_t s2 = __shfl_down_sync(0xffffffffu, s, 2);
+  const uint32_t s3 = __shfl_down_sync(0xffffffffu, s, 3);
+  // lane % 4 == 0 owns blocks b0 .. b0 + 3 (b0 a multiple of 4)
+  const uint32_t b0 = b & ~3u;
+  bool packed = b0 + 4u <= n_blk;  // all four blocks exist
   uint32_t off = b0;
   if (so.swizzled) {
     const uint32_t r = so.bpr.div(b0), c = b0 - r * so.blocks_per_row;
@@ -259,24 +297,29 @@ __device__ __forceinline__ void store_scales(const ScaleOut& so, uint32_t hb, ui
     off = swizzled_offset(r, c, so.Cp);
   }
   if (packed) {
-    if ((lane & 7u) == 0) *reinterpret_cast<uint32_t*>(so.p + off) = __byte_perm(s | (s1 << 8), s2 | (s3 << 8), 0x5410);
-  } else if ((lane & 1u) == 0 && hb < n_half) {
-    so.store(hb >> 1, s);
+    if ((lane & 3u) == 0) *reinterpret_cast<uint32_t*>(so.p + off) = __byte_perm(s | (s1 << 8), s2 | (s3 << 8), 0x5410);
+  } else if (b < n_blk) {
+    so.store(b, s);
   }
 }
 
-template <typename T, bool SR = false>
+// e2m1 codes of v[i] * k for 8 values, each product rounded to fp32.
+__device__ __forceinline__ uint32_t scaled_e2m1x8_at(const float (&v)[16], int o, float k) {
+  float h[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) h[j] = v[o + j];
+  return scaled_e2m1x8(h, k);
+}
+
+template <typename T, bool SR = false, bool V8 = false>
 __global__ void __launch_bounds__(kEwThreads) k_nvfp4_quantize(const __grid_constant__ QuantSegs q) {
-  // k = E / f8(s) for every scale byte s a block can get (0 <= s <= 0x7E:
-  // t >= 0 and the conversion saturates), per tensor: the IEEE quotient the
-  // method takes per block, computed once per CTA instead of once per block
   __shared__ float ktab[kMaxSegs][128];
   __shared__ float etab[kMaxSegs];
   const uint32_t lane = threadIdx.x & 31u;
   const uint32_t warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
-  Raw8<T> nxt[kUnroll];
-  load_unit<T>(q, warp, lane, nxt);  // the first unit's loads before the table
+  RawBlk<T> nxt[kBlkU];
+  load_unit<T, V8>(q, warp, lane, nxt);  // the first unit's loads before the table
   for (uint32_t i = threadIdx.x; i < q.count * 128u; i += blockDim.x) {
     const QuantSeg& sg = q.s[i >> 7];
     const float E = sg.g ? kGlobalEncode / __ldg(sg.g) : 1.0f;
@@ -286,63 +329,50 @@ __global__ void __launch_bounds__(kEwThreads) k_nvfp4_quantize(const __grid_cons
   }
   __syncthreads();
   for (uint32_t unit = warp; unit < q.units; unit += nwarps) {
-    Raw8<T> cur[kUnroll];
+    RawBlk<T> cur[kBlkU];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) cur[u] = nxt[u];
-    load_unit<T>(q, unit + nwarps, lane, nxt);  // next unit's loads in flight during this one
+    for (int u = 0; u < kBlkU; ++u) cur[u] = nxt[u];
+    load_unit<T, V8>(q, unit + nwarps, lane, nxt);  // next unit's loads in flight during this one
     const uint32_t si = seg_of(q, unit);
     const QuantSeg& sg = q.s[si];
-    const uint32_t base = (unit - sg.first_unit) * kUnitHalf;
+    const uint32_t base = (unit - sg.first_unit) * kUnitBlk;
     const float E = etab[si];
     const float* kt = ktab[si];
-    // stochastic rounding: half-blocks 2c and 2c + 1 share generator call c
-    // (words x, y for the even one, z, w for the odd one).  Over iterations
-    // (u, u + 1) the even lane of a pair calls the generator for u and the
-    // odd lane for u + 1; each hands its partner the two words it needs.
-    uint32_t wa[kUnroll], wb[kUnroll];
-    if constexpr (SR) {
 #pragma unroll
-      for (int u = 0; u < kUnroll; u += 2) {
-        const uint32_t odd = lane & 1u;
-        const uint64_t c0 = (uint64_t)(base + (uint32_t)(u + (int)odd) * 32u + (lane & ~1u)) >> 1;
-        const uint4 r4 = philox4x32_10(make_uint4((uint32_t)c0, (uint32_t)(c0 >> 32), 0u, 0u), (uint32_t)q.seed,
-                                       (uint32_t)(q.seed >> 32));
-        const uint32_t give0 = odd ? r4.x : r4.z, give1 = odd ? r4.y : r4.w;
-        const uint32_t got0 = __shfl_xor_sync(0xffffffffu, give0, 1);
-        const uint32_t got1 = __shfl_xor_sync(0xffffffffu, give1, 1);
-        // even lane: u from its own call (x, y), u + 1 from the partner's (x, y)
-        // odd lane:  u from the partner's call (z, w), u + 1 from its own (z, w)
-        wa[u] = odd ? got0 : r4.x;
-        wb[u] = odd ? got1 : r4.y;
-        wa[u + 1] = odd ? r4.z : got0;
-        wb[u + 1] = odd ? r4.w : got1;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const uint32_t hb = base + (uint32_t)u * 32u + lane;
-      float v[8];
-      unpack8<T>(cur[u].a, cur[u].b, v);
+    for (int u = 0; u < kBlkU; ++u) {
+      const uint32_t b = base + (uint32_t)u * 32u + lane;
+      float v[16];
+      unpack16<T>(cur[u], v);
       float a = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[j]));
-      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+      for (int j = 0; j < 16; ++j) a = fmaxf(a, fabsf(v[j]));
       float t = a / kE2M1Max;
       t = t * E;
       const uint32_t s = f32_to_e4m3(t);
-      uint32_t w = 0;
-      if (s != 0u) {  // f8(s) != 0
-        const float k = kt[s];
-        if constexpr (SR) {
+      uint2 w = make_uint2(0u, 0u);
+      if constexpr (SR) {
+        // the block's 16 random bytes: the four outputs of the generator at
+        // counter b (elements 4i..4i+3 from output i, byte j for element
+        // 4i+j); every lane calls it, outside the branches
+        const uint4 r4 = philox4x32_10(make_uint4(b, 0u, 0u, 0u), (uint32_t)q.seed, (uint32_t)(q.seed >> 32));
+        if (s != 0u) {
+          const float k = kt[s];
+          const uint32_t rw[4] = {r4.x, r4.y, r4.z, r4.w};
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            w |= e2m1_sr(v[j] * k, ((j < 4 ? wa[u] : wb[u]) >> (8 * (j & 3))) & 0xFFu) << (4 * j);
-        } else {
-          w = scaled_e2m1x8(v, k);
+          for (int j = 0; j < 8; ++j) {
+            w.x |= e2m1_sr(v[j] * k, (rw[j >> 2] >> (8 * (j & 3))) & 0xFFu) << (4 * j);
+            w.y |= e2m1_sr(v[8 + j] * k, (rw[2 + (j >> 2)] >> (8 * (j & 3))) & 0xFFu) << (4 * j);
+          }
+        }
+      } else {
+        if (s != 0u) {  // f8(s) != 0
+          const float k = kt[s];
+          w.x = scaled_e2m1x8_at(v, 0, k);
+          w.y = scaled_e2m1x8_at(v, 8, k);
         }
       }
-      if (hb < sg.n_half) sg.codes[hb] = w;
-      store_scales(sg.so, hb, sg.n_half, s, lane);
+      if (b < sg.n_blk) reinterpret_cast<uint2*>(sg.codes)[b] = w;
+      store_scales(sg.so, b, sg.n_blk, s, lane);
     }
   }
   for (uint32_t i = 0; i < q.count; ++i) zero_scale_padding(q.s[i].so, q.s[i].rows);
@@ -365,10 +395,13 @@ __global__ void __launch_bounds__(kEwThreads) k_nvfp4_quantize(const __grid_cons
 // ---------------------------------------------------------------------------
 constexpr int kColR = 128, kColC = 64, kColThreads = 256;
 
-template <typename T>
+// SR: stochastic rounding of the codes with the row-wise quantizer's bits,
+// taken over x^T: block (c, r / 16) of x^T [C, R] uses the four outputs of
+// the generator at counter c * (R / 16) + r / 16 (its flat block index).
+template <typename T, bool SR = false>
 __global__ void __launch_bounds__(kColThreads) k_nvfp4_quantize_columnwise(
     const T* __restrict__ x, uint32_t R, uint32_t C, const float* __restrict__ g, uint32_t* __restrict__ codes,
-    ScaleOut so) {
+    ScaleOut so, uint64_t seed = 0) {
   __shared__ float tile[kColC][kColR + 1];
   __shared__ uint2 qcodes[kColC][kColR / 16];
   const float E = g ? kGlobalEncode / __ldg(g) : 1.0f;
@@ -404,7 +437,20 @@ __global__ void __launch_bounds__(kColThreads) k_nvfp4_quantize_columnwise(
     const uint32_t s = f32_to_e4m3(t);
     const float fs = e4m3_to_f32(s);
     uint32_t w0 = 0, w1 = 0;
-    if (fs != 0.0f) {
+    const uint32_t c = c0 + cc, r = r0 + rb * 16;
+    if constexpr (SR) {
+      const uint4 r4 = philox4x32_10(make_uint4(c * (R / 16u) + r / 16u, 0u, 0u, 0u), (uint32_t)seed,
+                                     (uint32_t)(seed >> 32));
+      if (fs != 0.0f) {
+        const float k = E / fs;
+        const uint32_t rw[4] = {r4.x, r4.y, r4.z, r4.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          w0 |= e2m1_sr(v[j] * k, (rw[j >> 2] >> (8 * (j & 3))) & 0xFFu) << (4 * j);
+          w1 |= e2m1_sr(v[8 + j] * k, (rw[2 + (j >> 2)] >> (8 * (j & 3))) & 0xFFu) << (4 * j);
+        }
+      }
+    } else if (fs != 0.0f) {
       const float k = E / fs;
       float q0[8], q1[8];
 #pragma unroll
@@ -416,7 +462,6 @@ __global__ void __launch_bounds__(kColThreads) k_nvfp4_quantize_columnwise(
       w1 = f32x8_to_e2m1x8(q1);
     }
     qcodes[cc][rb] = make_uint2(w0, w1);
-    const uint32_t c = c0 + cc, r = r0 + rb * 16;
     if (c < C && r < R) so.store(c * (R / 16u) + r / 16u, s);
   }
   __syncthreads();

@@ -51,6 +51,7 @@ SIGNATURES = [
     ("nvfp4_quantize_columnwise", _I, [_P, _I, _I64, _I64, _P, _P, _P, _I, _P]),
     ("nvfp4_dequantize", _I, [_P, _P, _I, _I64, _I64, _P, _P, _I, _P]),
     ("nvfp4_quantize_sr", _I, [_P, _I, _I64, _I64, _P, ctypes.c_uint64, _P, _P, _I, _P]),
+    ("nvfp4_quantize_columnwise_sr", _I, [_P, _I, _I64, _I64, _P, ctypes.c_uint64, _P, _P, _I, _P]),
     ("mxfp8_quantize", _I, [_P, _I, _I64, _I64, _P, _P, _I, _P]),
     ("mxfp8_dequantize", _I, [_P, _P, _I, _I64, _I64, _P, _I, _P]),
     ("mxfp4_quantize", _I, [_P, _I, _I64, _I64, _P, _P, _I, _P]),
@@ -59,6 +60,7 @@ SIGNATURES = [
     ("qqmm", _I, [_I, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I, _P]),
     ("qmv", _I, [_P, _I, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     ("qmv_pdl", _I, [_P, _I, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    ("qmv_mx", _I, [_I, _P, _I, _P, _P, _I64, _I64, _I64, _P, _P]),
     ("gather_qmm", _I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     ("gather_qmm_kn", _I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     ("gather_qmm_workspace_size", _SZ, [_I64, _I64, _I64]),
@@ -239,9 +241,11 @@ def nvfp4_quantize_multi(jobs):
 
 
 def nvfp4_quantize_columnwise(x: torch.Tensor, g: torch.Tensor | None = None, layout: str = "linear",
-                              codes: torch.Tensor | None = None, scales: torch.Tensor | None = None):
+                              codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                              seed: int | None = None):
     """(codes [cols, rows/8], scales) of x^T quantized along the rows of a 2-D x
-    (equal to nvfp4_quantize(x.T.contiguous(), g, layout))."""
+    (equal to nvfp4_quantize(x.T.contiguous(), g, layout)); with a seed,
+    nvfp4_quantize_columnwise_sr (equal to nvfp4_quantize_sr of x^T)."""
     rows, cols = x.shape
     _need_g(g)
     _need_bytes(codes, cols * (rows // 8) * 4, "codes")
@@ -251,8 +255,12 @@ def nvfp4_quantize_columnwise(x: torch.Tensor, g: torch.Tensor | None = None, la
         codes = torch.empty(cols, rows // 8, dtype=torch.int32, device=x.device)
     if scales is None:
         scales = torch.empty(scale_shape(cols, rows // 16, layout), dtype=torch.uint8, device=x.device)
-    _check(lib().nvfp4_quantize_columnwise(_ptr(x), DT[x.dtype], rows, cols, _ptr(g), _ptr(codes), _ptr(scales),
-                                           LAYOUT[layout], _stream()))
+    if seed is None:
+        _check(lib().nvfp4_quantize_columnwise(_ptr(x), DT[x.dtype], rows, cols, _ptr(g), _ptr(codes), _ptr(scales),
+                                               LAYOUT[layout], _stream()))
+    else:
+        _check(lib().nvfp4_quantize_columnwise_sr(_ptr(x), DT[x.dtype], rows, cols, _ptr(g), seed, _ptr(codes),
+                                                  _ptr(scales), LAYOUT[layout], _stream()))
     return codes, scales
 
 
@@ -428,6 +436,25 @@ def qmv(x: torch.Tensor, w_codes, w_scales, g_x=None, g_w=None, out=None, pdl: b
     fn = lib().qmv_pdl if pdl else lib().qmv
     _check(fn(_ptr(x), DT[x.dtype], _ptr(g_x), _ptr(w_codes), _ptr(w_scales), _ptr(g_w), M, N, K, _ptr(out),
               _stream()))
+    return out
+
+
+def qmv_mx(x: torch.Tensor, w_codes, w_scales, mode: str, out=None) -> torch.Tensor:
+    """y [M, N] (x's dtype) = x_hat . w_hat^T in an MX mode ("mxfp8": codes
+    [N, K/4], "mxfp4": codes [N, K/8]; e8m0 scales LINEAR [N, K/32]), M <= 8."""
+    if mode not in ("mxfp8", "mxfp4"):
+        raise ValueError("qmv_mx: mode must be mxfp8 or mxfp4")
+    M, K = x.shape
+    N = w_codes.shape[0]
+    _need_bytes(w_codes, N * (K if mode == "mxfp8" else K // 2), "w_codes")
+    _need_bytes(w_scales, N * (K // 32), "w_scales")
+    _need_dtype(out, x.dtype, "out")
+    _need_bytes(out, M * N * x.element_size(), "out")
+    _need_cuda(x, w_codes, w_scales, out)
+    if out is None:
+        out = torch.empty(M, N, dtype=x.dtype, device=x.device)
+    _check(lib().qmv_mx(MODE[mode], _ptr(x), DT[x.dtype], _ptr(w_codes), _ptr(w_scales), M, N, K, _ptr(out),
+                        _stream()))
     return out
 
 

@@ -452,6 +452,26 @@ def qmv(x, x_dt, g_x, w_codes, w_scales, g_w):
     return {"y_ref": y_ref, "abs_ref": abs_ref, "y": round_to(y_ref, x_dt)}
 
 
+def qmv_mx(x, x_dt, w_codes, w_scales, mode):
+    """qmv in an MX mode ([P2] qqmm.cpp M=1 route: fp_quantize_dequantize of x
+    with the mode's group size 32 and bits, then fp_qmv; no global scales,
+    [P1] validate_global_scale).  x_hat = the mode's quantize then dequantize
+    of x, in x's type (materialized); w_hat = code * 2^(s-127) decoded
+    exactly.  float64 sum, one rounding to T."""
+    if mode == "mxfp8":
+        quant, deq, dec = mxfp8_quantize, mxfp8_dequantize, mxfp8_decode_exact
+    elif mode == "mxfp4":
+        quant, deq, dec = mxfp4_quantize, mxfp4_dequantize, mxfp4_decode_exact
+    else:
+        raise ValueError(mode)
+    xc, xs = quant(x, x_dt)
+    xh = to_f64(deq(xc, xs, x_dt), x_dt)
+    wh = dec(w_codes, w_scales)
+    y_ref = xh @ wh.T
+    abs_ref = np.abs(xh) @ np.abs(wh).T
+    return {"y_ref": y_ref, "abs_ref": abs_ref, "y": round_to(y_ref, x_dt)}
+
+
 # --------------------------------------------------------------------------
 # a10: gather_qmm (MoE) with per-expert global scales
 # --------------------------------------------------------------------------

@@ -123,6 +123,12 @@ def test_quantize_sr_checks(L):
     assert L.nvfp4_quantize_sr(A, 2, 4, 32, None, 7, A, A, 5, None) == 1  # layout
     assert L.nvfp4_quantize_sr(A + 8, 2, 4, 32, None, 7, A, A, 0, None) == 1
     assert "aligned" in msg(L)
+    # column-wise: the quantized dimension is the rows of x
+    assert L.nvfp4_quantize_columnwise_sr(A, 2, 24, 4, None, 7, A, A, 0, None) == 1
+    assert "group size 16" in msg(L)
+    assert L.nvfp4_quantize_columnwise_sr(A, 2, 32, 4, None, 7, A, A, 5, None) == 1  # layout
+    assert L.nvfp4_quantize_columnwise_sr(None, 2, 32, 0, None, 7, None, None, 1, None) == 0  # empty
+    assert L.nvfp4_quantize_columnwise_sr(A, 2, 32, 4, None, 7, A, A, 0, None) not in (0, 1, 2)  # needs a device
 
 
 def test_gather_kn_checks(L):
@@ -293,3 +299,15 @@ def test_multi_tensor_entries_check_every_item(L):
     assert am(AmaxItem(A, -1, A)) == 1
     assert am(AmaxItem(A, 16, A + 2)) == 1 and "4-byte aligned" in msg(L)
     assert am(AmaxItem(A, 16, A), AmaxItem(A, 0, A + 4)) not in (0, 1, 2)
+
+
+def test_qmv_mx_checks(L):
+    N0 = None
+    assert L.qmv_mx(0, A, 2, A, A, 1, 64, 256, A, N0) == 1 and "mxfp8 or mxfp4" in msg(L)  # nvfp4 mode
+    assert L.qmv_mx(1, A, 2, A, A, 9, 64, 256, A, N0) == 1 and "M must be" in msg(L)
+    assert L.qmv_mx(2, A, 2, A, A, 1, 64, 48, A, N0) == 1 and "K % 32" in msg(L)
+    assert L.qmv_mx(2, A, 7, A, A, 1, 64, 256, A, N0) == 2
+    assert L.qmv_mx(1, A + 8, 2, A, A, 1, 64, 256, A, N0) == 1 and "aligned" in msg(L)
+    assert L.qmv_mx(1, A, 2, A, A, 8, 64, 8192, A, N0) == 2 and "160 KiB" in msg(L)
+    assert L.qmv_mx(2, N0, 2, N0, N0, 1, 0, 256, N0, N0) == 0  # empty output
+    assert L.qmv_mx(2, A, 2, A, A, 1, 64, 256, A, N0) not in (0, 1, 2)  # needs a device

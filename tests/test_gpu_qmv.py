@@ -144,3 +144,23 @@ def test_qmv_pdl_chain_orders_reads_and_writes(nv):
     nv.check_device_errors()
     for u, v in zip(want, got):
         assert torch.equal(u.view(torch.int16), v.view(torch.int16))
+
+
+@pytest.mark.parametrize("mode", ["mxfp8", "mxfp4"])
+@pytest.mark.parametrize("dt", ["bf16", "f16", "f32"])
+@pytest.mark.parametrize("M,N,K", [(1, 200, 256), (2, 130, 1024), (3, 77, 96), (8, 257, 2048), (1, 4096, 4096)])
+def test_qmv_mx_parity(nv, orc, mode, dt, M, N, K):
+    """qmv in the MX modes against the oracle (x quantize-dequantized with
+    the mode's 32-blocks and e8m0 scales, the weight decoded exactly)."""
+    from mxfp8_block_scaled_nvfp4_b200 import workloads
+    x = workloads.normal((M, K), 1.0, 90 + M + K, TORCH_DT[dt])
+    w = workloads.normal((N, K), 0.02, 91 + N, TORCH_DT[dt])
+    quant = nv.mxfp8_quantize if mode == "mxfp8" else nv.mxfp4_quantize
+    oquant = orc.mxfp8_quantize if mode == "mxfp8" else orc.mxfp4_quantize
+    wc, ws = quant(w.cuda(), "linear")
+    y = nv.qmv_mx(x.cuda(), wc, ws, mode)
+    nv.check_device_errors()
+    owc, ows = oquant(raw(w), dt)
+    assert np.array_equal(raw(wc), owc) and np.array_equal(raw(ws), ows)
+    r = orc.qmv_mx(raw(x), dt, owc, ows, mode)
+    check_gemm_output(raw(y), r, dt, orc)

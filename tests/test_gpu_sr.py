@@ -96,3 +96,21 @@ def test_sr_full_size_sampled_rows(nv, orc):
                 want = orc.e2m1_sr(float(t), orc.sr_bits(99, r * 16384 + kk))
                 got = (int(codes_c[n, kk // 8]) >> (4 * (kk % 8))) & 15
                 assert got == want, (r, kk)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("shape", [(16, 1), (48, 3), (256, 67), (1040, 200), (4096, 130)])
+@pytest.mark.parametrize("layout", ["linear", "swizzled"])
+def test_sr_columnwise_parity(nv, orc, dt, shape, layout):
+    """Column-wise stochastic rounding equals the oracle's stochastic
+    rounding of the transposed, contiguous matrix with the same seed."""
+    x = make_x(shape, dt, 900 + shape[0] + shape[1], std=0.02)
+    xg = x.cuda()
+    g = nv.amax(xg)
+    seed = 0xDEAD_BEEF_0000 + shape[1]
+    codes, scales = nv.nvfp4_quantize_columnwise(xg, g, layout, seed=seed)
+    nv.check_device_errors()
+    oc, os_ = orc.nvfp4_quantize_sr(raw(x.t().contiguous()), dt, g.item(), seed=seed)
+    assert np.array_equal(raw(codes), oc)
+    want_s = os_ if layout == "linear" else orc.swizzle_scales(os_)
+    assert np.array_equal(raw(scales), want_s)
