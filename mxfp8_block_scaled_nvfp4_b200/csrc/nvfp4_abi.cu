@@ -537,7 +537,8 @@ static nvfp4_status qmv_launch(const void* x, nvfp4_dtype x_dt, const float* g_x
     CUtensorMap mw;
     if (!qtc::make_map(&mw, w_codes, (uint64_t)N, (uint64_t)K))
       return fail(NVFP4_ERR_CUDA, "[qmv] cuTensorMapEncodeTiled failed");
-    qtc::Args a{x, g_x, w_codes, w_scales, g_w, y, (uint32_t)M, (uint32_t)N, (uint32_t)K, stages};
+    const qtc::Groups gr = qtc::pick_groups(stages, (uint32_t)(K / 256));
+    qtc::Args a{x, g_x, w_codes, w_scales, g_w, y, (uint32_t)M, (uint32_t)N, (uint32_t)K, stages, gr.g0, gr.g};
     const uint32_t MM = M == 1 ? 1u : 2u;
     const size_t smem = qtc::smem_needed(stages, MM, (uint32_t)K, esz);
     const unsigned grid = (unsigned)((N + qtc::BM - 1) / qtc::BM);

@@ -32,8 +32,10 @@
 // memory, one ring half ahead).  Warp 0 first copies x into shared memory
 // (one bulk copy, ahead of the weight in the memory queues) and then starts
 // the weight stream; warps 1-11 compute the x_hat planes from that copy.
-// TMEM: a 256-column ring of MMA outputs drained in 128-column halves and
-// one tile of unit scales used by both operands.
+// TMEM: a ring of NSEG 128-column segments of MMA outputs, each drained by
+// the epilogue as a whole, and one tile of unit scales used by both
+// operands.  With three segments a segment is reused only after the
+// epilogue has long drained it, so the MMA chain rarely waits on it.
 //
 // Every mbarrier wait of the MMA thread costs about as much as several of
 // these small MMAs (its shared-memory access queues behind the tensor
@@ -41,7 +43,10 @@
 // the stages of a group complete on one barrier (the producer posts each
 // stage's bytes on it; two such barriers alternate, and the ring holds two
 // groups, so a group barrier is not reused before the MMA warp has passed
-// its previous phase); ring halves that were never used are not waited on.
+// its previous phase); segments that were never used are not waited on.
+// The first group is small, so the MMAs start as soon as the x planes are
+// ready; a stage's slot is released (commit) only when a later stage will
+// reuse it.
 #pragma once
 
 #include <cuda.h>
@@ -59,8 +64,8 @@ constexpr int MAX_STAGES = 12;
 constexpr int A_STAGE = BM * 128;  // 16 KiB of codes (256 K)
 constexpr int STAGE_BYTES = A_STAGE;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t D_RING = 256;     // MMA output columns [0, 256)
-constexpr uint32_t T_ONES = 256;     // unit block scales (both operands)
+constexpr uint32_t NSEG = 3;         // 128-column segments of MMA outputs: columns [0, 384)
+constexpr uint32_t T_ONES = 384;     // unit block scales (both operands)
 
 // shared memory carve-up (bytes, from a 1024-aligned base)
 struct Layout {
@@ -85,6 +90,38 @@ __host__ __device__ inline uint32_t smem_needed(uint32_t stages, uint32_t M, uin
   return L.total + 1024u;
 }
 
+// Stage groups: group 0 holds the first g0 stages, every later group g
+// stages; all stages of a group complete on one barrier.
+constexpr uint32_t NGRP = 4;  // group barriers, used round robin
+struct Groups {
+  uint32_t g0, g;
+  __host__ __device__ uint32_t start(uint32_t grp) const { return grp == 0 ? 0u : g0 + (grp - 1u) * g; }
+  __host__ __device__ uint32_t of(uint32_t kb) const { return kb < g0 ? 0u : 1u + (kb - g0) / g; }
+  __host__ __device__ uint32_t count(uint32_t kb_count) const {
+    return kb_count <= g0 ? 1u : 1u + (kb_count - g0 + g - 1u) / g;
+  }
+};
+
+// Group sizes for a ring of S slots and kb_count stages: a small first
+// group (the MMAs start early) where the ring allows it.  No group may hold
+// more than S stages (its stages are all in the ring before the MMA warp
+// consumes any of them).  A group barrier is rearmed by the producer for
+// group grp + NGRP only after the slot of a stage that group reuses was
+// released, i.e. after the MMA warp consumed stage kb - S, which must lie
+// in group grp or later, so that the MMA warp has already waited on group
+// grp's phase.
+inline Groups pick_groups(uint32_t S, uint32_t kb_count) {
+  const uint32_t cand[3][2] = {{2u, 4u}, {2u, S / 2u}, {S / 2u, S / 2u}};
+  for (auto& c : cand) {
+    Groups gr{c[0], c[1]};
+    if (gr.g == 0 || gr.g0 == 0 || gr.g > S || gr.g0 > S) continue;
+    bool ok = true;
+    for (uint32_t kb = S; kb < kb_count && ok; ++kb) ok = gr.of(kb - S) + NGRP > gr.of(kb);
+    if (ok) return gr;
+  }
+  return Groups{S / 2u, S / 2u};
+}
+
 struct Args {
   const void* x;
   const float* g_x;
@@ -93,6 +130,7 @@ struct Args {
   const float* g_w;
   void* y;
   uint32_t M, N, K, stages;
+  uint32_t g0, g;  // stage groups (pick_groups)
 };
 
 // K-major operand without swizzle: 8-row x 16-byte core matrices, `lbo`
@@ -116,56 +154,73 @@ template <> struct Range<__nv_bfloat16> {
 
 // x_hat = quantize-dequantize(x, g_x) of all M rows as plane codes and
 // plane scales (layout in the header comment), from x staged in shared
-// memory.  One lane per half-block; threads 32.. (warps 1 and up) take
-// part, warp 0 streams the weight.  Returns false on a thread that met a
-// block outside the exact range.
+// memory.  One thread per 16-element block; threads 32.. (warps 1 and up)
+// take part, warp 0 streams the weight.  Returns false on a thread that met
+// a block outside the exact range.
 template <typename T>
 __device__ __forceinline__ bool x_planes(const T* xs, float gx, uint32_t M, uint32_t K, uint8_t* planes,
                                          float* uplane) {
   const float E = kGlobalEncode / gx;
   const float d = gx / kGlobalEncode;
-  const uint32_t n_half = M * K / 8u;  // a multiple of 32: whole warps take part in the pair shuffle
+  const uint32_t n_blk = M * K / 16u;
   const uint32_t nb = K / 16u;
   bool exact = true;
-  const uint32_t nthr = blockDim.x - 32u;  // warps 1 and up (a multiple of 32)
-  for (uint32_t hb = threadIdx.x - 32u; threadIdx.x >= 32u && hb < n_half; hb += nthr) {
-    float v[8];
-    load8_shared<T>(xs + (size_t)hb * 8, v);
+  const uint32_t nthr = blockDim.x - 32u;  // warps 1 and up
+  for (uint32_t blk = threadIdx.x - 32u; threadIdx.x >= 32u && blk < n_blk; blk += nthr) {
+    float v[16];
+    {
+      float lo[8], hi[8];
+      load8_shared<T>(xs + (size_t)blk * 16, lo);
+      load8_shared<T>(xs + (size_t)blk * 16 + 8, hi);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        v[j] = lo[j];
+        v[8 + j] = hi[j];
+      }
+    }
     float a = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) a = fmaxf(a, fabsf(v[j]));
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    for (int j = 0; j < 16; ++j) a = fmaxf(a, fabsf(v[j]));
     const float t = (a / kE2M1Max) * E;
     const float fs = e4m3_to_f32(f32_to_e4m3(t));
     const float sd = fs * d;
-    uint32_t w = 0;
+    uint32_t w[2] = {0u, 0u};
     if (fs != 0.0f) {
       const float k = E / fs;
-      float q[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) q[j] = v[j] * k;
-      w = f32x8_to_e2m1x8(q);
+      for (int hf = 0; hf < 2; ++hf) {
+        float q[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) q[j] = v[8 * hf + j] * k;
+        w[hf] = f32x8_to_e2m1x8(q);
+      }
     }
     const float asd = fabsf(sd);
     exact = exact && (sd == 0.0f || (0.5f * asd >= Range<T>::kMinNormal && 6.0f * asd <= Range<T>::kMaxFinite));
     // codes of magnitude 1.5, 3, 6 (odd magnitude code >= 3) go to plane B
     // as 1, 2, 4 (the code minus one); all others stay in plane A
-    const uint32_t odd3 = w & 0x11111111u & ((w >> 1) | (w >> 2));
-    const uint32_t mask = odd3 * 15u;
-    const uint32_t pa = w & ~mask, pbw = (w - odd3) & mask;
-    // plane tile of k-step g = k0/64, block bl = (k0/16)%4, half hf of the block
-    const uint32_t m = (hb * 8u) / K, k0 = hb * 8u - m * K;
-    const uint32_t g = k0 >> 6, bl = (k0 >> 4) & 3u, hf = (k0 >> 3) & 1u;
-    uint8_t* tile = planes + (size_t)g * 256u * M;  // [h][row group][8 rows][16 B], rows = m*8 + bl*2 + p
-    const uint32_t h = bl >> 1, byte = 8u * (bl & 1u) + 4u * hf;
-    const uint32_t rowA = m * 8u + bl * 2u, rowB = rowA + 1u;
-    *reinterpret_cast<uint32_t*>(tile + h * 128u * M + (rowA >> 3) * 128u + (rowA & 7u) * 16u + byte) = pa;
-    *reinterpret_cast<uint32_t*>(tile + h * 128u * M + (rowB >> 3) * 128u + (rowB & 7u) * 16u + byte) = pbw;
-    if (hf == 0) {
-      const uint32_t b = k0 >> 4;
-      uplane[m * 2u * nb + 2u * b] = Elem<T>::to_f(Elem<T>::from_f(sd));
-      uplane[m * 2u * nb + 2u * b + 1u] = Elem<T>::to_f(Elem<T>::from_f(1.5f * sd));
+    uint32_t pa[2], pbw[2];
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const uint32_t odd3 = w[hf] & 0x11111111u & ((w[hf] >> 1) | (w[hf] >> 2));
+      const uint32_t mask = odd3 * 15u;
+      pa[hf] = w[hf] & ~mask;
+      pbw[hf] = (w[hf] - odd3) & mask;
     }
+    // plane tile of k-step g = k0/64, block bl = (k0/16)%4; the block's two
+    // code words are 8 contiguous bytes of its plane row
+    const uint32_t m = (blk * 16u) / K, k0 = blk * 16u - m * K;
+    const uint32_t g = k0 >> 6, bl = (k0 >> 4) & 3u;
+    uint8_t* tile = planes + (size_t)g * 256u * M;  // [h][row group][8 rows][16 B], rows = m*8 + bl*2 + p
+    const uint32_t h = bl >> 1, byte = 8u * (bl & 1u);
+    const uint32_t rowA = m * 8u + bl * 2u, rowB = rowA + 1u;
+    *reinterpret_cast<uint2*>(tile + h * 128u * M + (rowA >> 3) * 128u + (rowA & 7u) * 16u + byte) =
+        make_uint2(pa[0], pa[1]);
+    *reinterpret_cast<uint2*>(tile + h * 128u * M + (rowB >> 3) * 128u + (rowB & 7u) * 16u + byte) =
+        make_uint2(pbw[0], pbw[1]);
+    const uint32_t b = k0 >> 4;
+    uplane[m * 2u * nb + 2u * b] = Elem<T>::to_f(Elem<T>::from_f(sd));
+    uplane[m * 2u * nb + 2u * b + 1u] = Elem<T>::to_f(Elem<T>::from_f(1.5f * sd));
   }
   return exact;
 }
@@ -181,10 +236,10 @@ template <typename T, int MM, bool PDL = false>
 __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ CUtensorMap tmap_w, Args a) {
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t gfull[2];  // all stages of a group landed
+  __shared__ __align__(8) uint64_t gfull[NGRP];  // all stages of a group landed
   __shared__ __align__(8) uint64_t empty_bar[MAX_STAGES];
-  __shared__ __align__(8) uint64_t dfull_bar[2];
-  __shared__ __align__(8) uint64_t dempty_bar[2];
+  __shared__ __align__(8) uint64_t dfull_bar[NSEG];
+  __shared__ __align__(8) uint64_t dempty_bar[NSEG];
   __shared__ __align__(8) uint64_t xbar;  // x landed in shared memory
   __shared__ uint32_t tmem_holder;
   __shared__ int abort_flag;
@@ -204,37 +259,35 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
   const uint32_t ncols = 8u * MM;         // MMA N
   const uint32_t steps_per_half = 128u / ncols;
   const uint32_t nb = a.K / 16u;
-  const uint32_t G = S / 2;               // stages per group (S is even)
-  const uint32_t groups = (kb_count + G - 1) / G;
+  const Groups GR{a.g0, a.g};
+  const uint32_t groups = GR.count(kb_count);
 
   // stage kb into ring slot kb % S; its bytes complete on its group's
-  // barrier, and the last stage of a short final group also arrives for the
-  // stages that group lacks
+  // barrier (group grp on gfull[grp % NGRP], phase (grp / NGRP) & 1); the
+  // group's last stage (or the last stage of all) also arrives
   auto issue = [&](uint32_t kb) {
-    const uint32_t grp = kb / G, bar = smem_u32(&gfull[grp & 1u]);
-    mbar_expect_tx(bar, A_STAGE);
+    const uint32_t grp = GR.of(kb), bar = smem_u32(&gfull[grp % NGRP]);
+    if (kb + 1 == GR.start(grp + 1) || kb + 1 == kb_count) mbar_expect_tx(bar, A_STAGE);
+    else asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(A_STAGE) : "memory");
     tma_load_2d(sbase + L.ring + (kb % S) * STAGE_BYTES, &tmap_w, (int)(kb * 128u), (int)row0, bar);
-    if (kb + 1 == kb_count) {
-      const uint32_t missing = G - (kb_count - grp * G);
-      if (missing)
-        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(missing) : "memory");
-    }
   };
-  // the latest phases of both group barriers (all copies still in flight
-  // belong to the last two groups issued)
+  // the latest phases of the group barriers (all copies still in flight
+  // belong to the last NGRP groups issued); after an abort the last group
+  // may lack its arriving stage, so the producer arrives for it first
   auto drain = [&](uint32_t issued) {
     if (issued == 0) return;
-    const uint32_t last = (issued - 1) / G;
-    for (uint32_t gr = last > 0 ? last - 1 : 0; gr <= last; ++gr)
-      mbar_wait(smem_u32(&gfull[gr & 1u]), (gr >> 1) & 1u);
+    const uint32_t last = GR.of(issued - 1);
+    if (issued != kb_count && GR.start(last + 1) != issued)
+      asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&gfull[last % NGRP])) : "memory");
+    for (uint32_t gr = last + 1 > NGRP ? last + 1 - NGRP : 0; gr <= last; ++gr)
+      mbar_wait(smem_u32(&gfull[gr % NGRP]), (gr / NGRP) & 1u);
   };
 
   uint32_t issued = 0;  // weight stages issued (thread 0)
   if (threadIdx.x == 0) {
     for (uint32_t s = 0; s < S; ++s) mbar_init(smem_u32(&empty_bar[s]), 1);
-    mbar_init(smem_u32(&gfull[0]), G);
-    mbar_init(smem_u32(&gfull[1]), G);
-    for (int h = 0; h < 2; ++h) {
+    for (uint32_t i = 0; i < NGRP; ++i) mbar_init(smem_u32(&gfull[i]), 1);
+    for (uint32_t h = 0; h < NSEG; ++h) {
       mbar_init(smem_u32(&dfull_bar[h]), 1);
       mbar_init(smem_u32(&dempty_bar[h]), 4);
     }
@@ -337,18 +390,19 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
     uint32_t g = 0;  // global k-step
     bool ok = true;
     for (uint32_t grp = 0; grp < groups && ok; ++grp) {
-      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&gfull[grp & 1u]), (grp >> 1) & 1u)) ||
+      if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&gfull[grp % NGRP]), (grp / NGRP) & 1u)) ||
           *(volatile int*)&abort_flag) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t kb1 = min((grp + 1) * G, kb_count);
-      for (uint32_t kb = grp * G; kb < kb1; ++kb) {
+      const uint32_t kb1 = min(GR.start(grp + 1), kb_count);
+      for (uint32_t kb = GR.start(grp); kb < kb1; ++kb) {
         const uint32_t s = kb % S;
-        const uint32_t hf = (g / steps_per_half) & 1u;  // ring half of this stage
-        const uint32_t use = g / (2u * steps_per_half);   // times this half was used before
-        if (g % steps_per_half == 0 && use > 0) {         // reuse: wait until the half is drained
+        const uint32_t seg = g / steps_per_half;          // segment use number
+        const uint32_t hf = seg % NSEG;                   // ring segment of this stage
+        const uint32_t use = seg / NSEG;                  // times this segment was used before
+        if (g % steps_per_half == 0 && use > 0) {         // reuse: wait until the segment is drained
           if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&dempty_bar[hf]), (use & 1u) ^ 1u))) {
             ok = false;
             break;
@@ -356,7 +410,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
           tc_fence_after();
         }
         if (leader) {
-          const uint32_t dcol = (g % (2u * steps_per_half)) * ncols;
+          const uint32_t dcol = hf * 128u + (g % steps_per_half) * ncols;
 #pragma unroll
           for (uint32_t j = 0; j < 4; ++j)
             mma_block_scaled<kNV>(tmem + dcol + j * ncols,
@@ -364,7 +418,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
                                     mk((uint32_t)b_base + (((g + j) * 256u * MM) >> 4), b_hi), idesc, tmem + T_ONES,
                                     tmem + T_ONES, 0u);
           if ((g + 4) % steps_per_half == 0 || g + 4 == ksteps) mma_commit(smem_u32(&dfull_bar[hf]));
-          mma_commit(smem_u32(&empty_bar[s]));
+          if (kb + S < kb_count) mma_commit(smem_u32(&empty_bar[s]));  // the slot is refilled later
         }
         __syncwarp();
         g += 4;
@@ -396,12 +450,13 @@ __global__ void __launch_bounds__(THREADS, 1) k_qmv_tc(const __grid_constant__ C
     load_scales(0, sc);
     bool ok = true;
     for (uint32_t h = 0; h < halves; ++h) {
-      const uint32_t hf = h & 1u;
+      const uint32_t hf = h % NSEG;
       uint4 cur[SPH / 4];
 #pragma unroll
       for (int j = 0; j < SPH / 4; ++j) cur[j] = sc[j];
       if (h + 1 < halves) load_scales(h + 1, sc);  // next half's scales in flight
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&dfull_bar[hf]), (h >> 1) & 1u)) && !*(volatile int*)&abort_flag;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&dfull_bar[hf]), (h / NSEG) & 1u)) &&
+           !*(volatile int*)&abort_flag;
       tc_fence_after();
       if (!ok) break;
       const uint32_t g0 = h * steps_per_half;
