@@ -64,7 +64,6 @@ L2_FLUSH_BYTES = 256 << 20
 # dominant kernel, from one ncu capture of that kernel as it is now (the
 # summaries under profiles/ give the commands and the other counters).
 NCU_TRAFFIC_BYTES = {
-    "gather_qmm": 126970112 + 56426240,         # profiles/gather_qmm_moe_T4096_top8_E64_N1408_K2048.md
     "gather_qmm (kn)": 127318528 + 56494080,    # profiles/gather_qmm_kn_moe_T4096_top8_E64_N1408_K2048.md
     "k_nvfp4_quantize<SR>": 1120127232 + 319645184,  # profiles/quantize_sr_32768x16384.md
 }
@@ -481,9 +480,11 @@ class PrefillBwd(Row):
 
 
 class Moe(Row):
-    name, launches = "moe", 2  # k_route + k_gather_mma
+    """The MoE config through gather_qmm with a staged workspace: routing,
+    the staged copy of the routed x rows, the SM-pair tensor-core kernel."""
+    name, launches = "moe", 3  # k_route + k_stage_x + k_gather_mma_ts
     b2b_label = "gather_qmm"
-    b2b_kernels = 2  # routing + the tensor-core kernel
+    b2b_kernels = 3
     b2b_transpose = True
 
     def b2b(self):  # two copies of the 108 MB expert weights, alternating
@@ -506,7 +507,8 @@ class Moe(Row):
         del w, wc, ws
         T, topk = self.idx.shape
         self.T, self.topk = T, topk
-        self.ws_buf = torch.empty(self.nv.gather_qmm_workspace_size(T, topk, E), dtype=torch.uint8, device=self.dev)
+        self.ws_buf = torch.empty(self.nv.gather_qmm_staged_workspace_size(T, topk, E, K), dtype=torch.uint8,
+                                  device=self.dev)
         self.y = torch.empty(T, topk, N, dtype=torch.bfloat16, device=self.dev)
         self.flop = 2 * T * topk * N * K
         self.bytes = self.wc.numel() * 4 + self.ws.numel() + self.x.numel() * 2 + self.y.numel() * 2 + self.idx.numel() * 4
@@ -530,7 +532,8 @@ class MoeKN(Moe):
     """The MoE config with the expert weights stored [E, K, N] and quantized
     along N (gather_qmm with transpose=False): same tokens, routing and
     per-expert global scales as the moe row."""
-    name, launches = "moe_kn", 2
+    name, launches = "moe_kn", 2  # k_route + k_gather_mma<true>
+    b2b_kernels = 2
     b2b_transpose = False
 
     def setup(self):

@@ -316,8 +316,13 @@ NVFP4_API nvfp4_status qmv_pdl(const void* x, nvfp4_dtype x_dt, const float* g_x
  * y [T, topk, N] bf16.  K % 64 == 0, N % 16 == 0; T*topk, N and K at most
  * 2^30; 1 <= E <= 1024 and E*N < 2^31 (E*K for gather_qmm_kn), the
  * weight rows a 32-bit TMA coordinate reaches (beyond: NVFP4_ERR_UNSUPPORTED).
- * workspace: device scratch of gather_qmm_workspace_size(T, topk, E) bytes,
- * 16-byte aligned, contents undefined on entry and exit. */
+ * workspace: device scratch of at least gather_qmm_workspace_size(T, topk, E)
+ * bytes, 16-byte aligned, contents undefined on entry and exit.  With at
+ * least gather_qmm_staged_workspace_size(T, topk, E, K) bytes, calls with
+ * T > 16 first copy the routed x rows, grouped by expert, into the
+ * workspace and run the SM-pair tensor-core kernel on that copy; with less
+ * they run the single-SM kernel that gathers x rows itself.  Both compute
+ * the same result (the fp32 sums may differ in rounding order only). */
 NVFP4_API nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const uint8_t* w_scales,
                         const float* g, const int32_t* idx, int64_t T, int64_t topk,
                         int64_t E, int64_t N, int64_t K, void* y, void* workspace,
@@ -339,6 +344,12 @@ NVFP4_API nvfp4_status gather_qmm_kn(const void* x, const uint32_t* w_codes, con
  * 0 for a triple they reject (T < 0, topk < 1, E outside [1, 1024],
  * T*topk > 2^30).  Host only. */
 NVFP4_API size_t gather_qmm_workspace_size(int64_t T, int64_t topk, int64_t E);
+
+/* Bytes of workspace with which gather_qmm stages the routed x rows (see
+ * gather_qmm): gather_qmm_workspace_size(T, topk, E) rounded up to 256,
+ * plus T*topk*K*2 bytes for the bf16 copy.  0 for arguments gather_qmm
+ * rejects (as above, and K outside [0, 2^30]).  Host only. */
+NVFP4_API size_t gather_qmm_staged_workspace_size(int64_t T, int64_t topk, int64_t E, int64_t K);
 
 /* gather_qmm without a workspace argument; the pages have no counterpart of
  * this entry point.  It is for callers that cannot allocate device memory

@@ -652,6 +652,14 @@ size_t gather_qmm_workspace_size(int64_t T, int64_t topk, int64_t E) {
   return gather_workspace_bytes(T, topk, E);
 }
 
+size_t gather_qmm_staged_workspace_size(int64_t T, int64_t topk, int64_t E, int64_t K) {
+  if (T < 0 || topk < 1 || E < 1 || E > gq::MAX_E || K < 0 || K > (1 << 30) || product_exceeds(T, topk, 1 << 30))
+    return 0;
+  const int64_t P = T * topk;
+  if (K > 0 && P > (int64_t)(SIZE_MAX / 4) / K) return 0;
+  return gather_staged_workspace_bytes(T, topk, E, K);
+}
+
 // Host checks shared by the gather entries: shapes (K % 64, N % n_mult, K > 0
 // when there is output), pointers and, where the caller passes one
 // (check_ws), the workspace size.
@@ -695,8 +703,8 @@ nvfp4_status gather_qmm(const void* x, const uint32_t* w_codes, const uint8_t* w
   DeviceInfo d;
   st = device_info("gather_qmm", &d);
   if (st != NVFP4_OK) return st;
-  return gather_qmm_launch(x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, workspace, d.sm_count, stream, t_msg,
-                           sizeof(t_msg));
+  return gather_qmm_launch(x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, workspace, workspace_bytes, d.sm_count,
+                           stream, t_msg, sizeof(t_msg));
 }
 
 nvfp4_status gather_qmm_kn(const void* x, const uint32_t* w_codes, const uint8_t* w_scales, const float* g,
@@ -709,8 +717,8 @@ nvfp4_status gather_qmm_kn(const void* x, const uint32_t* w_codes, const uint8_t
   DeviceInfo d;
   st = device_info("gather_qmm_kn", &d);
   if (st != NVFP4_OK) return st;
-  return gather_qmm_launch(x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, workspace, d.sm_count, stream, t_msg,
-                           sizeof(t_msg), true);
+  return gather_qmm_launch(x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, workspace, workspace_bytes, d.sm_count,
+                           stream, t_msg, sizeof(t_msg), true);
 }
 
 // Identity of the calling thread's current context (0 if none can be read):
@@ -785,8 +793,8 @@ nvfp4_status gather_qmm_noalloc(const void* x, const uint32_t* w_codes, const ui
   st = noalloc_scratch(&scratch);
   if (st != NVFP4_OK) return st;
   // The routing kernel rewrites every scratch entry the grouped kernel reads
-  // (tile count, tile list, permutation), so nothing needs clearing between
-  // calls.
+  // (tile count, tile list, permutation; the staging kernel the staged rows
+  // of every routed pair), so nothing needs clearing between calls.
   return gather_qmm(x, w_codes, w_scales, g, idx, T, topk, E, N, K, y, scratch, kNoAllocScratchBytes, stream);
 }
 

@@ -45,22 +45,34 @@ __global__ void __launch_bounds__(kEwThreads) k_amax(const __grid_constant__ Ama
     const int64_t n = a.n[sgi];
     const int64_t nvec = n / 8;
     float m = 0.0f;
-    for (int64_t i = tid; i < nvec; i += 4 * nthr) {
-      float v[4][8];
+    // raw 16-byte words of 4 vectors, the next 4 in flight while these are
+    // reduced (zero words past the end reduce to 0)
+    constexpr int W = sizeof(T) == 4 ? 2 : 1;
+    uint4 nxt[4][W];
+    auto load4 = [&](int64_t i0) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const int64_t j = i + k * nthr;
-        if (j < nvec) {
-          load8<T>(x + j * 8, v[k]);
-        } else {
+        const int64_t j = i0 + k * nthr;
+        const uint4* q = reinterpret_cast<const uint4*>(x + j * 8);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) v[k][e] = 0.0f;
-        }
+        for (int w = 0; w < W; ++w) nxt[k][w] = j < nvec ? __ldg(q + w) : make_uint4(0, 0, 0, 0);
       }
+    };
+    load4(tid);
+    for (int64_t i = tid; i < nvec; i += 4 * nthr) {
+      uint4 cur[4][W];
 #pragma unroll
       for (int k = 0; k < 4; ++k)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[k][e]));
+        for (int w = 0; w < W; ++w) cur[k][w] = nxt[k][w];
+      load4(i + 4 * nthr);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float v[8];
+        unpack8<T>(cur[k][0], cur[k][W - 1], v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+      }
     }
     for (int64_t i = nvec * 8 + tid; i < n; i += nthr) m = fmaxf(m, fabsf(Elem<T>::to_f(x[i])));
 #pragma unroll

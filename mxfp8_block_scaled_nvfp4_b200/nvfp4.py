@@ -64,6 +64,7 @@ SIGNATURES = [
     ("gather_qmm", _I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     ("gather_qmm_kn", _I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     ("gather_qmm_workspace_size", _SZ, [_I64, _I64, _I64]),
+    ("gather_qmm_staged_workspace_size", _SZ, [_I64, _I64, _I64, _I64]),
     ("gather_qmm_noalloc", _I, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P]),
 ]
 
@@ -462,6 +463,10 @@ def gather_qmm_workspace_size(T: int, topk: int, E: int) -> int:
     return int(lib().gather_qmm_workspace_size(T, topk, E))
 
 
+def gather_qmm_staged_workspace_size(T: int, topk: int, E: int, K: int) -> int:
+    return int(lib().gather_qmm_staged_workspace_size(T, topk, E, K))
+
+
 def _need_gather(x, w_codes, w_scales, g, idx, out, T, topk, E, N, K, transpose):
     """Types and sizes the gather entries read and write through raw pointers."""
     _need_dtype(x, torch.bfloat16, "x")
@@ -488,8 +493,9 @@ def gather_qmm(x, w_codes, w_scales, g, idx, workspace=None, out=None, transpose
     N = w_codes.shape[1] if transpose else w_codes.shape[2] * 8
     _need_gather(x, w_codes, w_scales, g, idx, out, T, topk, E, N, K, transpose)
     _need_cuda(x, w_codes, w_scales, g, idx, workspace, out)
-    if workspace is None:
-        workspace = torch.empty(gather_qmm_workspace_size(T, topk, E), dtype=torch.uint8, device=x.device)
+    if workspace is None:  # the staged form where it applies (weights [E, N, K])
+        size = gather_qmm_staged_workspace_size(T, topk, E, K) if transpose else gather_qmm_workspace_size(T, topk, E)
+        workspace = torch.empty(size, dtype=torch.uint8, device=x.device)
     if out is None:
         out = torch.empty(T, topk, N, dtype=torch.bfloat16, device=x.device)
     fn = lib().gather_qmm if transpose else lib().gather_qmm_kn

@@ -311,3 +311,15 @@ def test_qmv_mx_checks(L):
     assert L.qmv_mx(1, A, 2, A, A, 8, 64, 8192, A, N0) == 2 and "160 KiB" in msg(L)
     assert L.qmv_mx(2, N0, 2, N0, N0, 1, 0, 256, N0, N0) == 0  # empty output
     assert L.qmv_mx(2, A, 2, A, A, 1, 64, 256, A, N0) not in (0, 1, 2)  # needs a device
+
+
+def test_gather_staged_workspace_size(L):
+    """The staged workspace holds the routing workspace, 256-byte aligned,
+    then a bf16 copy of every routed x row (T*topk rows of K elements)."""
+    for T, topk, E, K in [(4096, 8, 64, 2048), (17, 3, 5, 192), (1, 1, 1, 64), (0, 2, 4, 128)]:
+        base = L.gather_qmm_workspace_size(T, topk, E)
+        staged = L.gather_qmm_staged_workspace_size(T, topk, E, K)
+        assert staged == ((base + 255) // 256) * 256 + T * topk * K * 2
+    for bad in [(-1, 2, 4, 64), (16, 0, 4, 64), (16, 2, 0, 64), (16, 2, 1025, 64), (16, 2, 4, -64),
+                (16, 2, 4, (1 << 30) + 64), (1 << 62, 4, 4, 64)]:
+        assert L.gather_qmm_staged_workspace_size(*bad) == 0

@@ -45,9 +45,13 @@ def oracle_operands(orc, w, g):
 @pytest.mark.parametrize("T,topk,E,N,K", [(64, 2, 4, 128, 256), (200, 3, 7, 272, 192), (130, 1, 3, 512, 2048),
                                           (300, 8, 16, 1408, 128)])
 @pytest.mark.parametrize("use_g", [True, False])
-def test_gather_qmm_parity(nv, orc, T, topk, E, N, K, use_g):
+@pytest.mark.parametrize("staged", [True, False])  # SM-pair kernel on staged rows / single-SM gathering kernel
+def test_gather_qmm_parity(nv, orc, T, topk, E, N, K, use_g, staged):
     x, w, idx, g, wc, ws = make_case(nv, T, topk, E, N, K, use_g, seed=T + E + N)
-    y = nv.gather_qmm(x.cuda(), wc, ws, g, idx.cuda())
+    size = (nv.gather_qmm_staged_workspace_size if staged else
+            lambda T, topk, E, K: nv.gather_qmm_workspace_size(T, topk, E))(T, topk, E, K)
+    work = torch.empty(size, dtype=torch.uint8, device="cuda")
+    y = nv.gather_qmm(x.cuda(), wc, ws, g, idx.cuda(), workspace=work)
     nv.check_device_errors()
     oc, os_, gs = oracle_operands(orc, w, g)
     assert np.array_equal(raw(wc).reshape(oc.shape), oc)
@@ -67,7 +71,8 @@ def test_gather_qmm_experts_without_tokens(nv, orc):
     check_gemm_output(raw(y), r, "bf16", orc)
 
 
-def test_gather_worked_example_bf16_before_the_sum(nv):
+@pytest.mark.parametrize("T", [3, 24])  # the decode kernel and the tensor-core kernel
+def test_gather_worked_example_bf16_before_the_sum(nv, T):
     """"[Metal] global scale for qmm": codes 6, block scale 0.5, decode factor
     0.1; the weight rounds to bf16 0.30078125 before the matmul, so x = ones
     with K = 192 gives 192 * 0.30078125 = 57.75 (scaling after the matmul
@@ -76,17 +81,18 @@ def test_gather_worked_example_bf16_before_the_sum(nv):
     wc = torch.full((E, N, K // 8), 0x77777777, dtype=torch.int32).cuda()
     ws = torch.full((E, N, K // 16), 0x30, dtype=torch.uint8).cuda()
     g = torch.tensor([268.8, 2688.0], dtype=torch.float32).cuda()
-    x = torch.ones(3, K, dtype=torch.bfloat16).cuda()
-    idx = torch.tensor([[0, 1], [1, 0], [0, 1]], dtype=torch.int32).cuda()
+    x = torch.ones(T, K, dtype=torch.bfloat16).cuda()
+    idx = torch.tensor([[t % 2, 1 - t % 2] for t in range(T)], dtype=torch.int32).cuda()
     y = nv.gather_qmm(x, wc, ws, g, idx).float().cpu()
-    for t in range(3):
+    for t in range(T):
         for j in range(2):
             want = 57.75 if idx[t, j].item() == 0 else 192 * 3.0
             assert torch.all(y[t, j] == want), (t, j, y[t, j, :4])
 
 
-def test_gather_out_of_range_expert_sets_error_and_zero_rows(nv):
-    T, topk, E, N, K = 8, 2, 4, 32, 64
+@pytest.mark.parametrize("T", [8, 40])  # the decode kernel and the tensor-core kernel
+def test_gather_out_of_range_expert_sets_error_and_zero_rows(nv, T):
+    topk, E, N, K = 2, 4, 32, 64
     x, w, idx, g, wc, ws = make_case(nv, T, topk, E, N, K, True, seed=4)
     idx = idx.clone()
     idx[3, 1] = E  # out of range
