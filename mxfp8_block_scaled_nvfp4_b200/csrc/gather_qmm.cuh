@@ -673,7 +673,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
 // bf16 weights, their stores, codes) per the same FLOPs on one SM.
 //
 // A pipeline stage covers 128 K (8 MMAs): the MMA warp waits on one
-// barrier and commits once per stage.  Measured with 64-K stages and
+// barrier and commits once per stage.  Four A stages fill the tensor
+// memory beside the accumulator; x has four shared-memory slots (an x
+// stage was measured to land 1.0-1.6 us after its load was issued).  Measured with 64-K stages and
 // separate x and A barriers, the MMA warp's own loop (three satisfied
 // waits of ~130 ns each, two commits, four MMAs) took ~0.7 us per stage
 // against 0.26 us of tensor-core work.
@@ -696,7 +698,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
 // barrier the forwarder acquired; the MMA that reads it is issued only
 // after the even CTA observes the arrive.  Two groups of dequantize warps
 // take alternate stages.  The epilogue warps of both CTAs arrive on the
-// even CTA's accumulator-empty barrier.  The even CTA's MMA warp issues
+// even CTA's accumulator-empty barrier, relaxed as well, after their last
+// tcgen05.ld of the accumulator has completed.  The even CTA's MMA warp issues
 // every MMA and its commits arrive on the barriers at the same offset in
 // both CTAs (multicast commit).  No TMA load uses cluster multicast.
 // Every wait is bounded; both CTAs reach the closing cluster barrier.
@@ -705,8 +708,9 @@ constexpr int P_CTA = 128;           // pairs of the tile in each CTA (its half 
 constexpr int W_CTA = 128;           // weight rows of the unit in each CTA (its half of A)
 constexpr int UNIT_N = 2 * W_CTA;    // output columns per unit
 constexpr int BKS = 128;             // K elements per pipeline stage
-constexpr int S = 3;                 // stages of x (shared memory) and A (tensor memory)
-constexpr int RS = 6;                // code stages
+constexpr int S = 4;                 // pipeline stages: barriers and A stages (tensor memory)
+constexpr int SX = 4;                // x slots (shared memory); step it uses slot it % SX
+constexpr int RS = 3;                // code stages
 constexpr int EPI_WARPS = 8;
 constexpr int DEQ_GROUP = 8;         // dequantize warps per stage (4 lane quarters x 2 K halves)
 constexpr int DEQ_WARPS = 2 * DEQ_GROUP;  // two groups, alternating stages
@@ -718,7 +722,7 @@ constexpr int R_STAGE = W_CTA * (BKS / 2);  // 8 KiB of codes
 constexpr int EPI_BLOCK = 32 * 64;   // 32 pairs x 32 weight rows of bf16
 constexpr int EPI_BUF = 4 * EPI_BLOCK;  // an epilogue warp's four blocks of a unit
 constexpr int SMEM_X = 0;
-constexpr int SMEM_R = SMEM_X + S * X_STAGE;
+constexpr int SMEM_R = SMEM_X + SX * X_STAGE;
 constexpr int SMEM_E = SMEM_R + RS * R_STAGE;
 constexpr int SMEM_BYTES = SMEM_E + EPI_WARPS * EPI_BUF;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
@@ -726,6 +730,7 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_A = 256;     // accumulator in columns 0-255, A stages after it
 constexpr uint32_t A_COLS = BKS / 2; // tensor-memory columns of an A stage (two bf16 per column)
 constexpr int PREFETCH = 4;          // stages of block scales each dequantize thread has in flight
+constexpr uint32_t X_AHEAD = 3;      // stages ahead of its loads that the x warp prefetches into L2
 static_assert(TMEM_A + S * A_COLS <= TMEM_COLS, "A stages exceed tensor memory");
 static_assert(SMEM_ALLOC <= 227 * 1024 - 8 * 1024, "shared memory");
 
@@ -742,9 +747,6 @@ __device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
   return r;
-}
-__device__ __forceinline__ void arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // Remote arrive without a release fence (see the forwarder).
 __device__ __forceinline__ void arrive_cluster_relaxed(uint32_t cluster_addr) {
@@ -800,6 +802,12 @@ __device__ __forceinline__ void tma_load_pair(uint32_t dst, const CUtensorMap* m
       "[%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
       : "memory");
+}
+// Prefetch of a 2-D box of the tensor into L2 (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
 }
 // 32 consecutive 32-bit columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
@@ -901,17 +909,33 @@ __global__ void __launch_bounds__(ts::THREADS, 1) k_gather_mma_ts(const __grid_c
     // two 64 x 128 boxes of the staged rows per stage: tile rows 128 * rank
     // .. + 127; rows past the tile's end are other tiles' rows or past the
     // staged rows (zero fill), K past the end is zero fill, and nothing of
-    // either reaches a stored output
+    // either reaches a stored output.  The boxes of the stage X_AHEAD steps
+    // later are prefetched into L2 when a stage is loaded (measured: a stage
+    // took 1.2-1.6 us from load to landing, longer than the three x slots
+    // cover at the tensor-core rate).
     const bool leader = elect_one();
     uint32_t it = 0;
     bool ok = true;
+    auto row_of = [&](uint32_t uu) {
+      return a.ws.tile_row0[uu / (uint32_t)a.n_tiles_n] + ts::P_CTA * (int)rank;
+    };
+    int xrow_next = pair + npairs < units ? row_of(pair + npairs) : 0;
     for (uint32_t u = pair; u < units && ok; u += npairs) {
-      uint32_t tile, n0;
-      unit_coords(u, (uint32_t)a.n_tiles_n, tile, n0);
-      const int xrow = a.ws.tile_row0[tile] + ts::P_CTA * (int)rank;
+      const int xrow = u == pair ? row_of(u) : xrow_next;
+      if (u != pair) xrow_next = u + npairs < units ? row_of(u + npairs) : 0;
+      if (u == pair && leader)
+        for (uint32_t kp = 0; kp < ts::X_AHEAD && kp < kb_count; ++kp) {  // the first stages
+          ts::tma_prefetch_l2(&tmap_x, (int)(kp * ts::BKS), xrow);
+          ts::tma_prefetch_l2(&tmap_x, (int)(kp * ts::BKS + 64u), xrow);
+        }
       for (uint32_t kb = 0; kb < kb_count; ++kb, ++it) {
         const uint32_t s = it % ts::S;
-        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&empty[s]), ((it / ts::S) & 1u) ^ 1u)) ||
+        // slot it % SX is free once the MMAs of step it - SX have completed
+        // (their commit is that step's phase of its empty barrier; step it + 1,
+        // the next phase of the same barrier, cannot complete before this load)
+        const uint32_t prev = it - ts::SX;
+        if (!__all_sync(0xffffffffu,
+                        it < (uint32_t)ts::SX || mbar_wait(smem_u32(&empty[prev % ts::S]), (prev / ts::S) & 1u)) ||
             *(volatile int*)&abort_flag) {
           ok = false;
           break;
@@ -919,9 +943,17 @@ __global__ void __launch_bounds__(ts::THREADS, 1) k_gather_mma_ts(const __grid_c
         if (leader) {
           const uint32_t bar = ts::peer_addr(smem_u32(&full[s]), 0);
           if (lead) mbar_expect_tx(smem_u32(&full[s]), 2u * ts::X_STAGE);  // both CTAs' boxes
-          const uint32_t dst = sbase + ts::SMEM_X + s * ts::X_STAGE;
+          const uint32_t dst = sbase + ts::SMEM_X + (it % ts::SX) * ts::X_STAGE;
           ts::tma_load_pair(dst, &tmap_x, (int)(kb * ts::BKS), xrow, bar);
           ts::tma_load_pair(dst + ts::X_BOX, &tmap_x, (int)(kb * ts::BKS + 64u), xrow, bar);
+          const uint32_t kp = kb + ts::X_AHEAD;  // the stage X_AHEAD steps later
+          if (kp < kb_count) {
+            ts::tma_prefetch_l2(&tmap_x, (int)(kp * ts::BKS), xrow);
+            ts::tma_prefetch_l2(&tmap_x, (int)(kp * ts::BKS + 64u), xrow);
+          } else if (u + npairs < units && kp - kb_count < kb_count) {
+            ts::tma_prefetch_l2(&tmap_x, (int)((kp - kb_count) * ts::BKS), xrow_next);
+            ts::tma_prefetch_l2(&tmap_x, (int)((kp - kb_count) * ts::BKS + 64u), xrow_next);
+          }
         }
         __syncwarp();
       }
@@ -980,7 +1012,7 @@ __global__ void __launch_bounds__(ts::THREADS, 1) k_gather_mma_ts(const __grid_c
         }
         tc_fence_after();
         if (leader) {
-          const uint32_t xl = (uint32_t)x_base + s * (ts::X_STAGE >> 4);
+          const uint32_t xl = (uint32_t)x_base + (it % ts::SX) * (ts::X_STAGE >> 4);
           const uint32_t at = tmem + ts::TMEM_A + ts::A_COLS * s;
           const uint32_t nk = min(8u, ((uint32_t)a.K - kb * ts::BKS) / 16u);  // K = 16 slices of the stage
           for (uint32_t j = 0; j < nk; ++j)  // slice j: box j / 4, 32 bytes per slice inside it
@@ -1155,7 +1187,9 @@ __global__ void __launch_bounds__(ts::THREADS, 1) k_gather_mma_ts(const __grid_c
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) ts::arrive_cluster(empty_addr);  // the accumulator is free for the next unit
+      // the accumulator is free for the next unit: every tcgen05.ld of it has
+      // completed (tcgen05.wait::ld) before this relaxed arrive is issued
+      if (lane == 0) ts::arrive_cluster_relaxed(empty_addr);
       const uint32_t n = nw + 8u * ((uint32_t)lane & 3u);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
