@@ -64,8 +64,10 @@ L2_FLUSH_BYTES = 256 << 20
 # dominant kernel, from one ncu capture of that kernel as it is now (the
 # summaries under profiles/ give the commands and the other counters).
 NCU_TRAFFIC_BYTES = {
-    "gather_qmm (kn)": 127318528 + 56494080,    # profiles/gather_qmm_kn_moe_T4096_top8_E64_N1408_K2048.md
-    "k_nvfp4_quantize<SR>": 1120127232 + 319645184,  # profiles/quantize_sr_32768x16384.md
+    "qqmm_sm100 (nvfp4)": 18959872 + 134656,     # profiles/qqmm_nvfp4_4096x4096x4096.md
+    "k_qmv_tc": 33114880 + 0,                    # profiles/qmv_tc_gemv_14336x4096.md
+    "gather_qmm": 238368512 + 72332288,          # profiles/gather_qmm_moe_T4096_top8_E64_N1408_K2048.md (k_gather_mma_ts)
+    "k_gather_qmv": 43878400 + 6400,             # profiles/gather_qmv_decode_T4_top8_E64_N1408_K2048.md
 }
 
 

@@ -1324,7 +1324,7 @@ __device__ __forceinline__ void gqmv_rows(const uint32_t* __restrict__ wc, const
   }
 }
 
-// CTA (row block, tile): weight rows n0..n0+15 of the tile's expert against// CTA (row block, tile): weight rows n0..n0+15 of the tile's expert against
+// CTA (row block, tile): weight rows n0..n0+15 of the tile's expert against
 // every pair of the tile, kQmvPairs pairs per pass; x of those pairs in
 // shared memory as fp32 [kQmvPairs][K] in qmv's swizzled 32-element chunks
 // (xs_index): lane l reads chunk l, and the swizzle puts the 8 lanes of a
