@@ -67,7 +67,10 @@ NCU_TRAFFIC_BYTES = {
     "qqmm_sm100 (nvfp4)": 18959872 + 134656,     # profiles/qqmm_nvfp4_4096x4096x4096.md
     "k_qmv_tc": 33114880 + 0,                    # profiles/qmv_tc_gemv_14336x4096.md
     "gather_qmm": 238368512 + 72332288,          # profiles/gather_qmm_moe_T4096_top8_E64_N1408_K2048.md (k_gather_mma_ts)
-    "k_gather_qmv": 43878400 + 6400,             # profiles/gather_qmv_decode_T4_top8_E64_N1408_K2048.md
+    "gather_qmm (kn)": 127801600 + 56908544,     # profiles/gather_qmm_kn_moe_T4096_top8_E64_N1408_K2048.md
+    "qqmm_sm100 (mxfp4)": 103694592 + 103843584, # profiles/qqmm_mxfp4_8192x8192x8192.md
+    "k_nvfp4_quantize<SR>": 1136302336 + 326791168,  # profiles/quantize_sr_32768x16384.md
+    "k_nvfp4_quantize": 1082603008 + 288834048,  # profiles/quantize_nvfp4_32768x16384.md
 }
 
 

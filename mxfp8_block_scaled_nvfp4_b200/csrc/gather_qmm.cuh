@@ -1328,8 +1328,11 @@ __device__ __forceinline__ void gqmv_rows(const uint32_t* __restrict__ wc, const
 // every pair of the tile, kQmvPairs pairs per pass; x of those pairs in
 // shared memory as fp32 [kQmvPairs][K] in qmv's swizzled 32-element chunks
 // (xs_index): lane l reads chunk l, and the swizzle puts the 8 lanes of a
-// 128-bit load phase on distinct banks.
-__global__ void __launch_bounds__(QV_THREADS) k_gather_qmv(const __nv_bfloat16* __restrict__ x,
+// 128-bit load phase on distinct banks.  Three CTAs per SM (at most 80
+// registers a thread): 4 % faster on the 4-token MoE decode than the
+// unbounded 127 registers at two CTAs per SM; four (64 registers) spilled
+// and was slower.
+__global__ void __launch_bounds__(QV_THREADS, 3) k_gather_qmv(const __nv_bfloat16* __restrict__ x,
                                                            const uint32_t* __restrict__ wc, Args a) {
   extern __shared__ float xs[];  // [kQmvPairs][K]
   const int tile = blockIdx.y;
