@@ -1239,6 +1239,29 @@ __device__ __forceinline__ void ffma2(float& a0, float& a1, float w0, float w1, 
       : "f"(w0), "f"(w1), "f"(x0), "f"(x1));
 }
 
+// a0 += w.lo * x.lo, a1 += w.hi * x.hi for two bf16x2 words: fp32 fused
+// multiply-adds with bf16 operands (each product exact in fp32, one rounding
+// per add, as fmaf on the widened operands).
+__device__ __forceinline__ void bfma2(float& a0, float& a1, uint32_t w, uint32_t x) {
+  asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+      "mov.b32 {wl, wh}, %2;\n\t"
+      "mov.b32 {xl, xh}, %3;\n\t"
+      "fma.rn.f32.bf16 %0, wl, xl, %0;\n\t"
+      "fma.rn.f32.bf16 %1, wh, xh, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(w), "r"(x));
+}
+
+// Byte offset of the 8 bf16 of x starting at k (k % 8 == 0) in routed row q
+// of the decode kernel's shared memory: 64-byte chunks of 32 elements, the
+// four 16-byte segments of a chunk rotated by chunk / 2, so that the 8 lanes
+// of a 128-bit load phase (chunks c .. c+7, one segment) hit 8 distinct
+// 4-bank groups.
+__device__ __forceinline__ uint32_t xb_offset(uint32_t q, uint32_t K, uint32_t k) {
+  const uint32_t c = k >> 5, seg = (k >> 3) & 3u;
+  return q * K * 2u + c * 64u + ((seg ^ ((c >> 1) & 3u)) << 4);
+}
+
 // Weight row r (< QV_ROWS) of this CTA's block: lane l loads 128-bit code
 // chunks g*128 + 32i + l (i < 4) and their two scale bytes.
 __device__ __forceinline__ void gqmv_load(const uint32_t* __restrict__ wc, const Args& a, int e, int nr, uint32_t chunks,
@@ -1264,7 +1287,7 @@ __device__ __forceinline__ void gqmv_load(const uint32_t* __restrict__ wc, const
 // fused multiply-adds.  qb / sb hold the first unit's loads on entry; the
 // next unit's loads are issued before the current unit is computed.
 template <int NQ>
-__device__ __forceinline__ void gqmv_rows(const uint32_t* __restrict__ wc, const Args& a, const float* xs,
+__device__ __forceinline__ void gqmv_rows(const uint32_t* __restrict__ wc, const Args& a, const uint8_t* xs,
                                           const int* perm, int e, int nr, float d, uint32_t groups, uint32_t chunks,
                                           uint4 (&qb)[4], uint32_t (&sb)[4], int& ur, uint32_t& ug) {
   const uint32_t lane = threadIdx.x & 31u;
@@ -1299,13 +1322,11 @@ __device__ __forceinline__ void gqmv_rows(const uint32_t* __restrict__ wc, const
           const uint32_t k0 = c * 32u + (uint32_t)h * 8u;
 #pragma unroll
           for (int q = 0; q < NQ; ++q) {
-            const float4 xa = *reinterpret_cast<const float4*>(xs + xs_index((uint32_t)q, K, k0));
-            const float4 xb = *reinterpret_cast<const float4*>(xs + xs_index((uint32_t)q, K, k0 + 4u));
-            const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              ffma2(acc[q][0], acc[q][1], __uint_as_float(pw[j] << 16), __uint_as_float(pw[j] & 0xFFFF0000u),
-                    xv[2 * j], xv[2 * j + 1]);
+            const uint4 xw = *reinterpret_cast<const uint4*>(xs + xb_offset((uint32_t)q, K, k0));
+            bfma2(acc[q][0], acc[q][1], pw[0], xw.x);
+            bfma2(acc[q][0], acc[q][1], pw[1], xw.y);
+            bfma2(acc[q][0], acc[q][1], pw[2], xw.z);
+            bfma2(acc[q][0], acc[q][1], pw[3], xw.w);
           }
         }
       }
@@ -1326,15 +1347,15 @@ __device__ __forceinline__ void gqmv_rows(const uint32_t* __restrict__ wc, const
 
 // CTA (row block, tile): weight rows n0..n0+15 of the tile's expert against
 // every pair of the tile, kQmvPairs pairs per pass; x of those pairs in
-// shared memory as fp32 [kQmvPairs][K] in qmv's swizzled 32-element chunks
-// (xs_index): lane l reads chunk l, and the swizzle puts the 8 lanes of a
-// 128-bit load phase on distinct banks.  Three CTAs per SM (at most 80
+// shared memory as bf16 [kQmvPairs][K] (xb_offset): lane l reads 16 bytes
+// of chunk l per 8 weights, and the swizzle puts the 8 lanes of a 128-bit
+// load phase on distinct banks.  Three CTAs per SM (at most 80
 // registers a thread): 4 % faster on the 4-token MoE decode than the
 // unbounded 127 registers at two CTAs per SM; four (64 registers) spilled
 // and was slower.
 __global__ void __launch_bounds__(QV_THREADS, 3) k_gather_qmv(const __nv_bfloat16* __restrict__ x,
                                                            const uint32_t* __restrict__ wc, Args a) {
-  extern __shared__ float xs[];  // [kQmvPairs][K]
+  extern __shared__ __align__(16) uint8_t xs[];  // [kQmvPairs][K] bf16 (xb_offset)
   const int tile = blockIdx.y;
   if (tile >= *a.ws.ntiles) return;  // uniform per CTA
   const int e = a.ws.tile_expert[tile], row0 = a.ws.tile_row0[tile], nrows = a.ws.tile_rows[tile];
@@ -1358,14 +1379,8 @@ __global__ void __launch_bounds__(QV_THREADS, 3) k_gather_qmv(const __nv_bfloat1
     for (int q = 0; q < nq; ++q) {
       const int tok = a.ws.perm[row0 + q0 + q] / a.topk;
       const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)tok * K);
-      for (int i = threadIdx.x; i < K / 8; i += blockDim.x) {
-        float v[8];
-        load8<__nv_bfloat16>(reinterpret_cast<const __nv_bfloat16*>(src + i), v);
-        *reinterpret_cast<float4*>(xs + xs_index((uint32_t)q, (uint32_t)K, (uint32_t)(i * 8))) =
-            make_float4(v[0], v[1], v[2], v[3]);
-        *reinterpret_cast<float4*>(xs + xs_index((uint32_t)q, (uint32_t)K, (uint32_t)(i * 8 + 4))) =
-            make_float4(v[4], v[5], v[6], v[7]);
-      }
+      for (int i = threadIdx.x; i < K / 8; i += blockDim.x)
+        *reinterpret_cast<uint4*>(xs + xb_offset((uint32_t)q, (uint32_t)K, (uint32_t)(i * 8))) = __ldg(src + i);
     }
     __syncthreads();
     const int* perm = a.ws.perm + row0 + q0;
@@ -1452,7 +1467,7 @@ inline nvfp4_status gather_qmm_launch(const void* x, const uint32_t* w_codes, co
     k_route<<<1, ROUTE_THREADS, rsmem, stream>>>(idx, (int)P, (int)E, (int)N, ws, static_cast<__nv_bfloat16*>(y));
     err = cudaGetLastError();
   }
-  const size_t qv_smem = (size_t)kQmvPairs * (size_t)K * sizeof(float);
+  const size_t qv_smem = (size_t)kQmvPairs * (size_t)K * sizeof(__nv_bfloat16);  // x rows as bf16
   if (err == cudaSuccess && decode) {
     // decode: gather_qmv
     err = cudaFuncSetAttribute(k_gather_qmv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qv_smem);
