@@ -1226,19 +1226,6 @@ constexpr int kQmvPairs = 4;     // routed x rows per pass
 constexpr int QV_THREADS = 256;
 constexpr int QV_ROWS = 16;      // weight rows per CTA (2 per warp)
 
-// a0 += w0 * x0, a1 += w1 * x1 (one packed fp32x2 fused multiply-add,
-// each lane rounded as fmaf rounds).
-__device__ __forceinline__ void ffma2(float& a0, float& a1, float w0, float w1, float x0, float x1) {
-  asm("{\n\t.reg .b64 acc, w, x;\n\t"
-      "mov.b64 acc, {%0, %1};\n\t"
-      "mov.b64 w, {%2, %3};\n\t"
-      "mov.b64 x, {%4, %5};\n\t"
-      "fma.rn.f32x2 acc, w, x, acc;\n\t"
-      "mov.b64 {%0, %1}, acc;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "f"(w0), "f"(w1), "f"(x0), "f"(x1));
-}
-
 // a0 += w.lo * x.lo, a1 += w.hi * x.hi for two bf16x2 words: fp32 fused
 // multiply-adds with bf16 operands (each product exact in fp32, one rounding
 // per add, as fmaf on the widened operands).
