@@ -71,6 +71,7 @@ NCU_TRAFFIC_BYTES = {
     "qqmm_sm100 (mxfp4)": 103694592 + 103843584, # profiles/qqmm_mxfp4_8192x8192x8192.md
     "k_nvfp4_quantize<SR>": 1136302336 + 326791168,  # profiles/quantize_sr_32768x16384.md
     "k_nvfp4_quantize": 1082603008 + 288834048,  # profiles/quantize_nvfp4_32768x16384.md
+    "k_gather_qmv": 43878656 + 4864,               # profiles/gather_qmv_decode_T4_top8_E64_N1408_K2048.md
 }
 
 
