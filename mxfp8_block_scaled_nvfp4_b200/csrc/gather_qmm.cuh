@@ -6,13 +6,16 @@
 //   y[t, j, :] = x[t, :] . w_hat_e^T,   e = idx[t, j]
 //   w_hat_e[n, k] = bf16( e2m1(q) * fp32(f8(s) * (g[e] / 2688)) )
 //
-// Two kernels:
+// Kernels:
 //  1. k_route (one CTA): histogram of the T*topk (token, slot) pairs by
 //     expert, exclusive prefix sum, a list of 256-pair tiles (expert, first
 //     row of the expert's run, rows) and the permutation of pair ids grouped
 //     by expert.  Expert ids outside [0, E) set the device error word and
 //     their output rows are written as zeros.
-//  2. k_gather_mma, persistent (one CTA per SM): work units are (256-pair
+//  2. With a staged workspace and weights [E, N, K]: k_stage_x (the routed
+//     x rows copied once, grouped by expert) and k_gather_mma_ts, the SM-pair
+//     kernel with the dequantized weights in tensor memory (section 2b).
+//  3. Otherwise k_gather_mma, persistent (one CTA per SM): work units are (256-pair
 //     tile, 256 output columns), handed out round-robin, the column tiles of
 //     a pair tile adjacent so that CTAs running together share x rows and the
 //     expert's weight in L2.  Each dequantized weight stage feeds the MMAs of
@@ -42,7 +45,7 @@
 // instead streams each routed expert's weight rows once per tile of pairs:
 // a warp per weight row, 128-bit coalesced code loads, the same bf16
 // rounding of the dequantized weight as above, fp32 dot products with up to
-// kQmvPairs routed x rows held in shared memory at a time.
+// kQmvPairs routed x rows held in shared memory (as bf16) at a time.
 #pragma once
 
 #include <cuda.h>
@@ -673,12 +676,12 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
 // bf16 weights, their stores, codes) per the same FLOPs on one SM.
 //
 // A pipeline stage covers 128 K (8 MMAs): the MMA warp waits on one
-// barrier and commits once per stage.  Four A stages fill the tensor
-// memory beside the accumulator; x has four shared-memory slots (an x
-// stage was measured to land 1.0-1.6 us after its load was issued).  Measured with 64-K stages and
+// barrier and commits once per stage.  Measured with 64-K stages and
 // separate x and A barriers, the MMA warp's own loop (three satisfied
 // waits of ~130 ns each, two commits, four MMAs) took ~0.7 us per stage
-// against 0.26 us of tensor-core work.
+// against 0.26 us of tensor-core work.  Four A stages fill the tensor
+// memory beside the accumulator; x has four shared-memory slots (an x
+// stage was measured to land 1.0-1.6 us after its load was issued).
 //
 // The accumulator (fp32, 256 columns) holds weight rows on TMEM lanes and
 // pairs on columns; the epilogue transposes 32 x 32 blocks through shared
@@ -699,10 +702,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_gather_mma(const __grid_constant
 // after the even CTA observes the arrive.  Two groups of dequantize warps
 // take alternate stages.  The epilogue warps of both CTAs arrive on the
 // even CTA's accumulator-empty barrier, relaxed as well, after their last
-// tcgen05.ld of the accumulator has completed.  The even CTA's MMA warp issues
-// every MMA and its commits arrive on the barriers at the same offset in
-// both CTAs (multicast commit).  No TMA load uses cluster multicast.
-// Every wait is bounded; both CTAs reach the closing cluster barrier.
+// tcgen05.ld of the accumulator has completed.  The even CTA's MMA warp
+// issues every MMA and its commits arrive on the barriers at the same
+// offset in both CTAs (multicast commit).  No TMA load uses cluster
+// multicast.  Every wait is bounded; both CTAs reach the closing cluster
+// barrier.
 namespace ts {
 constexpr int P_CTA = 128;           // pairs of the tile in each CTA (its half of B)
 constexpr int W_CTA = 128;           // weight rows of the unit in each CTA (its half of A)
